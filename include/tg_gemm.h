@@ -1,0 +1,208 @@
+/*
+ * tg_gemm.h -- C ABI of the B200 (sm_100a) fused fp16 tensor-core GEMM.
+ *
+ * Operation (all entry points):
+ *
+ *     C[i][j] = g( sum_k A[i][k] * B[k][j]  +  beta[j] )      (fp32 accumulate)
+ *
+ *   A is M x K, B is K x N, C is M x N, all fp16 (IEEE binary16), dense and
+ *   row-major (leading dimensions K, N and N elements).  Products are formed
+ *   from the fp16 inputs and summed in fp32; the epilogue runs on the fp32
+ *   accumulator and the result is rounded once to fp16 (nearest, ties to
+ *   even) and stored.
+ *   Definition: "Designing High-Performance GPU Kernels with TileLang"
+ *   (thecryptopost.io), the make_matmul kernel and its 2048^3 benchmark
+ *   section: float16 A (M,K), B (K,N), C (M,N) with a "float" accumulator
+ *   fragment.
+ *
+ *   beta[j] = bias[j] (converted to fp32) for TG_EPILOGUE_BIAS and
+ *   TG_EPILOGUE_BIAS_GELU, 0 for TG_EPILOGUE_NONE.  bias == NULL means a zero
+ *   bias.  g is the identity, except for TG_EPILOGUE_BIAS_GELU where
+ *   g(v) = v * Phi(v) = 0.5 * v * (1 + erf(v / sqrt(2))) (the erf form of
+ *   GELU).  Definition: the same tutorial (ainovat.com), fused-epilogue
+ *   section: bias add and GELU applied to the register-resident accumulator
+ *   before the single write of the output.
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers are DEVICE pointers on the current CUDA device (except where
+ *     an entry point says "host"); the caller owns every buffer.  The library
+ *     keeps no pointer after the call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous with respect to the host and never
+ *     synchronise the device, except tg_gemm_check_error.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     non-TG_OK status means nothing was launched (except TG_ERR_LAUNCH /
+ *     TG_ERR_CUDA, which report a CUDA runtime failure).  Nothing throws
+ *     across this ABI.
+ *   - M == 0 or N == 0: nothing to do, TG_OK.  K == 0: C = g(beta).
+ *   - Each of M, N, K must be below 2^31 and the number of 128 x 64 output
+ *     tiles below 2^31, else TG_ERR_INVALID_ARG.
+ *   - A, B, C, bias must be 2-byte aligned (TG_ERR_MISALIGNED otherwise).
+ *     Any 2-byte-aligned address and any K, N are accepted: when a row pitch
+ *     or base address is not a multiple of 16 bytes the operands are first
+ *     repacked into a padded temporary, a stream-ordered allocation on
+ *     `stream` from a memory pool private to the library (freed on `stream`
+ *     after the GEMM); TG_ERR_OOM if that allocation fails.
+ *   - C must not overlap A, B or bias (TG_ERR_INVALID_ARG).
+ *   - The device must be compute capability 10.0 (B200 class, sm_100a);
+ *     otherwise TG_ERR_UNSUPPORTED_DEVICE.  There is no CPU fallback.
+ *   - Device-side waits are bounded.  If one expires (it should not in a
+ *     correct run) the kernel records the fact in a per-device error word,
+ *     leaves C partly written and exits cleanly; tg_gemm_check_error reports
+ *     it as TG_ERR_TIMEOUT.
+ */
+#ifndef TG_GEMM_H
+#define TG_GEMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TG_EPILOGUE_NONE = 0,      /* C = A.B                      */
+    TG_EPILOGUE_BIAS = 1,      /* C = A.B + bias               */
+    TG_EPILOGUE_BIAS_GELU = 2  /* C = GELU_erf(A.B + bias)     */
+} tg_epilogue_t;
+
+typedef enum {
+    TG_OK = 0,
+    TG_ERR_INVALID_ARG = 1,        /* null pointer, bad size/epilogue, overlap  */
+    TG_ERR_MISALIGNED = 2,         /* a pointer is not 2-byte aligned           */
+    TG_ERR_UNSUPPORTED_DEVICE = 3, /* current device is not sm_100              */
+    TG_ERR_LAUNCH = 4,             /* a kernel launch failed                    */
+    TG_ERR_TIMEOUT = 5,            /* a device-side bounded wait expired        */
+    TG_ERR_OOM = 6,                /* a temporary could not be allocated        */
+    TG_ERR_CUDA = 7                /* another CUDA runtime error                */
+} tg_status_t;
+
+/*
+ * tg_gemm -- C = g(A.B + beta) as defined above, on `stream`.
+ *
+ *   A     device, fp16 [M, K] row-major (leading dimension K), read only
+ *   B     device, fp16 [K, N] row-major (leading dimension N), read only
+ *   bias  device, fp16 [N], or NULL; read only; ignored for TG_EPILOGUE_NONE
+ *   C     device, fp16 [M, N] row-major (leading dimension N), written
+ *   epilogue  one of tg_epilogue_t
+ *   stream    cudaStream_t or NULL
+ *
+ * The tile configuration (tile width, pipeline depth, CTA pairing,
+ * rasterisation) comes from a per-shape table built by an offline sweep;
+ * see tg_gemm_select_config.  Results are deterministic: the same inputs and
+ * configuration give bit-identical C.
+ */
+tg_status_t tg_gemm(const void *A, const void *B, const void *bias, void *C,
+                    int64_t M, int64_t N, int64_t K, int epilogue, void *stream);
+
+/*
+ * Tile configuration descriptor (read-only view of one table entry).
+ *   id         index in [0, tg_num_configs())
+ *   block_m    output rows per MMA tile (128 per CTA; 256 with a CTA pair)
+ *   block_n    output columns per MMA tile (64, 128 or 256)
+ *   block_k    K elements per pipeline stage (64)
+ *   stages     depth of the shared-memory operand ring
+ *   cta_pair   1 if two CTAs of a cluster share one 2-SM MMA (cta_group::2)
+ *   group_m    M-tiles per rasterisation panel (L2 reuse)
+ *   epi_warps  warps that drain the accumulator
+ */
+typedef struct {
+    int id;
+    int block_m;
+    int block_n;
+    int block_k;
+    int stages;
+    int cta_pair;
+    int group_m;
+    int epi_warps;
+} tg_config_t;
+
+/* Number of compiled tile configurations. */
+int tg_num_configs(void);
+
+/* Describe configuration `id`.  Host only, no device call.
+ * TG_ERR_INVALID_ARG for a bad id or a NULL `out`. */
+tg_status_t tg_config_info(int id, tg_config_t *out);
+
+/*
+ * The configuration tg_gemm would use for this problem (host only, no device
+ * call; `num_sms` is the device's SM count, 148 on B200).  The choice comes
+ * from the compiled per-shape table (an offline sweep's winners) and falls
+ * back to a size rule for shapes the table does not list.
+ */
+tg_status_t tg_gemm_select_config(int64_t M, int64_t N, int64_t K, int epilogue,
+                                  int num_sms, tg_config_t *out);
+
+/*
+ * tg_gemm_ex -- tg_gemm with explicit options.  `opts` may be NULL (same as
+ * tg_gemm).  Used by the offline sweep and the tests.
+ *
+ *   config_id      -1: table choice; otherwise a configuration id
+ *   wait_limit_ns  0: default (2 s); else the limit of every device-side wait
+ *   inject         0 normally.  TG_INJECT_SKIP_FIRST_LOAD makes the first CTA
+ *                  skip one operand load, so that the consumer's bounded
+ *                  wait expires; for testing the timeout path only.  The
+ *                  kernel then exits cleanly and tg_gemm_check_error returns
+ *                  TG_ERR_TIMEOUT.
+ */
+#define TG_INJECT_SKIP_FIRST_LOAD 1
+typedef struct {
+    int config_id;
+    uint64_t wait_limit_ns;
+    int inject;
+} tg_options_t;
+
+tg_status_t tg_gemm_ex(const void *A, const void *B, const void *bias, void *C,
+                       int64_t M, int64_t N, int64_t K, int epilogue,
+                       const tg_options_t *opts, void *stream);
+
+/*
+ * tg_gemm_host -- the same GEMM on HOST buffers (end-to-end path).
+ *
+ *   A_host, B_host, bias_host (or NULL)  host fp16 inputs, row-major as above
+ *                                        (pinned memory gives async copies)
+ *   C_host                               host fp16 output [M, N]
+ *   workspace                            device buffer of at least
+ *                                        tg_gemm_host_workspace_size(M, N, K, has_bias)
+ *                                        bytes, 256-byte aligned; owned by the caller
+ *
+ * Enqueues on `stream`: host-to-device copies of the inputs into the
+ * workspace, tg_gemm, and the device-to-host copy of C.  Returns after
+ * enqueueing; synchronise `stream` before reading C_host.  Allocates nothing.
+ */
+size_t tg_gemm_host_workspace_size(int64_t M, int64_t N, int64_t K, int has_bias);
+
+tg_status_t tg_gemm_host(const void *A_host, const void *B_host, const void *bias_host,
+                         void *C_host, int64_t M, int64_t N, int64_t K, int epilogue,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * tg_gemm_launch_count -- number of kernels tg_gemm would launch for these
+ * arguments (host only, no device call): 0 for an empty problem, 1 for the
+ * GEMM kernel (or the K == 0 kernel), plus one repacking kernel for each of
+ * A and B whose base address or row pitch is not a multiple of 16 bytes.
+ * Returns -1 if the arguments would be rejected.
+ */
+int tg_gemm_launch_count(const void *A, const void *B, const void *bias, const void *C,
+                         int64_t M, int64_t N, int64_t K, int epilogue);
+
+/*
+ * tg_gemm_check_error -- synchronise `stream`, then read and clear the
+ * current device's error word.  TG_ERR_TIMEOUT if a bounded wait expired in
+ * any kernel since the last check, TG_ERR_CUDA if the stream reports a CUDA
+ * error, else TG_OK.
+ */
+tg_status_t tg_gemm_check_error(void *stream);
+
+/* Static, human-readable name of a status code (never NULL). */
+const char *tg_status_string(int status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int tg_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TG_GEMM_H */

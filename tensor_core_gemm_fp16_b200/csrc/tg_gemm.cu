@@ -1,0 +1,476 @@
+// tg_gemm.cu -- host side of the C ABI declared in include/tg_gemm.h:
+// argument validation, per-shape configuration choice, TMA tensor-map
+// encoding, operand repacking for unaligned pitches, and kernel launch.
+//
+// The operation is the tutorial's tiled fp16 tensor-core GEMM with an fp32
+// accumulator ("Designing High-Performance GPU Kernels with TileLang",
+// thecryptopost.io, make_matmul and the 2048^3 section) with the fused
+// bias + GELU epilogue of its fused-epilogue section (ainovat.com).  Its
+// schedule knobs (tile sizes, stages, L2 swizzle; the schedule-sweep
+// section) become the compiled configuration table below.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "tg_gemm.h"
+#include "tg_kernels.cuh"
+
+// Per-device error word: bounded-wait expiries are OR-ed in here.
+__device__ unsigned g_tg_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;   // 2 s
+
+// ------------------------------------------------------------------ configs
+using LaunchFn = cudaError_t (*)(const CUtensorMap &, const CUtensorMap &,
+                                 const tg::GemmParams &, int, cudaStream_t);
+
+template <int BN, int ST, int EPI, bool VEC>
+cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const tg::GemmParams &p,
+                        int grid, cudaStream_t stream)
+{
+    auto kern = tg::gemm_persistent_kernel<BN, ST, EPI, VEC>;
+    constexpr int smem = tg::SmemLayout<BN, ST>::kDynamicBytes;
+    static std::atomic<uint64_t> attr_set{0};   // one bit per device
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+    if (!bit || !(attr_set.load() & bit)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        attr_set.fetch_or(bit);
+    }
+    kern<<<grid, tg::kThreads, smem, stream>>>(ta, tb, p);
+    return cudaGetLastError();
+}
+
+struct KernelConfig {
+    tg_config_t info;
+    LaunchFn fn[3][2];   // [epilogue][vectorised C]
+};
+
+#define TG_FNS(BN, ST)                                                                      \
+    {                                                                                       \
+        {launch_gemm<BN, ST, 0, false>, launch_gemm<BN, ST, 0, true>},                      \
+            {launch_gemm<BN, ST, 1, false>, launch_gemm<BN, ST, 1, true>},                  \
+            {launch_gemm<BN, ST, 2, false>, launch_gemm<BN, ST, 2, true>},                  \
+    }
+
+// {id, block_m, block_n, block_k, stages, cta_pair, group_m, epi_warps}
+const KernelConfig kConfigs[] = {
+    {{0, 128, 256, 64, 4, 0, 8, 4}, TG_FNS(256, 4)},
+    {{1, 128, 128, 64, 6, 0, 8, 4}, TG_FNS(128, 6)},
+    {{2, 128, 64, 64, 8, 0, 8, 4}, TG_FNS(64, 8)},
+    {{3, 128, 256, 64, 4, 0, 16, 4}, TG_FNS(256, 4)},
+    {{4, 128, 128, 64, 6, 0, 16, 4}, TG_FNS(128, 6)},
+    {{5, 128, 256, 64, 4, 0, 4, 4}, TG_FNS(256, 4)},
+};
+constexpr int kNumConfigs = sizeof(kConfigs) / sizeof(kConfigs[0]);
+
+struct TableRow {
+    int64_t M, N, K;
+    int epilogue;
+    int config;
+};
+#include "tg_configs.inc"
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Size rule for shapes missing from the table: minimise
+// waves(BN) * BN / efficiency(BN), i.e. the last wave's finishing time in
+// units of a 128 x BN tile, with wider tiles credited for their better
+// operand reuse.
+int rule_config(int64_t M, int64_t N, int num_sms)
+{
+    const int ids[3] = {0, 1, 2};
+    const double eff[3] = {1.0, 0.9, 0.75};
+    int best = 0;
+    double best_score = 0;
+    for (int t = 0; t < 3; ++t) {
+        const int bn = kConfigs[ids[t]].info.block_n;
+        const int64_t tiles = ceil_div(M, 128) * ceil_div(N, bn);
+        const double waves = static_cast<double>(ceil_div(tiles, num_sms > 0 ? num_sms : 148));
+        const double score = waves * bn / eff[t];
+        if (t == 0 || score < best_score - 1e-9) {
+            best = ids[t];
+            best_score = score;
+        }
+    }
+    return best;
+}
+
+int choose_config(int64_t M, int64_t N, int64_t K, int epilogue, int num_sms)
+{
+    for (const TableRow &r : kShapeTable)
+        if (r.M == M && r.N == N && r.K == K && (r.epilogue < 0 || r.epilogue == epilogue) &&
+            r.config >= 0 && r.config < kNumConfigs)
+            return r.config;
+    return rule_config(M, N, num_sms);
+}
+
+// ------------------------------------------------------------------ devices
+struct DeviceState {
+    bool init = false;
+    tg_status_t status = TG_OK;
+    int num_sms = 0;
+    unsigned *error_word = nullptr;
+    cudaMemPool_t pool = nullptr;
+};
+DeviceState g_devices[kMaxDevices];
+std::mutex g_mutex;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+tg_status_t device_state(DeviceState **out, int *dev_out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return TG_ERR_UNSUPPORTED_DEVICE;
+    }
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceState &d = g_devices[dev];
+    if (!d.init) {
+        d.init = true;
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            major != 10 || minor != 0) {
+            d.status = TG_ERR_UNSUPPORTED_DEVICE;
+        } else if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) !=
+                       cudaSuccess ||
+                   cudaGetSymbolAddress(reinterpret_cast<void **>(&d.error_word),
+                                        g_tg_error_word) != cudaSuccess) {
+            d.status = TG_ERR_CUDA;
+        } else {
+            // A private stream-ordered pool for repacking temporaries; it
+            // keeps freed memory for reuse instead of returning it at every
+            // synchronisation.
+            cudaMemPoolProps props;
+            std::memset(&props, 0, sizeof(props));
+            props.allocType = cudaMemAllocationTypePinned;
+            props.location.type = cudaMemLocationTypeDevice;
+            props.location.id = dev;
+            if (cudaMemPoolCreate(&d.pool, &props) != cudaSuccess) {
+                d.pool = nullptr;
+                d.status = TG_ERR_CUDA;
+            } else {
+                uint64_t keep = 1ull << 30;
+                cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep);
+            }
+        }
+        if (d.status == TG_OK && !g_encode) {
+            cudaDriverEntryPointQueryResult q;
+            void *fn = nullptr;
+            if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000,
+                                                 cudaEnableDefault, &q) != cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || !fn)
+                d.status = TG_ERR_CUDA;
+            else
+                g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+        cudaGetLastError();
+    }
+    *out = &d;
+    if (dev_out) *dev_out = dev;
+    return d.status;
+}
+
+bool encode_2d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t outer,
+               uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer)
+{
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {pitch_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool overlaps(const void *a, int64_t a_bytes, const void *b, int64_t b_bytes)
+{
+    if (!a || !b || a_bytes <= 0 || b_bytes <= 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + static_cast<uintptr_t>(b_bytes) && b0 < a0 + static_cast<uintptr_t>(a_bytes);
+}
+
+bool aligned(const void *p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
+
+constexpr int64_t kDimLimit = (1ll << 31) - 1;
+
+// Checks that need no device.
+tg_status_t validate(const void *A, const void *B, const void *bias, const void *C, int64_t M,
+                     int64_t N, int64_t K, int epilogue)
+{
+    if (epilogue < TG_EPILOGUE_NONE || epilogue > TG_EPILOGUE_BIAS_GELU) return TG_ERR_INVALID_ARG;
+    if (M < 0 || N < 0 || K < 0 || M > kDimLimit || N > kDimLimit || K > kDimLimit)
+        return TG_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return TG_OK;
+    if (!C || (K > 0 && (!A || !B))) return TG_ERR_INVALID_ARG;
+    if (!aligned(C, 2) || (A && !aligned(A, 2)) || (B && !aligned(B, 2)) ||
+        (bias && !aligned(bias, 2)))
+        return TG_ERR_MISALIGNED;
+    if (ceil_div(M, tg::kBlockM) * ceil_div(N, 64) > kDimLimit) return TG_ERR_INVALID_ARG;
+    const int64_t c_bytes = 2 * M * N;
+    if (overlaps(C, c_bytes, A, 2 * M * K) || overlaps(C, c_bytes, B, 2 * K * N) ||
+        (epilogue != TG_EPILOGUE_NONE && overlaps(C, c_bytes, bias, 2 * N)))
+        return TG_ERR_INVALID_ARG;
+    return TG_OK;
+}
+
+tg_status_t launch_k0(const void *bias, void *C, int64_t M, int64_t N, int epilogue,
+                      cudaStream_t stream, int num_sms)
+{
+    const int64_t total = M * N;
+    const int grid = static_cast<int>(std::min<int64_t>(ceil_div(total, 256), 8ll * num_sms));
+    const __half *b = static_cast<const __half *>(bias);
+    __half *c = static_cast<__half *>(C);
+    if (epilogue == TG_EPILOGUE_NONE)
+        tg::k0_epilogue_kernel<0><<<grid, 256, 0, stream>>>(b, c, M, N);
+    else if (epilogue == TG_EPILOGUE_BIAS)
+        tg::k0_epilogue_kernel<1><<<grid, 256, 0, stream>>>(b, c, M, N);
+    else
+        tg::k0_epilogue_kernel<2><<<grid, 256, 0, stream>>>(b, c, M, N);
+    return cudaGetLastError() == cudaSuccess ? TG_OK : TG_ERR_LAUNCH;
+}
+
+tg_status_t launch_pack(const void *src, int64_t rows, int64_t cols, void *dst, int64_t ld_dst,
+                        cudaStream_t stream, int num_sms)
+{
+    const int64_t groups = rows * (ld_dst / 8);
+    if (groups == 0) return TG_OK;
+    const int grid = static_cast<int>(std::min<int64_t>(ceil_div(groups, 256), 16ll * num_sms));
+    tg::pack_pad_kernel<<<grid, 256, 0, stream>>>(static_cast<const __half *>(src), rows, cols,
+                                                  static_cast<__half *>(dst), ld_dst);
+    return cudaGetLastError() == cudaSuccess ? TG_OK : TG_ERR_LAUNCH;
+}
+
+tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, int64_t M,
+                      int64_t N, int64_t K, int epilogue, const tg_options_t *opts,
+                      cudaStream_t stream)
+{
+    tg_status_t st = validate(A, B, bias, C, M, N, K, epilogue);
+    if (st != TG_OK || M == 0 || N == 0) return st;
+    if (opts && (opts->config_id < -1 || opts->config_id >= kNumConfigs)) return TG_ERR_INVALID_ARG;
+    if (opts && (opts->inject != 0 && opts->inject != TG_INJECT_SKIP_FIRST_LOAD))
+        return TG_ERR_INVALID_ARG;
+    DeviceState *dev = nullptr;
+    st = device_state(&dev, nullptr);
+    if (st != TG_OK) return st;
+    if (epilogue == TG_EPILOGUE_NONE) bias = nullptr;
+    if (K == 0) return launch_k0(bias, C, M, N, epilogue, stream, dev->num_sms);
+
+    const int cfg_id = (opts && opts->config_id >= 0)
+                           ? opts->config_id
+                           : choose_config(M, N, K, epilogue, dev->num_sms);
+    const KernelConfig &cfg = kConfigs[cfg_id];
+    const int bn = cfg.info.block_n;
+
+    // TMA needs 16-byte aligned bases and pitches; otherwise repack.
+    const bool a_direct = aligned(A, 16) && (K % 8 == 0);
+    const bool b_direct = aligned(B, 16) && (N % 8 == 0);
+    const bool vec = aligned(C, 16) && (N % 8 == 0) && (!bias || aligned(bias, 16));
+    const int64_t lda = a_direct ? K : (K + 7) / 8 * 8;
+    const int64_t ldb = b_direct ? N : (N + 7) / 8 * 8;
+    void *tmp = nullptr;
+    const void *Aeff = A, *Beff = B;
+    if (!a_direct || !b_direct) {
+        const size_t a_bytes = a_direct ? 0 : static_cast<size_t>(2 * M * lda);
+        const size_t a_pad = (a_bytes + 255) / 256 * 256;
+        const size_t b_bytes = b_direct ? 0 : static_cast<size_t>(2 * K * ldb);
+        if (cudaMallocFromPoolAsync(&tmp, a_pad + b_bytes, dev->pool, stream) != cudaSuccess) {
+            cudaGetLastError();
+            return TG_ERR_OOM;
+        }
+        if (!a_direct) {
+            st = launch_pack(A, M, K, tmp, lda, stream, dev->num_sms);
+            Aeff = tmp;
+        }
+        if (st == TG_OK && !b_direct) {
+            void *bdst = static_cast<char *>(tmp) + a_pad;
+            st = launch_pack(B, K, N, bdst, ldb, stream, dev->num_sms);
+            Beff = bdst;
+        }
+        if (st != TG_OK) {
+            cudaFreeAsync(tmp, stream);
+            return st;
+        }
+    }
+
+    CUtensorMap ta, tb;
+    if (!encode_2d(&ta, Aeff, K, M, 2 * lda, tg::kBlockK, tg::kBlockM) ||
+        !encode_2d(&tb, Beff, N, K, 2 * ldb, tg::kBChunkN, tg::kBlockK)) {
+        if (tmp) cudaFreeAsync(tmp, stream);
+        return TG_ERR_CUDA;
+    }
+
+    tg::GemmParams p;
+    p.bias = static_cast<const __half *>(bias);
+    p.C = static_cast<__half *>(C);
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.ldc = N;
+    p.num_m_tiles = static_cast<int>(ceil_div(M, tg::kBlockM));
+    p.num_n_tiles = static_cast<int>(ceil_div(N, bn));
+    p.num_k_blocks = static_cast<int>(ceil_div(K, tg::kBlockK));
+    p.num_tiles = p.num_m_tiles * p.num_n_tiles;
+    p.group_m = cfg.info.group_m;
+    p.inject = opts ? opts->inject : 0;
+    p.wait_limit_ns = (opts && opts->wait_limit_ns) ? opts->wait_limit_ns : kDefaultWaitLimitNs;
+    p.error_word = dev->error_word;
+    const int grid = static_cast<int>(std::min<int64_t>(p.num_tiles, dev->num_sms));
+
+    cudaError_t e = cfg.fn[epilogue][vec ? 1 : 0](ta, tb, p, grid, stream);
+    if (tmp) cudaFreeAsync(tmp, stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_LAUNCH;
+    }
+    return TG_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+}  // namespace
+
+extern "C" {
+
+tg_status_t tg_gemm(const void *A, const void *B, const void *bias, void *C, int64_t M, int64_t N,
+                    int64_t K, int epilogue, void *stream)
+{
+    return gemm_impl(A, B, bias, C, M, N, K, epilogue, nullptr,
+                     static_cast<cudaStream_t>(stream));
+}
+
+tg_status_t tg_gemm_ex(const void *A, const void *B, const void *bias, void *C, int64_t M,
+                       int64_t N, int64_t K, int epilogue, const tg_options_t *opts, void *stream)
+{
+    return gemm_impl(A, B, bias, C, M, N, K, epilogue, opts, static_cast<cudaStream_t>(stream));
+}
+
+int tg_num_configs(void) { return kNumConfigs; }
+
+tg_status_t tg_config_info(int id, tg_config_t *out)
+{
+    if (!out || id < 0 || id >= kNumConfigs) return TG_ERR_INVALID_ARG;
+    *out = kConfigs[id].info;
+    return TG_OK;
+}
+
+tg_status_t tg_gemm_select_config(int64_t M, int64_t N, int64_t K, int epilogue, int num_sms,
+                                  tg_config_t *out)
+{
+    if (!out || M < 0 || N < 0 || K < 0 || epilogue < TG_EPILOGUE_NONE ||
+        epilogue > TG_EPILOGUE_BIAS_GELU || num_sms <= 0)
+        return TG_ERR_INVALID_ARG;
+    *out = kConfigs[choose_config(M, N, K, epilogue, num_sms)].info;
+    return TG_OK;
+}
+
+size_t tg_gemm_host_workspace_size(int64_t M, int64_t N, int64_t K, int has_bias)
+{
+    if (M < 0 || N < 0 || K < 0) return 0;
+    return round256(2 * static_cast<size_t>(M * K)) + round256(2 * static_cast<size_t>(K * N)) +
+           round256(has_bias ? 2 * static_cast<size_t>(N) : 0) +
+           round256(2 * static_cast<size_t>(M * N));
+}
+
+tg_status_t tg_gemm_host(const void *A_host, const void *B_host, const void *bias_host,
+                         void *C_host, int64_t M, int64_t N, int64_t K, int epilogue,
+                         void *workspace, size_t workspace_bytes, void *stream)
+{
+    tg_status_t st = validate(A_host, B_host, bias_host, C_host, M, N, K, epilogue);
+    if (st != TG_OK || M == 0 || N == 0) return st;
+    const bool has_bias = bias_host != nullptr && epilogue != TG_EPILOGUE_NONE;
+    if (!workspace || !aligned(workspace, 256) ||
+        workspace_bytes < tg_gemm_host_workspace_size(M, N, K, has_bias ? 1 : 0))
+        return TG_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char *w = static_cast<char *>(workspace);
+    const size_t a_bytes = 2 * static_cast<size_t>(M * K), b_bytes = 2 * static_cast<size_t>(K * N);
+    const size_t bias_bytes = has_bias ? 2 * static_cast<size_t>(N) : 0;
+    const size_t c_bytes = 2 * static_cast<size_t>(M * N);
+    char *dA = w;
+    char *dB = dA + round256(a_bytes);
+    char *dbias = dB + round256(b_bytes);
+    char *dC = dbias + round256(bias_bytes);
+    if ((a_bytes && cudaMemcpyAsync(dA, A_host, a_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) ||
+        (b_bytes && cudaMemcpyAsync(dB, B_host, b_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) ||
+        (bias_bytes &&
+         cudaMemcpyAsync(dbias, bias_host, bias_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)) {
+        cudaGetLastError();
+        return TG_ERR_CUDA;
+    }
+    st = gemm_impl(dA, dB, has_bias ? dbias : nullptr, dC, M, N, K, epilogue, nullptr, s);
+    if (st != TG_OK) return st;
+    if (cudaMemcpyAsync(C_host, dC, c_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_CUDA;
+    }
+    return TG_OK;
+}
+
+int tg_gemm_launch_count(const void *A, const void *B, const void *bias, const void *C,
+                         int64_t M, int64_t N, int64_t K, int epilogue)
+{
+    if (validate(A, B, bias, C, M, N, K, epilogue) != TG_OK) return -1;
+    if (M == 0 || N == 0) return 0;
+    if (K == 0) return 1;
+    const bool a_direct = aligned(A, 16) && (K % 8 == 0);
+    const bool b_direct = aligned(B, 16) && (N % 8 == 0);
+    return 1 + (a_direct ? 0 : 1) + (b_direct ? 0 : 1);
+}
+
+tg_status_t tg_gemm_check_error(void *stream)
+{
+    DeviceState *dev = nullptr;
+    tg_status_t st = device_state(&dev, nullptr);
+    if (st != TG_OK) return st;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_CUDA;
+    }
+    unsigned word = 0;
+    if (cudaMemcpy(&word, dev->error_word, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_CUDA;
+    }
+    if (word) {
+        const unsigned zero = 0;
+        cudaMemcpy(dev->error_word, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+        return TG_ERR_TIMEOUT;
+    }
+    return TG_OK;
+}
+
+const char *tg_status_string(int status)
+{
+    switch (status) {
+    case TG_OK: return "TG_OK";
+    case TG_ERR_INVALID_ARG: return "TG_ERR_INVALID_ARG: invalid argument";
+    case TG_ERR_MISALIGNED: return "TG_ERR_MISALIGNED: pointer not 2-byte aligned";
+    case TG_ERR_UNSUPPORTED_DEVICE: return "TG_ERR_UNSUPPORTED_DEVICE: needs an sm_100 GPU";
+    case TG_ERR_LAUNCH: return "TG_ERR_LAUNCH: kernel launch failed";
+    case TG_ERR_TIMEOUT: return "TG_ERR_TIMEOUT: a device-side wait expired";
+    case TG_ERR_OOM: return "TG_ERR_OOM: temporary allocation failed";
+    case TG_ERR_CUDA: return "TG_ERR_CUDA: CUDA runtime error";
+    default: return "unknown tg_status_t";
+    }
+}
+
+int tg_version(void) { return 100; }
+
+}  // extern "C"

@@ -16,3 +16,13 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA B200 GPU and the built library")
+
+
+def pytest_sessionstart(session):
+    # The CUDA library and the oracle are built in-tree; (re)build them if a
+    # source is newer than the binary so that every test sees current code.
+    from tensor_core_gemm_fp16_b200 import build as tg_build
+    import oracle
+
+    tg_build.build()
+    oracle.build()

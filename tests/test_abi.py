@@ -1,0 +1,123 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments on the host before touching any
+device.  All pointers passed here are rejected by host-side validation, so
+nothing is ever launched."""
+import ctypes
+
+import pytest
+import torch
+
+from tensor_core_gemm_fp16_b200 import binding
+
+NONE, BIAS, GELU = 0, 1, 2
+
+
+def test_library_exports_every_header_symbol():
+    lib = binding.load()
+    names = binding.header_symbols()
+    assert "tg_gemm" in names and "tg_gemm_check_error" in names
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in tg_gemm.h but not exported"
+
+
+def test_status_strings():
+    for st in range(8):
+        s = binding.tg_status_string(st)
+        assert s.startswith("TG_")
+    assert "unknown" in binding.tg_status_string(99)
+
+
+def test_config_table_is_consistent():
+    n = binding.tg_num_configs()
+    assert n >= 3
+    ids = set()
+    for i in range(n):
+        c = binding.tg_config_info(i)
+        assert c["id"] == i
+        ids.add(i)
+        assert c["block_m"] == 128 * (2 if c["cta_pair"] else 1)
+        assert c["block_n"] in (64, 128, 256)
+        assert c["block_k"] == 64
+        assert 2 <= c["stages"] <= 12
+        assert c["group_m"] >= 1
+    with pytest.raises(binding.TgError):
+        binding.tg_config_info(n)
+    with pytest.raises(binding.TgError):
+        binding.tg_config_info(-1)
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 256, 256), (2048, 2048, 2048), (3000, 1537, 2050),
+                                   (8192, 8192, 8192), (1, 1, 1), (100000, 64, 64)])
+def test_select_config_is_host_only_and_valid(M, N, K):
+    c = binding.tg_gemm_select_config(M, N, K, GELU, 148)
+    assert 0 <= c["id"] < binding.tg_num_configs()
+
+
+def test_select_config_prefers_more_tiles_for_small_problems():
+    small = binding.tg_gemm_select_config(256, 256, 256, NONE, 148)
+    big = binding.tg_gemm_select_config(8192, 8192, 8192, GELU, 148)
+    assert small["block_n"] <= big["block_n"]
+
+
+def test_select_config_rejects_bad_args():
+    with pytest.raises(binding.TgError):
+        binding.tg_gemm_select_config(-1, 4, 4, NONE, 148)
+    with pytest.raises(binding.TgError):
+        binding.tg_gemm_select_config(4, 4, 4, 3, 148)
+    with pytest.raises(binding.TgError):
+        binding.tg_gemm_select_config(4, 4, 4, 0, 0)
+
+
+def test_host_validation_rejects_bad_calls_without_a_device():
+    g = binding.tg_gemm
+    # bad epilogue
+    assert g(0x1000, 0x2000, None, 0x30000, 4, 4, 4, 7, None) == binding.TG_ERR_INVALID_ARG
+    # negative and oversized dimensions
+    assert g(0x1000, 0x2000, None, 0x30000, -1, 4, 4, 0, None) == binding.TG_ERR_INVALID_ARG
+    assert g(0x1000, 0x2000, None, 0x30000, 4, 1 << 31, 4, 0, None) == binding.TG_ERR_INVALID_ARG
+    # null C / null A with K > 0
+    assert g(0x1000, 0x2000, None, None, 4, 4, 4, 0, None) == binding.TG_ERR_INVALID_ARG
+    assert g(None, 0x2000, None, 0x30000, 4, 4, 4, 0, None) == binding.TG_ERR_INVALID_ARG
+    # odd addresses
+    assert g(0x1001, 0x2000, None, 0x30000, 4, 4, 4, 0, None) == binding.TG_ERR_MISALIGNED
+    assert g(0x1000, 0x2000, 0x5001, 0x30000, 4, 4, 4, 1, None) == binding.TG_ERR_MISALIGNED
+    # C overlapping A, B or bias
+    assert g(0x10000, 0x20000, None, 0x10010, 4, 4, 4, 0, None) == binding.TG_ERR_INVALID_ARG
+    assert g(0x10000, 0x20000, None, 0x1FFF8, 4, 4, 4, 0, None) == binding.TG_ERR_INVALID_ARG
+    assert g(0x10000, 0x20000, 0x40004, 0x40000, 4, 4, 4, 1, None) == binding.TG_ERR_INVALID_ARG
+    # bad options
+    assert binding.tg_gemm_ex(0x1000, 0x2000, None, 0x30000, 4, 4, 4, 9) == binding.TG_ERR_INVALID_ARG
+
+
+def test_empty_problems_are_ok_without_a_device():
+    assert binding.tg_gemm(None, None, None, None, 0, 4, 4, 0, None) == binding.TG_OK
+    assert binding.tg_gemm(None, None, None, None, 4, 0, 4, 2, None) == binding.TG_OK
+
+
+def test_host_entry_validation():
+    lib = binding
+    need = lib.tg_gemm_host_workspace_size(10, 20, 30, True)
+    assert need == 768 + 1280 + 256 + 512   # 600, 1200, 40, 400 bytes, each rounded to 256
+    assert lib.tg_gemm_host_workspace_size(-1, 2, 3, False) == 0
+    # workspace too small / misaligned
+    assert lib.tg_gemm_host(0x1000, 0x20000, None, 0x40000, 10, 20, 30, 0, 0x100000, 10) == \
+        binding.TG_ERR_INVALID_ARG
+    assert lib.tg_gemm_host(0x1000, 0x20000, None, 0x40000, 10, 20, 30, 0, 0x100010, need) == \
+        binding.TG_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device answer")
+def test_valid_call_without_a_device_reports_unsupported_device():
+    # Passes host validation, then finds no sm_100 device: nothing runs.
+    st = binding.tg_gemm(0x100000, 0x200000, None, 0x300000, 4, 4, 4, 0, None)
+    assert st == binding.TG_ERR_UNSUPPORTED_DEVICE
+    assert binding.tg_gemm_check_error(None) == binding.TG_ERR_UNSUPPORTED_DEVICE
+
+
+def test_binding_checks_tensor_arguments():
+    a = torch.zeros(4, 4, dtype=torch.float32)
+    with pytest.raises(TypeError):
+        binding.gemm(a, a)
+    h = torch.zeros(4, 4, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        binding.gemm(h, h)          # not CUDA tensors

@@ -1,0 +1,275 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Every test here launches kernels on cuda:0 and is marked ``gpu``.  Inputs are
+the seeded synthetic workloads; expected values come only from ``oracle``.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import assert_bits_equal, assert_close, run_gpu, run_oracle
+from tensor_core_gemm_fp16_b200 import binding
+from tensor_core_gemm_fp16_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+NONE, BIAS, GELU = binding.TG_EPILOGUE_NONE, binding.TG_EPILOGUE_BIAS, binding.TG_EPILOGUE_BIAS_GELU
+CONFIG_IDS = list(range(binding.tg_num_configs()))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.init()
+    yield
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------- exact layouts
+
+@pytest.mark.parametrize("config_id", CONFIG_IDS)
+@pytest.mark.parametrize("M,N", [(128, 256), (300, 200), (257, 520)])
+def test_identity_left_bit_exact(config_id, M, N):
+    """A = I: C must equal B bit for bit (pins A/B layouts and descriptors)."""
+    K = M
+    _, B, _ = wl.make_inputs(1, N, K, seed=100 + M)
+    A = torch.eye(M, dtype=torch.float16)
+    C = run_gpu(A, B, None, NONE, config_id=config_id)
+    assert_bits_equal(C, wl.to_bits(B), f"I @ B cfg{config_id}")
+
+
+@pytest.mark.parametrize("config_id", CONFIG_IDS)
+@pytest.mark.parametrize("M,K", [(128, 64), (200, 136), (129, 264)])
+def test_identity_right_bit_exact(config_id, M, K):
+    A, _, _ = wl.make_inputs(M, 1, K, seed=200 + K)
+    B = torch.eye(K, dtype=torch.float16)
+    C = run_gpu(A, B, None, NONE, config_id=config_id)
+    assert_bits_equal(C, wl.to_bits(A), f"A @ I cfg{config_id}")
+
+
+@pytest.mark.parametrize("config_id", [0, 1, 2])
+def test_permutations_bit_exact(config_id):
+    M = K = 384
+    N = 328
+    _, B, _ = wl.make_inputs(1, N, K, seed=300)
+    p = wl.permutation(M, seed=301)
+    P = torch.zeros(M, K, dtype=torch.float16)
+    P[np.arange(M), p] = 1.0
+    C = run_gpu(P, B, None, NONE, config_id=config_id)
+    assert_bits_equal(C, wl.to_bits(B)[p], "P @ B")
+    A, _, _ = wl.make_inputs(200, 1, 264, seed=302)
+    q = wl.permutation(264, seed=303)
+    Q = torch.zeros(264, 264, dtype=torch.float16)
+    Q[q, np.arange(264)] = 1.0
+    C = run_gpu(A, Q, None, NONE, config_id=config_id)
+    assert_bits_equal(C, wl.to_bits(A)[:, q], "A @ Q")
+
+
+@pytest.mark.parametrize("config_id", CONFIG_IDS)
+def test_integer_inputs_bit_exact(config_id):
+    A, B, bias = wl.integer_inputs(333, 520, 1000, seed=400, lo=-1, hi=1, bias=True)
+    exp = oracle.gemm_int_exact(wl.to_bits(A), wl.to_bits(B))
+    assert_bits_equal(run_gpu(A, B, None, NONE, config_id=config_id), exp, "int NONE")
+    exp_b = oracle.gemm_int_exact(wl.to_bits(A), wl.to_bits(B), wl.to_bits(bias), oracle.EPI_BIAS)
+    assert_bits_equal(run_gpu(A, B, bias, BIAS, config_id=config_id), exp_b, "int BIAS")
+
+
+def test_integer_inputs_large_sums_round_like_the_oracle():
+    # {-2..2} with K = 4096: sums reach beyond 2048, where fp16 spacing is 2+
+    A, B, _ = wl.integer_inputs(256, 256, 4096, seed=401, lo=0, hi=2)
+    exp = oracle.gemm_int_exact(wl.to_bits(A), wl.to_bits(B))
+    assert_bits_equal(run_gpu(A, B, None, NONE), exp, "int large sums")
+
+
+def test_rank1_closed_form():
+    M, N, K = 256, 512, 1024
+    u = torch.tensor([2.0 ** (i % 9 - 6) for i in range(M)])
+    v = torch.tensor([(-1) ** j * 2.0 ** (j % 5 - 4) for j in range(N)])
+    A = u[:, None].expand(M, K).to(torch.float16).contiguous()
+    B = v[None, :].expand(K, N).to(torch.float16).contiguous()
+    exact = (K * torch.outer(u, v).double()).numpy()
+    C = run_gpu(A, B, None, NONE)
+    assert_bits_equal(C, exact.astype(np.float16).view(np.uint16), "rank-1")
+
+
+# ---------------------------------------------------------------- epilogue
+
+def test_gelu_epilogue_within_one_ulp():
+    """A = 0, so C = fp16(GELU(bias)); sweep bias over [-8, 8]."""
+    M, N, K = 128, 4096, 64
+    A = torch.zeros(M, K, dtype=torch.float16)
+    B = torch.zeros(K, N, dtype=torch.float16)
+    bias = torch.linspace(-8, 8, N).to(torch.float16)
+    C = run_gpu(A, B, bias, GELU)
+    ref = run_oracle(A, B, bias, oracle.EPI_BIAS_GELU)
+    exp_bits = oracle.double_to_half_rne(ref).astype(np.int32)
+    got_bits = wl.to_bits(C).astype(np.int32)
+    # fp16 bit patterns of same-sign values are monotone: ulp distance = |diff|
+    same_sign = (exp_bits & 0x8000) == (got_bits & 0x8000)
+    dist = np.where(same_sign, np.abs(exp_bits - got_bits),
+                    (exp_bits & 0x7FFF) + (got_bits & 0x7FFF))
+    assert dist.max() <= 1, f"max ulp distance {dist.max()}"
+    assert_close(C, ref, "gelu sweep")
+
+
+def test_bias_epilogue_exact_when_representable():
+    M, N, K = 200, 300, 128
+    A, B, _ = wl.integer_inputs(M, N, K, seed=500, lo=-1, hi=1)
+    bias = torch.arange(N, dtype=torch.float32).remainder(17).sub(8).to(torch.float16)
+    exp = oracle.gemm_int_exact(wl.to_bits(A), wl.to_bits(B), wl.to_bits(bias), oracle.EPI_BIAS)
+    assert_bits_equal(run_gpu(A, B, bias, BIAS), exp, "bias exact")
+
+
+def test_gelu_without_bias_is_gelu_of_product():
+    A, B, _ = wl.make_inputs(192, 320, 256, seed=501)
+    C = run_gpu(A, B, None, GELU)
+    assert_close(C, run_oracle(A, B, None, oracle.EPI_BIAS_GELU), "gelu no bias")
+
+
+def test_none_epilogue_ignores_bias():
+    A, B, bias = wl.make_inputs(130, 136, 200, seed=502, bias=True)
+    c1 = run_gpu(A, B, bias, NONE)
+    c2 = run_gpu(A, B, None, NONE)
+    assert torch.equal(c1, c2)
+
+
+# ---------------------------------------------------------------- shapes
+
+RAGGED = [(1, 1, 1), (1, 8, 8), (7, 9, 13), (63, 65, 64), (64, 64, 65), (65, 63, 127),
+          (127, 129, 128), (128, 128, 129), (129, 257, 255), (255, 255, 257), (300, 1, 70),
+          (1, 300, 300), (17, 31, 1), (256, 264, 72)]
+
+
+@pytest.mark.parametrize("M,N,K", RAGGED)
+@pytest.mark.parametrize("epilogue", [NONE, GELU])
+def test_ragged_shapes(M, N, K, epilogue):
+    A, B, bias = wl.make_inputs(M, N, K, seed=M * 7919 + N * 31 + K, bias=True)
+    C = run_gpu(A, B, bias, epilogue)
+    assert_close(C, run_oracle(A, B, bias, epilogue), f"{M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("config_id", CONFIG_IDS)
+def test_every_config_multi_tile_ragged(config_id):
+    A, B, bias = wl.make_inputs(517, 777, 333, seed=600, dist="uniform", bias=True)
+    C = run_gpu(A, B, bias, GELU, config_id=config_id)
+    assert_close(C, run_oracle(A, B, bias, GELU), f"cfg{config_id}")
+
+
+def test_k_zero_gives_epilogue_of_bias():
+    M, N = 70, 90
+    bias = torch.linspace(-3, 3, N).to(torch.float16)
+    A = torch.zeros(M, 0, dtype=torch.float16)
+    B = torch.zeros(0, N, dtype=torch.float16)
+    for epi in (NONE, BIAS, GELU):
+        C = run_gpu(A, B, bias, epi)
+        assert_close(C, run_oracle(A, B, bias, epi), f"K=0 epi{epi}")
+
+
+def test_empty_m_or_n_is_a_no_op():
+    dev = torch.device("cuda:0")
+    for (M, N, K) in [(0, 5, 7), (5, 0, 7), (0, 0, 0)]:
+        a = torch.zeros(M, K, dtype=torch.float16, device=dev)
+        b = torch.zeros(K, N, dtype=torch.float16, device=dev)
+        c = binding.gemm(a, b)
+        assert c.shape == (M, N)
+
+
+def test_misaligned_operands_use_the_repacking_path():
+    """Views one element off a 16-byte boundary for A, B, bias and C."""
+    dev = torch.device("cuda:0")
+    M, N, K = 300, 260, 200
+    A, B, bias = wl.make_inputs(M, N, K, seed=700, bias=True)
+    a_buf = torch.zeros(M * K + 1, dtype=torch.float16, device=dev)
+    b_buf = torch.zeros(K * N + 1, dtype=torch.float16, device=dev)
+    bias_buf = torch.zeros(N + 1, dtype=torch.float16, device=dev)
+    c_buf = torch.zeros(M * N + 1, dtype=torch.float16, device=dev)
+    a = a_buf[1:].view(M, K)
+    b = b_buf[1:].view(K, N)
+    bb = bias_buf[1:]
+    c = c_buf[1:].view(M, N)
+    a.copy_(A.to(dev))
+    b.copy_(B.to(dev))
+    bb.copy_(bias.to(dev))
+    binding.gemm(a, b, bb, epilogue=GELU, out=c)
+    torch.cuda.synchronize()
+    assert c_buf[0].item() == 0.0, "wrote before C"
+    assert_close(c.cpu(), run_oracle(A, B, bias, GELU), "misaligned views")
+
+
+# ---------------------------------------------------------------- the workloads
+
+@pytest.mark.parametrize("name", ["gemm_256", "gemm_2048", "fused_2048", "ragged_fused"])
+def test_workload_full_parity(name):
+    w = wl.WORKLOADS[name]
+    A, B, bias = wl.workload_inputs(w)
+    C = run_gpu(A, B, bias, w.epilogue)
+    assert_close(C, run_oracle(A, B, bias, w.epilogue), name)
+
+
+def _sample_rows(M, n, seed):
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, 127, 128, 255, M // 2, M - 129, M - 128, M - 2, M - 1]
+    rnd = rng.choice(M, size=n, replace=False)
+    return sorted(set(int(r) for r in fixed + list(rnd) if 0 <= r < M))
+
+
+@pytest.mark.parametrize("name", ["fused_8192", "fused_8192_literal"])
+def test_large_workload_sampled_rows(name):
+    """Full-size 8192^3 launch (the benchmark's configuration); every column
+    of ~40 sampled rows against the oracle, plus whole-output sanity."""
+    w = wl.WORKLOADS[name]
+    A, B, bias = wl.workload_inputs(w)
+    C = run_gpu(A, B, bias, w.epilogue)
+    rows = _sample_rows(w.M, 30, seed=w.seed)
+    ref = run_oracle(A, B, bias, w.epilogue, rows=rows)
+    assert_close(C[rows], ref, f"{name} sampled rows")
+    assert torch.isfinite(C.float()).all()
+
+
+def test_deterministic():
+    A, B, bias = wl.make_inputs(1000, 1100, 900, seed=800, bias=True)
+    c1 = run_gpu(A, B, bias, GELU)
+    c2 = run_gpu(A, B, bias, GELU)
+    assert torch.equal(c1, c2)
+
+
+# ---------------------------------------------------------------- host entry, errors
+
+def test_host_entry_matches_device_entry():
+    A, B, bias = wl.make_inputs(520, 333, 264, seed=900, bias=True)
+    c_host = binding.gemm_host(A.pin_memory(), B.pin_memory(), bias.pin_memory(), epilogue=GELU)
+    c_dev = run_gpu(A, B, bias, GELU)
+    assert torch.equal(c_host, c_dev)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A skipped operand load makes the consumer's bounded wait expire: the
+    kernel exits cleanly, the host reads TG_ERR_TIMEOUT, and the next call
+    works."""
+    dev = torch.device("cuda:0")
+    A, B, bias = wl.make_inputs(256, 512, 512, seed=1000, bias=True)
+    a, b, bb = A.to(dev), B.to(dev), bias.to(dev)
+    c = torch.empty(256, 512, dtype=torch.float16, device=dev)
+    stream = torch.cuda.current_stream().cuda_stream
+    assert binding.tg_gemm_check_error(stream) == binding.TG_OK
+    st = binding.tg_gemm_ex(a.data_ptr(), b.data_ptr(), bb.data_ptr(), c.data_ptr(), 256, 512, 512,
+                            GELU, wait_limit_ns=50_000_000,
+                            inject=binding.TG_INJECT_SKIP_FIRST_LOAD, stream=stream)
+    assert st == binding.TG_OK
+    assert binding.tg_gemm_check_error(stream) == binding.TG_ERR_TIMEOUT
+    assert binding.tg_gemm_check_error(stream) == binding.TG_OK      # cleared
+    C = run_gpu(A, B, bias, GELU)
+    assert_close(C, run_oracle(A, B, bias, GELU), "after timeout")
+
+
+def test_invalid_arguments_on_device():
+    dev = torch.device("cuda:0")
+    a = torch.zeros(64, 64, dtype=torch.float16, device=dev)
+    stream = torch.cuda.current_stream().cuda_stream
+    # C overlapping A
+    st = binding.tg_gemm(a.data_ptr(), a.data_ptr(), None, a.data_ptr(), 64, 64, 64, NONE, stream)
+    assert st == binding.TG_ERR_INVALID_ARG
+    with pytest.raises(binding.TgError):
+        binding.gemm(a, a, epilogue=NONE, config_id=999)

@@ -335,6 +335,15 @@ def run_ours(args, w, rank, world):
         del s2
 
     # ---------------------------------------------------------------- end to end (host buffers)
+    e2e = run_e2e(torch, binding, w, s, args, dev, stream, barrier, max_over_ranks, world) \
+        if not args.no_e2e else None
+
+    # ---------------------------------------------------------------- roofline + CPU baseline
+    return finish(torch, binding, dist, w, s, args, rank, world, dev, step_ms, value, kernel_ms,
+                  region_ms, launches_per_step, clocks, also, e2e)
+
+
+def run_e2e(torch, binding, w, s, args, dev, stream, barrier, max_over_ranks, world):
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     A_h = s["A"].pin_memory()
     B_h = s["B"].pin_memory()
@@ -368,8 +377,13 @@ def run_ours(args, w, rank, world):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
     h2d = 2 * (w.M * w.K + w.K * w.N + (w.N if has_bias else 0))
     d2h = 2 * w.M * w.N
+    return {"value": world * w.flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+            "path": "tg_gemm_host: pinned host -> device copies, GEMM, copy back"}
 
-    # ---------------------------------------------------------------- roofline + CPU baseline
+
+def finish(torch, binding, dist, w, s, args, rank, world, dev, step_ms, value, kernel_ms,
+           region_ms, launches_per_step, clocks, also, e2e):
     peaks, peak_src = load_peaks()
     peak_kind = "burst" if region_ms < 1000.0 else "sustained"
     if s["big"] or w.flops / max(w.algorithmic_bytes, 1) > 100:
@@ -413,9 +427,7 @@ def run_ours(args, w, rank, world):
         "pct_of_fp16_dense_peak_nominal": 100.0 * value / world / NOMINAL_FP16_DENSE_TFLOPS,
         "roofline": roof,
         "cpu_baseline": cpu,
-        "e2e": {"value": world * w.flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "path": "tg_gemm_host: pinned host -> device copies, GEMM, copy back"},
+        "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "also": also,
@@ -436,10 +448,19 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--shape", type=int, nargs=3, metavar=("M", "N", "K"),
+                    help="custom fused workload (bias + GELU, N(0,1) inputs, B scaled by "
+                         "1/sqrt(K), seed 7) instead of --workload; for profiling cases")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)     # at least 3 untimed warm-up steps, always
     from tensor_core_gemm_fp16_b200 import workloads as wl
-    w = wl.WORKLOADS[args.workload]
+    if args.shape:
+        M, N, K = args.shape
+        w = wl.Workload(f"fused_{M}x{N}x{K}", M, N, K, wl.EPI_BIAS_GELU, "normal", 7,
+                        b_scale=1.0 / math.sqrt(max(K, 1)), has_bias=True)
+    else:
+        w = wl.WORKLOADS[args.workload]
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if world != args.gpus:

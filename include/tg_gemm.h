@@ -145,12 +145,15 @@ tg_status_t tg_gemm_select_config(int64_t M, int64_t N, int64_t K, int epilogue,
  *                  wait expires; for testing the timeout path only.  The
  *                  kernel then exits cleanly and tg_gemm_check_error returns
  *                  TG_ERR_TIMEOUT.
+ *   group_m        0: the configuration's rasterisation panel height; else
+ *                  the number of M-tiles per panel (1 .. 64)
  */
 #define TG_INJECT_SKIP_FIRST_LOAD 1
 typedef struct {
     int config_id;
     uint64_t wait_limit_ns;
     int inject;
+    int group_m;
 } tg_options_t;
 
 tg_status_t tg_gemm_ex(const void *A, const void *B, const void *bias, void *C,

@@ -52,7 +52,7 @@ class tg_config_t(ctypes.Structure):
 
 class tg_options_t(ctypes.Structure):
     _fields_ = [("config_id", ctypes.c_int), ("wait_limit_ns", ctypes.c_uint64),
-                ("inject", ctypes.c_int)]
+                ("inject", ctypes.c_int), ("group_m", ctypes.c_int)]
 
 
 _lib = None
@@ -110,8 +110,8 @@ def tg_gemm(A: int, B: int, bias: int | None, C: int, M: int, N: int, K: int, ep
 
 
 def tg_gemm_ex(A, B, bias, C, M, N, K, epilogue, config_id=-1, wait_limit_ns=0, inject=0,
-               stream=None) -> int:
-    opts = tg_options_t(config_id, wait_limit_ns, inject)
+               stream=None, group_m=0) -> int:
+    opts = tg_options_t(config_id, wait_limit_ns, inject, group_m)
     return load().tg_gemm_ex(A, B, bias, C, M, N, K, epilogue, ctypes.byref(opts), stream)
 
 
@@ -173,7 +173,8 @@ def _stream_handle(torch, device):
     return torch.cuda.current_stream(device).cuda_stream
 
 
-def gemm(a, b, bias=None, epilogue=None, out=None, *, config_id=-1, wait_limit_ns=0, inject=0):
+def gemm(a, b, bias=None, epilogue=None, out=None, *, config_id=-1, wait_limit_ns=0, inject=0,
+         group_m=0):
     """C = g(a @ b + bias) on the GPU through tg_gemm_ex.
 
     a: (M, K) fp16 CUDA, b: (K, N) fp16 CUDA, bias: (N,) fp16 CUDA or None,
@@ -207,7 +208,7 @@ def gemm(a, b, bias=None, epilogue=None, out=None, *, config_id=-1, wait_limit_n
         st = tg_gemm_ex(a.data_ptr(), b.data_ptr(), bias.data_ptr() if bias is not None else None,
                         out.data_ptr(), M, N, K, epi, config_id=config_id,
                         wait_limit_ns=wait_limit_ns, inject=inject,
-                        stream=_stream_handle(torch, a.device))
+                        stream=_stream_handle(torch, a.device), group_m=group_m)
     if st != TG_OK:
         raise TgError(st, "tg_gemm")
     return out

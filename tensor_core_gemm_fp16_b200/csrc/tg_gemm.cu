@@ -30,16 +30,14 @@ constexpr int kMaxDevices = 64;
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;   // 2 s
 
 // ------------------------------------------------------------------ configs
-using LaunchFn = cudaError_t (*)(const CUtensorMap &, const CUtensorMap &,
+using LaunchFn = cudaError_t (*)(const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
                                  const tg::GemmParams &, int, cudaStream_t);
+using ClusterQueryFn = int (*)(int num_sms);
 
-template <int BN, int ST, int EPI, bool VEC>
-cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const tg::GemmParams &p,
-                        int grid, cudaStream_t stream)
+// One bit per device: the kernel's dynamic shared-memory limit has been raised.
+template <class Kernel>
+cudaError_t ensure_smem_attr(Kernel kern, int smem, std::atomic<uint64_t> &attr_set)
 {
-    auto kern = tg::gemm_persistent_kernel<BN, ST, EPI, VEC>;
-    constexpr int smem = tg::SmemLayout<BN, ST>::kDynamicBytes;
-    static std::atomic<uint64_t> attr_set{0};   // one bit per device
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -49,30 +47,72 @@ cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const tg::
         if (e != cudaSuccess) return e;
         attr_set.fetch_or(bit);
     }
-    kern<<<grid, tg::kThreads, smem, stream>>>(ta, tb, p);
+    return cudaSuccess;
+}
+
+template <int BN, int ST_REQ, int EPI, bool PAIR, int EW, int STORE>
+cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc,
+                        const tg::GemmParams &p, int grid, cudaStream_t stream)
+{
+    constexpr int ST = tg::FittedStages<BN, ST_REQ, PAIR, EW, STORE>::value;
+    using S = tg::KernelShape<BN, ST, PAIR, EW, STORE>;
+    auto kern = tg::gemm_persistent_kernel<BN, ST, EPI, PAIR, EW, STORE>;
+    static std::atomic<uint64_t> attr_set{0};
+    cudaError_t e = ensure_smem_attr(kern, S::kDynamicBytes, attr_set);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(S::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = S::kDynamicBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (PAIR) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 struct KernelConfig {
     tg_config_t info;
-    LaunchFn fn[3][2];   // [epilogue][vectorised C]
+    int store_pref;       // store mode when C rows are 16-byte aligned
+    LaunchFn fn[3][2];    // [epilogue][0: element stores, 1: store_pref]
 };
 
-#define TG_FNS(BN, ST)                                                                      \
+#define TG_FNS(BN, ST, PAIR, EW, SP)                                                        \
     {                                                                                       \
-        {launch_gemm<BN, ST, 0, false>, launch_gemm<BN, ST, 0, true>},                      \
-            {launch_gemm<BN, ST, 1, false>, launch_gemm<BN, ST, 1, true>},                  \
-            {launch_gemm<BN, ST, 2, false>, launch_gemm<BN, ST, 2, true>},                  \
+        {launch_gemm<BN, ST, 0, PAIR, EW, tg::kStoreScalar>,                                \
+         launch_gemm<BN, ST, 0, PAIR, EW, SP>},                                             \
+            {launch_gemm<BN, ST, 1, PAIR, EW, tg::kStoreScalar>,                            \
+             launch_gemm<BN, ST, 1, PAIR, EW, SP>},                                         \
+            {launch_gemm<BN, ST, 2, PAIR, EW, tg::kStoreScalar>,                            \
+             launch_gemm<BN, ST, 2, PAIR, EW, SP>},                                         \
     }
 
-// {id, block_m, block_n, block_k, stages, cta_pair, group_m, epi_warps}
+#define TG_CONFIG(ID, BN, ST, PAIR, EW, SP, GROUP)                                          \
+    {{ID, 128 * ((PAIR) ? 2 : 1), BN, 64, ST, (PAIR) ? 1 : 0, GROUP, EW}, SP,               \
+     TG_FNS(BN, ST, PAIR, EW, SP)}
+
+// {id, BN, stages, CTA pair, epilogue warps, store mode for aligned C, group_m}
 const KernelConfig kConfigs[] = {
-    {{0, 128, 256, 64, 4, 0, 8, 4}, TG_FNS(256, 4)},
-    {{1, 128, 128, 64, 6, 0, 8, 4}, TG_FNS(128, 6)},
-    {{2, 128, 64, 64, 8, 0, 8, 4}, TG_FNS(64, 8)},
-    {{3, 128, 256, 64, 4, 0, 16, 4}, TG_FNS(256, 4)},
-    {{4, 128, 128, 64, 6, 0, 16, 4}, TG_FNS(128, 6)},
-    {{5, 128, 256, 64, 4, 0, 4, 4}, TG_FNS(256, 4)},
+    TG_CONFIG(0, 256, 6, true, 8, tg::kStoreTma, 8),
+    TG_CONFIG(1, 128, 8, true, 8, tg::kStoreTma, 8),
+    TG_CONFIG(2, 256, 4, false, 8, tg::kStoreTma, 8),
+    TG_CONFIG(3, 128, 6, false, 8, tg::kStoreTma, 8),
+    TG_CONFIG(4, 64, 8, false, 4, tg::kStoreTma, 8),
+    TG_CONFIG(5, 256, 6, true, 4, tg::kStoreTma, 8),
+    TG_CONFIG(6, 256, 6, true, 8, tg::kStoreTma, 16),
+    TG_CONFIG(7, 256, 4, false, 4, tg::kStoreVec, 8),
+    TG_CONFIG(8, 256, 7, true, 4, tg::kStoreVec, 8),
+    TG_CONFIG(9, 256, 5, true, 4, tg::kStoreTma, 8),
+    TG_CONFIG(10, 256, 4, true, 4, tg::kStoreTma, 8),
 };
 constexpr int kNumConfigs = sizeof(kConfigs) / sizeof(kConfigs[0]);
 
@@ -86,23 +126,27 @@ struct TableRow {
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Size rule for shapes missing from the table: minimise
-// waves(BN) * BN / efficiency(BN), i.e. the last wave's finishing time in
-// units of a 128 x BN tile, with wider tiles credited for their better
-// operand reuse.
+// waves * (per-SM tile work) / efficiency, i.e. the finishing time of the
+// last wave in units of one 128 x 64 per-SM tile slice, with wider tiles and
+// CTA pairs credited for their better operand reuse.
 int rule_config(int64_t M, int64_t N, int num_sms)
 {
-    const int ids[3] = {0, 1, 2};
-    const double eff[3] = {1.0, 0.9, 0.75};
+    struct Cand { int id; double eff; };
+    const Cand cands[] = {{0, 1.0}, {1, 0.93}, {3, 0.85}, {4, 0.7}};
+    const int sms = num_sms > 1 ? num_sms : 148;
     int best = 0;
     double best_score = 0;
-    for (int t = 0; t < 3; ++t) {
-        const int bn = kConfigs[ids[t]].info.block_n;
-        const int64_t tiles = ceil_div(M, 128) * ceil_div(N, bn);
-        const double waves = static_cast<double>(ceil_div(tiles, num_sms > 0 ? num_sms : 148));
-        const double score = waves * bn / eff[t];
-        if (t == 0 || score < best_score - 1e-9) {
-            best = ids[t];
+    bool first = true;
+    for (const Cand &c : cands) {
+        const tg_config_t &ci = kConfigs[c.id].info;
+        const int64_t tiles = ceil_div(M, ci.block_m) * ceil_div(N, ci.block_n);
+        const int64_t units = ci.cta_pair ? sms / 2 : sms;
+        const double waves = static_cast<double>(ceil_div(tiles, units));
+        const double score = waves * (ci.block_n / 64.0) / c.eff;
+        if (first || score < best_score - 1e-9) {
+            best = c.id;
             best_score = score;
+            first = false;
         }
     }
     return best;
@@ -111,7 +155,7 @@ int rule_config(int64_t M, int64_t N, int num_sms)
 int choose_config(int64_t M, int64_t N, int64_t K, int epilogue, int num_sms)
 {
     for (const TableRow &r : kShapeTable)
-        if (r.M == M && r.N == N && r.K == K && (r.epilogue < 0 || r.epilogue == epilogue) &&
+        if (r.M >= 0 && r.M == M && r.N == N && r.K == K && (r.epilogue < 0 || r.epilogue == epilogue) &&
             r.config >= 0 && r.config < kNumConfigs)
             return r.config;
     return rule_config(M, N, num_sms);
@@ -186,15 +230,16 @@ tg_status_t device_state(DeviceState **out, int *dev_out)
 }
 
 bool encode_2d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t outer,
-               uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer)
+               uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+               CUtensorMapSwizzle swizzle)
 {
     const cuuint64_t dims[2] = {inner, outer};
     const cuuint64_t strides[1] = {pitch_bytes};
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims,
-                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -266,6 +311,7 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
     if (opts && (opts->config_id < -1 || opts->config_id >= kNumConfigs)) return TG_ERR_INVALID_ARG;
     if (opts && (opts->inject != 0 && opts->inject != TG_INJECT_SKIP_FIRST_LOAD))
         return TG_ERR_INVALID_ARG;
+    if (opts && (opts->group_m < 0 || opts->group_m > 64)) return TG_ERR_INVALID_ARG;
     DeviceState *dev = nullptr;
     st = device_state(&dev, nullptr);
     if (st != TG_OK) return st;
@@ -281,7 +327,6 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
     // TMA needs 16-byte aligned bases and pitches; otherwise repack.
     const bool a_direct = aligned(A, 16) && (K % 8 == 0);
     const bool b_direct = aligned(B, 16) && (N % 8 == 0);
-    const bool vec = aligned(C, 16) && (N % 8 == 0) && (!bias || aligned(bias, 16));
     const int64_t lda = a_direct ? K : (K + 7) / 8 * 8;
     const int64_t ldb = b_direct ? N : (N + 7) / 8 * 8;
     void *tmp = nullptr;
@@ -309,9 +354,16 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
         }
     }
 
-    CUtensorMap ta, tb;
-    if (!encode_2d(&ta, Aeff, K, M, 2 * lda, tg::kBlockK, tg::kBlockM) ||
-        !encode_2d(&tb, Beff, N, K, 2 * ldb, tg::kBChunkN, tg::kBlockK)) {
+    const bool c_rows16 = aligned(C, 16) && (N % 8 == 0);
+    const int store = c_rows16 ? cfg.store_pref : tg::kStoreScalar;
+    CUtensorMap ta, tb, tc;
+    std::memset(&tc, 0, sizeof(tc));
+    if (!encode_2d(&ta, Aeff, K, M, 2 * lda, tg::kBlockK, tg::kBlockM,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&tb, Beff, N, K, 2 * ldb, tg::kBChunkN, tg::kBlockK,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        (store == tg::kStoreTma &&
+         !encode_2d(&tc, C, N, M, 2 * N, tg::kStoreCols, 32, CU_TENSOR_MAP_SWIZZLE_64B))) {
         if (tmp) cudaFreeAsync(tmp, stream);
         return TG_ERR_CUDA;
     }
@@ -323,17 +375,22 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
     p.N = N;
     p.K = K;
     p.ldc = N;
-    p.num_m_tiles = static_cast<int>(ceil_div(M, tg::kBlockM));
+    p.num_m_tiles = static_cast<int>(ceil_div(M, cfg.info.block_m));
     p.num_n_tiles = static_cast<int>(ceil_div(N, bn));
     p.num_k_blocks = static_cast<int>(ceil_div(K, tg::kBlockK));
     p.num_tiles = p.num_m_tiles * p.num_n_tiles;
-    p.group_m = cfg.info.group_m;
+    p.group_m = (opts && opts->group_m > 0) ? opts->group_m : cfg.info.group_m;
     p.inject = opts ? opts->inject : 0;
+    p.bias_vec = (bias && aligned(bias, 16)) ? 1 : 0;
     p.wait_limit_ns = (opts && opts->wait_limit_ns) ? opts->wait_limit_ns : kDefaultWaitLimitNs;
     p.error_word = dev->error_word;
-    const int grid = static_cast<int>(std::min<int64_t>(p.num_tiles, dev->num_sms));
+    // Persistent grid: one CTA (or CTA pair) per SM (pair of SMs), never
+    // more than there are tiles.
+    const int units = cfg.info.cta_pair ? dev->num_sms / 2 : dev->num_sms;
+    const int grid = static_cast<int>(std::min<int64_t>(p.num_tiles, units)) *
+                     (cfg.info.cta_pair ? 2 : 1);
 
-    cudaError_t e = cfg.fn[epilogue][vec ? 1 : 0](ta, tb, p, grid, stream);
+    cudaError_t e = cfg.fn[epilogue][store == tg::kStoreScalar ? 0 : 1](ta, tb, tc, p, grid, stream);
     if (tmp) cudaFreeAsync(tmp, stream);
     if (e != cudaSuccess) {
         cudaGetLastError();

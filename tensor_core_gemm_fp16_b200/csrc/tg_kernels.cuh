@@ -30,17 +30,14 @@
 
 namespace tg {
 
-constexpr int kBlockM = 128;   // rows of the MMA tile (one TMEM lane per row)
+constexpr int kBlockM = 128;   // rows of A (and of C) per CTA: one TMEM lane per row
 constexpr int kBlockK = 64;    // K per stage: 64 fp16 = one 128-byte swizzle row
 constexpr int kBChunkN = 64;   // B is loaded in 64-column boxes (128 bytes wide)
 constexpr int kUmmaK = 16;     // K of one kind::f16 MMA instruction
 constexpr int kABytesStage = kBlockM * kBlockK * 2;   // 16 KiB
 constexpr int kBChunkBytes = kBChunkN * kBlockK * 2;  // 8 KiB
-
-constexpr int kEpiWarps = 4;                       // warps 0..3 drain TMEM
-constexpr int kProducerWarp = 4;                   // TMA producer
-constexpr int kMmaWarp = 5;                        // MMA issuer + TMEM owner
-constexpr int kThreads = 32 * 6;
+constexpr int kStoreCols = 32;                        // C columns per TMEM load / TMA store box
+constexpr int kStoreBoxBytes = 32 * kStoreCols * 2;   // 32 rows x 32 fp16 = 2 KiB
 
 // Error word bits (OR-ed into the per-device error word on a wait expiry).
 constexpr unsigned kErrProducerWait = 1u;
@@ -49,35 +46,74 @@ constexpr unsigned kErrEpilogueWait = 4u;
 constexpr unsigned kErrDrain = 8u;
 
 enum : int { kEpiNone = 0, kEpiBias = 1, kEpiBiasGelu = 2 };
+// How the epilogue writes C: element stores (any pitch), 16-byte stores
+// (16-byte aligned rows), or TMA stores from a swizzled staging tile.
+enum : int { kStoreScalar = 0, kStoreVec = 1, kStoreTma = 2 };
 
 struct GemmParams {
     const __half *bias;     // [N] or nullptr
     __half *C;              // [M, ldc]
     int64_t M, N, K;
     int64_t ldc;
-    int num_m_tiles;
-    int num_n_tiles;
-    int num_k_blocks;
+    int num_m_tiles;        // ceil(M / tile_m), tile_m = 128 (single CTA) or 256 (CTA pair)
+    int num_n_tiles;        // ceil(N / BN)
+    int num_k_blocks;       // ceil(K / 64)
     int num_tiles;
     int group_m;
-    int inject;             // 1: CTA 0 skips its first operand load (timeout test)
+    int inject;             // 1: the first CTA skips its first operand load (timeout test)
+    int bias_vec;           // bias is 16-byte aligned: load it 8 values at a time
     uint64_t wait_limit_ns;
     unsigned *error_word;   // device address of the per-device error word
 };
 
-template <int BN, int STAGES>
-struct SmemLayout {
-    static constexpr int kBBytesStage = BN / kBChunkN * kBChunkBytes;
-    static constexpr int kStageBytes = kABytesStage + kBBytesStage;
+// Compile-time shape of one kernel variant.
+//   BN        output columns per tile (the MMA's N)
+//   STAGES    depth of the shared-memory operand ring
+//   PAIR      two CTAs of a cluster run one cta_group::2 MMA on a 256-row tile;
+//             each loads 128 rows of A and BN/2 columns of B
+//   EPI_WARPS 4 or 8 warps drain TMEM (8: two per lane quarter, halving columns)
+template <int BN, int STAGES, bool PAIR, int EPI_WARPS, int STORE>
+struct KernelShape {
+    static_assert(BN == 64 || BN == 128 || BN == 256, "BN must be 64, 128 or 256");
+    static_assert(!PAIR || BN >= 128, "a CTA pair needs BN >= 128");
+    static_assert(EPI_WARPS == 4 || EPI_WARPS == 8, "4 or 8 epilogue warps");
+    static constexpr int kCG = PAIR ? 2 : 1;
+    static constexpr int kTileM = kBlockM * kCG;
+    static constexpr int kCtaN = BN / kCG;                       // B columns loaded per CTA
+    static constexpr int kBChunks = kCtaN / kBChunkN;
+    static constexpr int kStageBytes = kABytesStage + kBChunks * kBChunkBytes;
+    static constexpr uint32_t kTxBytes = kCG * kStageBytes;      // both CTAs land on the leader
     static constexpr int kRingBytes = STAGES * kStageBytes;
+    static constexpr int kStagingBytes = STORE != kStoreVec ? EPI_WARPS * 2 * kStoreBoxBytes : 0;
     // barriers: full[STAGES], empty[STAGES], tmem_full[2], tmem_empty[2], drain
     static constexpr int kNumBars = 2 * STAGES + 5;
-    static constexpr int kBarOffset = kRingBytes;
+    static constexpr int kStagingOffset = kRingBytes;
+    static constexpr int kBarOffset = kRingBytes + kStagingBytes;
     static constexpr int kTmemSlotOffset = kBarOffset + kNumBars * 8;
     static constexpr int kAbortOffset = kTmemSlotOffset + 4;
     static constexpr int kUsedBytes = kAbortOffset + 4;
-    static constexpr int kDynamicBytes = kUsedBytes + 1024;   // slack for 1024-B alignment
-    static constexpr uint32_t kTmemCols = 2 * BN;             // double-buffered accumulator
+    static constexpr int kDynamicBytes = kUsedBytes + 1024;     // slack for 1024-B alignment
+    static constexpr uint32_t kTmemCols = 2 * BN;               // double-buffered accumulator
+    static constexpr int kProducerWarp = EPI_WARPS;
+    static constexpr int kMmaWarp = EPI_WARPS + 1;
+    static constexpr int kThreads = 32 * (EPI_WARPS + 2);
+    static constexpr int kChunksPerWarp = (BN / kStoreCols) / (EPI_WARPS / 4);
+    static constexpr uint32_t kTmemEmptyArrivals = kCG * EPI_WARPS;
+};
+
+constexpr int kMaxDynamicSmem = 232448;   // 227 KiB: the sm_100 per-block opt-in limit
+
+// STAGES, reduced by one when this store mode's staging buffers would push
+// the block past the shared-memory limit (the element-store fallback of a
+// configuration tuned for direct vector stores).
+template <int BN, int STAGES, bool PAIR, int EPI_WARPS, int STORE>
+struct FittedStages {
+    static constexpr int value =
+        KernelShape<BN, STAGES, PAIR, EPI_WARPS, STORE>::kDynamicBytes <= kMaxDynamicSmem
+            ? STAGES
+            : STAGES - 1;
+    static_assert(KernelShape<BN, value, PAIR, EPI_WARPS, STORE>::kDynamicBytes <= kMaxDynamicSmem,
+                  "shared-memory budget exceeded");
 };
 
 // Tile index -> (m tile, n tile), walking group_m M-tiles per panel so that
@@ -94,11 +130,28 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int 
     nt = r / rows;
 }
 
+// GELU(v) = v * Phi(v), Phi the standard normal CDF, Phi(v) = erfc(-v/sqrt 2)/2.
+// erfc(z) for z = |v|/sqrt(2) >= 0 is evaluated as t * exp(-z^2 + P(t)),
+// t = 1/(1 + z/2), the Chebyshev-type form of Numerical Recipes (2nd ed.,
+// section 6.2) with our own degree-7 fit of P (csrc/fit_erfc.py: max error
+// of P 6.2e-7 on z in [0, 9]); Phi(-|v|) = erfc(z)/2 and Phi(|v|) = 1 - that.
+// In fp32 the relative error of GELU stays below 6e-6 for |v| <= 8.5 (fp16's
+// half-ulp is 2.4e-4), and the tail keeps full relative accuracy (no 1 + erf
+// cancellation).  About 20 instructions per element.
 __device__ __forceinline__ float gelu_erf(float v)
 {
-    // v * Phi(v) with Phi(v) = erfc(-v / sqrt 2) / 2; erfc keeps relative
-    // accuracy in the far negative tail where 1 + erf(.) would cancel.
-    return 0.5f * v * erfcf(-v * 0.70710678118654752f);
+    const float z = fabsf(v) * 0.70710678118654752f;
+    const float t = __fdividef(1.0f, fmaf(0.5f, z, 1.0f));
+    float p = -1.811217638e-01f;
+    p = fmaf(p, t, 7.227813026e-01f);
+    p = fmaf(p, t, -9.495873675e-01f);
+    p = fmaf(p, t, 3.007620395e-01f);
+    p = fmaf(p, t, -1.279667006e-02f);
+    p = fmaf(p, t, 3.855720234e-01f);
+    p = fmaf(p, t, 9.999567273e-01f);
+    p = fmaf(p, t, -1.265566907e+00f);
+    const float tail = 0.5f * t * __expf(fmaf(-z, z, p));   // Phi(-|v|)
+    return v * (v > 0.0f ? 1.0f - tail : tail);
 }
 
 template <int EPI>
@@ -110,37 +163,80 @@ __device__ __forceinline__ float apply_epilogue(float acc, float beta)
     return v;
 }
 
+// Eight consecutive bias values as floats (zeros past N or without bias).
+template <int EPI>
+__device__ __forceinline__ void load_bias8(const __half *bias, int64_t col, int64_t N, bool vec,
+                                           float (&b)[8])
+{
+    if (EPI == kEpiNone || bias == nullptr) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) b[e] = 0.f;
+        return;
+    }
+    if (vec && col + 8 <= N) {
+        uint4 u = __ldg(reinterpret_cast<const uint4 *>(bias + col));
+        const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(h[e]);
+            b[2 * e] = f.x;
+            b[2 * e + 1] = f.y;
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) b[e] = (col + e < N) ? __half2float(bias[col + e]) : 0.f;
+    }
+}
+
+// Eight fp32 accumulators + bias -> epilogue -> eight fp16 packed in a uint4.
+template <int EPI>
+__device__ __forceinline__ uint4 epilogue8(const uint32_t *r, const float (&b)[8])
+{
+    uint4 u;
+    __half2 *h = reinterpret_cast<__half2 *>(&u);
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+        h[e] = __floats2half2_rn(apply_epilogue<EPI>(__uint_as_float(r[2 * e]), b[2 * e]),
+                                 apply_epilogue<EPI>(__uint_as_float(r[2 * e + 1]), b[2 * e + 1]));
+    return u;
+}
+
 // ---------------------------------------------------------------------------
 // Persistent warp-specialised GEMM.
-//   warps 0-3  epilogue: TMEM -> registers -> bias/GELU -> fp16 -> global
-//   warp 4     TMA producer (one lane)
-//   warp 5     TMEM allocator + MMA issuer (one lane)
-// VEC: C rows and bias are 16-byte addressable (N % 8 == 0, aligned bases).
-template <int BN, int STAGES, int EPI, bool VEC>
-__global__ void __launch_bounds__(kThreads, 1)
+//   warps [0, EPI_WARPS)  epilogue: TMEM -> registers -> bias/GELU -> fp16 -> C
+//   warp EPI_WARPS        TMA producer (one lane)
+//   warp EPI_WARPS + 1    TMEM allocator; MMA issuer (one lane; the leader CTA
+//                         of a pair issues for both)
+template <int BN, int STAGES, int EPI, bool PAIR, int EPI_WARPS, int STORE>
+__global__ void __launch_bounds__(KernelShape<BN, STAGES, PAIR, EPI_WARPS, STORE>::kThreads, 1)
     gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmA,
-                           const __grid_constant__ CUtensorMap tmB, const GemmParams p)
+                           const __grid_constant__ CUtensorMap tmB,
+                           const __grid_constant__ CUtensorMap tmC, const GemmParams p)
 {
-    using L = SmemLayout<BN, STAGES>;
-    static_assert(BN == 64 || BN == 128 || BN == 256, "BN must be 64, 128 or 256");
-    constexpr uint32_t kIdesc = idesc_f16_f32(kBlockM, BN);
-    constexpr uint32_t kTxBytes = L::kStageBytes;
+    using S = KernelShape<BN, STAGES, PAIR, EPI_WARPS, STORE>;
+    constexpr int CG = S::kCG;
+    constexpr uint32_t kIdesc = idesc_f16_f32(S::kTileM, BN);
 
     extern __shared__ uint8_t smem_raw[];
-    // Round the dynamic shared-memory base up to 1024 B (128-byte swizzle atom).
+    // Round the dynamic shared-memory base up to 1024 B (128-byte swizzle atom);
+    // the offset is the same in both CTAs of a pair.
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOffset);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S::kBarOffset);
     uint64_t *full_bar = bars;
     uint64_t *empty_bar = bars + STAGES;
     uint64_t *tmem_full_bar = bars + 2 * STAGES;
     uint64_t *tmem_empty_bar = bars + 2 * STAGES + 2;
     uint64_t *drain_bar = bars + 2 * STAGES + 4;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemSlotOffset);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kAbortOffset);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::kTmemSlotOffset);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + S::kAbortOffset);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t cta_rank = PAIR ? cluster_cta_rank() : 0u;
+    const bool leader = cta_rank == 0;
+    const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int num_units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -149,40 +245,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tmem_full_bar[b], 1);
-            mbar_init(&tmem_empty_bar[b], kEpiWarps);
+            mbar_init(&tmem_empty_bar[b], S::kTmemEmptyArrivals);
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == kProducerWarp && lane == 0) {
+    if (warp == S::kProducerWarp && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if (STORE == kStoreTma) tma_prefetch_desc(&tmC);
     }
-    if (warp == kMmaWarp) {
-        tmem_alloc(tmem_slot, L::kTmemCols);
-        tmem_relinquish();
+    if (warp == S::kMmaWarp) {
+        tmem_alloc<CG>(tmem_slot, S::kTmemCols);
+        tmem_relinquish<CG>();
     }
     tc_fence_before_sync();
     __syncthreads();
+    if (PAIR) cluster_sync();   // peer barriers initialised before any remote use
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
 
     const uint32_t smem_base = smem_u32(smem);
     const uint64_t limit = p.wait_limit_ns;
 
-    if (warp == kProducerWarp) {
+    if (warp == S::kProducerWarp) {
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            // Per stage: parity of the last load issued into it, or -1.
-            int pending_parity[STAGES];
+            // Per stage: 1 + parity of the last load whose bytes this CTA's
+            // full barrier expects, or 0 for none (drained before exit).
+            uint32_t pending[STAGES];
 #pragma unroll
-            for (int s = 0; s < STAGES; ++s) pending_parity[s] = -1;
+            for (int s = 0; s < STAGES; ++s) pending[s] = 0;
             bool skip_next = (p.inject == 1 && blockIdx.x == 0);
-            for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+            for (int tile = unit; tile < p.num_tiles; tile += num_units) {
                 int mt, nt;
                 tile_coords(tile, p.num_m_tiles, p.num_n_tiles, p.group_m, mt, nt);
+                const int a_row = mt * S::kTileM + static_cast<int>(cta_rank) * kBlockM;
+                const int b_col = nt * BN + static_cast<int>(cta_rank) * S::kCtaN;
                 bool ok = true;
                 for (int kb = 0; kb < p.num_k_blocks; ++kb) {
                     if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, abort_flag, limit,
@@ -193,15 +294,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (skip_next) {
                         skip_next = false;   // injected fault: this stage never fills
                     } else {
-                        const uint32_t a_dst = smem_base + stage * L::kStageBytes;
+                        const uint32_t a_dst = smem_base + stage * S::kStageBytes;
                         const uint32_t b_dst = a_dst + kABytesStage;
-                        mbar_arrive_expect_tx(&full_bar[stage], kTxBytes);
-                        tma_load_2d(a_dst, &tmA, &full_bar[stage], kb * kBlockK, mt * kBlockM);
+                        if (leader) {
+                            mbar_arrive_expect_tx(&full_bar[stage], S::kTxBytes);
+                            pending[stage] = 1u + phase;
+                        }
+                        if constexpr (PAIR) {
+                            const uint32_t bar = map_to_cta(smem_u32(&full_bar[stage]), 0);
+                            tma_load_2d_pair(a_dst, &tmA, bar, kb * kBlockK, a_row);
 #pragma unroll
-                        for (int j = 0; j < BN / kBChunkN; ++j)
-                            tma_load_2d(b_dst + j * kBChunkBytes, &tmB, &full_bar[stage],
-                                        nt * BN + j * kBChunkN, kb * kBlockK);
-                        pending_parity[stage] = static_cast<int>(phase);
+                            for (int j = 0; j < S::kBChunks; ++j)
+                                tma_load_2d_pair(b_dst + j * kBChunkBytes, &tmB, bar,
+                                                 b_col + j * kBChunkN, kb * kBlockK);
+                        } else {
+                            tma_load_2d(a_dst, &tmA, &full_bar[stage], kb * kBlockK, a_row);
+#pragma unroll
+                            for (int j = 0; j < S::kBChunks; ++j)
+                                tma_load_2d(b_dst + j * kBChunkBytes, &tmB, &full_bar[stage],
+                                            b_col + j * kBChunkN, kb * kBlockK);
+                        }
                     }
                     if (++stage == STAGES) {
                         stage = 0;
@@ -210,22 +322,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (!ok) break;
             }
-            // Let every load this thread issued land before the CTA can exit.
+            // Let the loads this CTA's full barriers track land before exit.
+            // (A pair's peer CTA is covered by the leader's drain plus the
+            // cluster barrier at teardown.)
 #pragma unroll
             for (int s = 0; s < STAGES; ++s)
-                if (pending_parity[s] >= 0 &&
-                    !mbar_wait_drain(&full_bar[s], static_cast<uint32_t>(pending_parity[s]), limit))
+                if (pending[s] != 0 && !mbar_wait_drain(&full_bar[s], pending[s] - 1u, limit))
                     atomicOr(p.error_word, kErrDrain);
         }
         __syncwarp();
-    } else if (warp == kMmaWarp) {
-        if (lane == 0) {
+    } else if (warp == S::kMmaWarp) {
+        if (lane == 0 && leader) {
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
             bool issued_any = false;
-            for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+            for (int tile = unit; tile < p.num_tiles; tile += num_units) {
                 if (!mbar_wait_bounded(&tmem_empty_bar[acc], acc_phase ^ 1u, abort_flag, limit,
                                        p.error_word, kErrMmaWait))
                     break;
@@ -239,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint32_t a_addr = smem_base + stage * L::kStageBytes;
+                    const uint32_t a_addr = smem_base + stage * S::kStageBytes;
                     const uint32_t b_addr = a_addr + kABytesStage;
                     // A: K-major, 128-B swizzle; 8-row groups 1024 B apart.
                     const uint64_t a_desc = smem_desc_sw128(a_addr, 16, 1024);
@@ -249,22 +362,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < kBlockK / kUmmaK; ++kk) {
                         // K step inside the swizzle row: +32 B for A; +16 rows
-                        // (2 KiB) for B.  Both are added to the start-address
-                        // field (units of 16 B).
+                        // (2 KiB) for B, added to the start-address field (16 B units).
                         const uint64_t a_k = a_desc + static_cast<uint64_t>((kk * kUmmaK * 2) >> 4);
                         const uint64_t b_k =
                             b_desc + static_cast<uint64_t>((kk * kUmmaK * 128) >> 4);
-                        mma_f16_ss(d_tmem, a_k, b_k, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                        mma_f16_ss<CG>(d_tmem, a_k, b_k, kIdesc, (kb | kk) != 0 ? 1u : 0u);
                     }
                     issued_any = true;
-                    mma_commit(&empty_bar[stage]);   // stage free once these MMAs finish
+                    // the stage is free (in both CTAs) once these MMAs finish
+                    if constexpr (PAIR)
+                        mma_commit_pair_multicast(&empty_bar[stage], 0x3);
+                    else
+                        mma_commit<1>(&empty_bar[stage]);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                mma_commit(&tmem_full_bar[acc]);     // accumulator ready for the epilogue
+                // accumulator ready for the epilogue (of both CTAs)
+                if constexpr (PAIR)
+                    mma_commit_pair_multicast(&tmem_full_bar[acc], 0x3);
+                else
+                    mma_commit<1>(&tmem_full_bar[acc]);
                 if (++acc == 2) {
                     acc = 0;
                     acc_phase ^= 1u;
@@ -272,16 +392,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // Wait for every MMA this thread issued before TMEM is released.
             if (issued_any) {
-                mma_commit(drain_bar);
+                mma_commit<CG>(drain_bar);
                 if (!mbar_wait_drain(drain_bar, 0, limit)) atomicOr(p.error_word, kErrDrain);
             }
         }
         __syncwarp();
     } else {
-        // Epilogue warps 0..3: warp w owns TMEM lanes [32w, 32w + 32) = tile rows.
+        // Epilogue warp w: TMEM lanes [32 (w % 4), +32) = 32 tile rows; with 8
+        // warps, w / 4 selects the half of the columns.
+        const int quarter = warp & 3;
+        const int chunk0 = (warp >> 2) * S::kChunksPerWarp;
+        const uint32_t empty_bar_leader =
+            PAIR ? map_to_cta(smem_u32(&tmem_empty_bar[0]), 0) : 0u;
+        const uint32_t staging = smem_base + S::kStagingOffset + warp * 2 * kStoreBoxBytes;
+        const bool bias_vec = p.bias_vec != 0;
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+        uint32_t store_count = 0;
+        for (int tile = unit; tile < p.num_tiles; tile += num_units) {
             int mt, nt;
             tile_coords(tile, p.num_m_tiles, p.num_n_tiles, p.group_m, mt, nt);
             int ok = 0;
@@ -294,86 +422,127 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             tc_fence_after_sync();
 
-            const int64_t row = static_cast<int64_t>(mt) * kBlockM + warp * 32 + lane;
+            const int64_t row0 = static_cast<int64_t>(mt) * S::kTileM +
+                                 static_cast<int64_t>(cta_rank) * kBlockM + quarter * 32;
+            const int64_t row = row0 + lane;
             const bool row_ok = row < p.M;
             __half *crow = p.C + row * p.ldc;
-            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) +
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(acc * BN);
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                const int64_t col0 = static_cast<int64_t>(nt) * BN + c * 32;
-                if (col0 >= p.N) break;          // warp-uniform: whole chunk past N
+            for (int c = chunk0; c < chunk0 + S::kChunksPerWarp; ++c) {
+                const int64_t col0 = static_cast<int64_t>(nt) * BN + c * kStoreCols;
+                // warp-uniform: the chunk lies entirely past N, or all 32 rows past M
+                if (col0 >= p.N || row0 >= p.M) break;
                 uint32_t r[32];
-                tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * 32), r);
+                tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * kStoreCols), r);
                 tmem_wait_ld();
-                const bool full_chunk = col0 + 32 <= p.N;
-                float beta[32];
-                if (EPI != kEpiNone && p.bias != nullptr) {
-                    if (VEC && full_chunk) {
-                        const uint4 *bp = reinterpret_cast<const uint4 *>(p.bias + col0);
+                if constexpr (STORE == kStoreTma) {
+                    // Stage a 32 x 32 fp16 box (64-B rows, 64-B swizzle) and let
+                    // one lane store it with TMA; two boxes alternate.
+                    const uint32_t buf = staging + (store_count & 1u) * kStoreBoxBytes;
+                    if (store_count >= 2) {
+                        if (lane == 0) bulk_wait_group_read<1>();
+                        __syncwarp();
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float b[8];
+                        load_bias8<EPI>(p.bias, col0 + q * 8, p.N, bias_vec, b);
+                        const uint4 u = epilogue8<EPI>(r + q * 8, b);
+                        const uint32_t phys = static_cast<uint32_t>(q) ^ ((lane >> 1) & 3u);
+                        const uint32_t addr = buf + lane * 64u + phys * 16u;
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                                     "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w)
+                                     : "memory");
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmC, buf, static_cast<int32_t>(col0),
+                                     static_cast<int32_t>(row0));
+                        bulk_commit_group();
+                    }
+                    ++store_count;
+                } else if constexpr (STORE == kStoreVec) {
+                    if (row_ok) {
+                        const bool full = col0 + kStoreCols <= p.N;
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-                            uint4 u = __ldg(bp + q);
-                            const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+                            float b[8];
+                            load_bias8<EPI>(p.bias, col0 + q * 8, p.N, bias_vec, b);
+                            const uint4 u = epilogue8<EPI>(r + q * 8, b);
+                            if (full) {
+                                *reinterpret_cast<uint4 *>(crow + col0 + q * 8) = u;
+                            } else {
+                                const __half *h = reinterpret_cast<const __half *>(&u);
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                float2 f = __half22float2(h[e]);
-                                beta[q * 8 + 2 * e] = f.x;
-                                beta[q * 8 + 2 * e + 1] = f.y;
+                                for (int e = 0; e < 8; ++e)
+                                    if (col0 + q * 8 + e < p.N) crow[col0 + q * 8 + e] = h[e];
                             }
                         }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            beta[j] = (col0 + j < p.N) ? __half2float(p.bias[col0 + j]) : 0.f;
                     }
                 } else {
+                    // Any pitch: stage the 32 x 32 box (same swizzled layout as
+                    // the TMA path), then write it back one row per
+                    // instruction, lane l storing column l (64 contiguous bytes).
+                    const uint32_t buf = staging + (store_count & 1u) * kStoreBoxBytes;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) beta[j] = 0.f;
-                }
-                if (row_ok) {
-                    if (VEC && full_chunk) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(crow + col0);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint4 u;
-                            __half2 *h = reinterpret_cast<__half2 *>(&u);
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int j = q * 8 + 2 * e;
-                                const float lo = apply_epilogue<EPI>(__uint_as_float(r[j]), beta[j]);
-                                const float hi =
-                                    apply_epilogue<EPI>(__uint_as_float(r[j + 1]), beta[j + 1]);
-                                h[e] = __floats2half2_rn(lo, hi);
-                            }
-                            dst[q] = u;
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (col0 + j < p.N)
-                                crow[col0 + j] = __float2half_rn(
-                                    apply_epilogue<EPI>(__uint_as_float(r[j]), beta[j]));
+                    for (int q = 0; q < 4; ++q) {
+                        float b[8];
+                        load_bias8<EPI>(p.bias, col0 + q * 8, p.N, false, b);
+                        const uint4 u = epilogue8<EPI>(r + q * 8, b);
+                        const uint32_t phys = static_cast<uint32_t>(q) ^ ((lane >> 1) & 3u);
+                        const uint32_t addr = buf + lane * 64u + phys * 16u;
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                                     "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w)
+                                     : "memory");
                     }
+                    __syncwarp();
+                    const bool col_ok = col0 + lane < p.N;
+                    const uint32_t q = static_cast<uint32_t>(lane) >> 3;
+                    const uint32_t within = (static_cast<uint32_t>(lane) & 7u) * 2u;
+#pragma unroll 4
+                    for (int rr = 0; rr < 32; ++rr) {
+                        const uint32_t phys = q ^ ((static_cast<uint32_t>(rr) >> 1) & 3u);
+                        unsigned short h;
+                        asm volatile("ld.shared.u16 %0, [%1];"
+                                     : "=h"(h)
+                                     : "r"(buf + static_cast<uint32_t>(rr) * 64u + phys * 16u +
+                                           within));
+                        if (col_ok && row0 + rr < p.M)
+                            p.C[(row0 + rr) * p.ldc + col0 + lane] = __ushort_as_half(h);
+                    }
+                    __syncwarp();
+                    ++store_count;
                 }
             }
+            // All TMEM reads of this accumulator are complete (wait::ld above).
             tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tmem_empty_bar[acc]);
+            if (lane == 0) {
+                if (PAIR)
+                    mbar_arrive_cluster(empty_bar_leader + static_cast<uint32_t>(acc * 8));
+                else
+                    mbar_arrive(&tmem_empty_bar[acc]);
+            }
             if (++acc == 2) {
                 acc = 0;
                 acc_phase ^= 1u;
             }
         }
+        if (STORE == kStoreTma && lane == 0) bulk_wait_group_all();
+        __syncwarp();
     }
 
     // Teardown: every role has returned (all waits are bounded), so no thread
-    // still reads TMEM and no MMA or copy is in flight.
+    // still reads TMEM and no MMA or copy tracked by this CTA is in flight.
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == kMmaWarp) {
+    if (PAIR) cluster_sync();   // the leader's MMAs into this CTA's TMEM are done
+    if (warp == S::kMmaWarp) {
         tc_fence_after_sync();
-        tmem_dealloc(tmem_base, L::kTmemCols);
+        tmem_dealloc<CG>(tmem_base, S::kTmemCols);
     }
 }
 

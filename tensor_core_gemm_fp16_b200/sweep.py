@@ -1,0 +1,216 @@
+"""Offline schedule sweep: time every compiled configuration on each shape
+and (optionally) rewrite csrc/tg_configs.inc with the winners.
+
+    python -m tensor_core_gemm_fp16_b200.sweep [--shapes all|NAME ...]
+        [--reps 20] [--warmup 5] [--write] [--json out.json]
+
+The tutorial sweeps tile sizes, pipeline stages, thread counts and an L2
+swizzle by hand on its 2048^3 GEMM and keeps the fastest that also passes
+its relative-Frobenius check ("Designing High-Performance GPU Kernels with
+TileLang", thecryptopost.io, section 3 "Knobs"), noting that the best
+schedule depends on the architecture and the shape.  This tool does the
+same over this library's compiled configurations on B200: every candidate
+is checked against torch's fp32 matmul of the same fp16 inputs (relative
+Frobenius error < 2e-2, as in the tutorial's sweep) before it is timed, and
+it is timed with CUDA events (median of `reps` launches; L2 flushed before
+each launch when the operands fit in L2).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+TABLE = os.path.join(HERE, "csrc", "tg_configs.inc")
+L2_BYTES = 126 * 1024 * 1024
+
+DEFAULT_SHAPES = {
+    # name: (M, N, K, epilogue)
+    "gemm_256": (256, 256, 256, 0),
+    "gemm_2048": (2048, 2048, 2048, 0),
+    "fused_2048": (2048, 2048, 2048, 2),
+    "ragged_fused": (3000, 1537, 2050, 2),
+    "fused_8192": (8192, 8192, 8192, 2),
+    "gemm_8192": (8192, 8192, 8192, 0),
+}
+
+
+def time_config(torch, binding, a, b, bias, c, M, N, K, epi, cfg, reps, warmup, flush, gm=0):
+    stream = torch.cuda.current_stream()
+    args = (a.data_ptr(), b.data_ptr(), bias.data_ptr() if bias is not None else None,
+            c.data_ptr(), M, N, K, epi)
+
+    def launch():
+        st = binding.tg_gemm_ex(*args, config_id=cfg, stream=stream.cuda_stream, group_m=gm)
+        if st != binding.TG_OK:
+            raise binding.TgError(st, f"config {cfg}")
+
+    for _ in range(warmup):
+        launch()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        if flush is not None:
+            flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        launch()
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    st = binding.tg_gemm_check_error(stream.cuda_stream)
+    if st != binding.TG_OK:
+        raise binding.TgError(st, f"config {cfg}")
+    return statistics.median(times)
+
+
+def time_library(torch, a, b, bias, epi, reps, warmup, flush):
+    """torch.matmul (cuBLAS) plus the eager bias + erf-GELU, for context only."""
+    F = torch.nn.functional
+
+    def run():
+        if epi == 0:
+            return a @ b
+        y = torch.addmm(bias, a, b)
+        return F.gelu(y) if epi == 2 else y
+
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        if flush is not None:
+            flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        run()
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def sweep_shape(torch, binding, name, M, N, K, epi, reps, warmup, configs, group_ms=(0,),
+                context=False):
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev).manual_seed(1234)
+    a = torch.randn(M, K, device=dev, generator=g).half()
+    b = (torch.randn(K, N, device=dev, generator=g) / math.sqrt(K)).half()
+    bias = torch.randn(N, device=dev, generator=g).half() if epi else None
+    c = torch.empty(M, N, device=dev, dtype=torch.float16)
+    ref = a.float() @ b.float()
+    if epi:
+        ref = torch.nn.functional.gelu(ref + bias.float()) if epi == 2 else ref + bias.float()
+    small = 2 * (M * K + K * N + M * N) <= L2_BYTES
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if small else None
+    rows = []
+    lib_ms = time_library(torch, a, b, bias, epi, reps, warmup, flush) if context else None
+    for cfg, gm in [(c, g) for c in configs for g in group_ms]:
+        info = dict(binding.tg_config_info(cfg))
+        if gm:
+            info["group_m"] = gm
+        st = binding.tg_gemm_ex(a.data_ptr(), b.data_ptr(),
+                                bias.data_ptr() if bias is not None else None, c.data_ptr(),
+                                M, N, K, epi, config_id=cfg, group_m=gm,
+                                stream=torch.cuda.current_stream().cuda_stream)
+        torch.cuda.synchronize()
+        if st != binding.TG_OK:
+            rows.append({"config": cfg, "error": binding.tg_status_string(st)})
+            continue
+        rel = float((c.float() - ref).norm() / ref.norm())
+        if not rel < 2e-2:
+            rows.append({"config": cfg, "error": f"numerically wrong (rel {rel:.2e})"})
+            continue
+        ms = time_config(torch, binding, a, b, bias, c, M, N, K, epi, cfg, reps, warmup, flush,
+                         gm)
+        rows.append({"config": cfg, "group_m_override": gm, "ms": ms, "tflops": 2.0 * M * N * K / (ms * 1e-3) / 1e12,
+                     "rel_err": rel, **{k: info[k] for k in ("block_m", "block_n", "stages",
+                                                           "cta_pair", "group_m", "epi_warps")}})
+    ok = [r for r in rows if "ms" in r]
+    best = min(ok, key=lambda r: r["ms"]) if ok else None
+    return {"shape": name, "M": M, "N": N, "K": K, "epilogue": epi, "rows": rows,
+            "best": best["config"] if best else None,
+            "best_group_m": best["group_m"] if best else None, "l2_flushed": small,
+            "library_ms": lib_ms}
+
+
+def write_table(results, path=TABLE):
+    lines = [
+        "// tg_configs.inc -- per-shape configuration table.",
+        "//",
+        "// Rows: {M, N, K, epilogue (-1 = any), config id}.  A row matches a problem",
+        "// of exactly that shape.  Rows are the winners of the offline sweep",
+        "// (tensor_core_gemm_fp16_b200/sweep.py), which rewrites this file; shapes it",
+        "// does not list fall back to the size rule in tg_gemm.cu.  The last row is a",
+        "// sentinel (M = -1).",
+        "//",
+        "// Written by the sweep on a B200; per row: median ms and TFLOP/s of the winner.",
+        "static const TableRow kShapeTable[] = {",
+    ]
+    for r in results:
+        if r["best"] is None:
+            continue
+        w = next(x for x in r["rows"] if x["config"] == r["best"])
+        lines.append(f"    {{{r['M']}, {r['N']}, {r['K']}, {r['epilogue']}, {r['best']}}},"
+                     f"  // {r['shape']}: {w['ms'] * 1e3:.1f} us, {w['tflops']:.0f} TFLOP/s")
+    lines += ["    {-1, -1, -1, -1, -1},", "};", ""]
+    with open(path, "w") as f:
+        f.write("\n".join(lines))
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__,
+                                 formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--shapes", nargs="*", default=["all"])
+    ap.add_argument("--reps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--configs", type=int, nargs="*", default=None)
+    ap.add_argument("--group-m", type=int, nargs="*", default=[0],
+                    help="rasterisation panel heights to try (0: the configuration's own)")
+    ap.add_argument("--context", action="store_true",
+                    help="also time torch.matmul (+ eager bias/GELU) on each shape")
+    ap.add_argument("--write", action="store_true", help="rewrite csrc/tg_configs.inc")
+    ap.add_argument("--json", default=None)
+    args = ap.parse_args(argv)
+    sys.path.insert(0, os.path.dirname(HERE))
+    import torch
+    from tensor_core_gemm_fp16_b200 import binding
+
+    names = list(DEFAULT_SHAPES) if args.shapes == ["all"] else args.shapes
+    configs = args.configs if args.configs is not None else list(range(binding.tg_num_configs()))
+    results = []
+    for name in names:
+        M, N, K, epi = DEFAULT_SHAPES[name]
+        r = sweep_shape(torch, binding, name, M, N, K, epi, args.reps, args.warmup, configs,
+                        tuple(args.group_m), args.context)
+        results.append(r)
+        print(f"== {name} ({M}x{N}x{K}, epilogue {epi}) best config {r['best']} "
+              f"group_m {r['best_group_m']}")
+        if r["library_ms"] is not None:
+            print(f"   torch/cuBLAS (context) {r['library_ms'] * 1e3:9.1f} us  "
+                  f"{2.0 * M * N * K / (r['library_ms'] * 1e-3) / 1e12:7.1f} TFLOP/s")
+        for row in r["rows"]:
+            if "ms" in row:
+                print(f"   cfg {row['config']:2d}  BM{row['block_m']:4d} BN{row['block_n']:4d} "
+                      f"st{row['stages']} pair{row['cta_pair']} g{row['group_m']:2d} "
+                      f"ew{row['epi_warps']}  {row['ms'] * 1e3:9.1f} us  "
+                      f"{row['tflops']:7.1f} TFLOP/s")
+            else:
+                print(f"   cfg {row['config']:2d}  {row['error']}")
+        sys.stdout.flush()
+    if args.json:
+        with open(args.json, "w") as f:
+            json.dump(results, f, indent=1)
+    if args.write:
+        write_table(results)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

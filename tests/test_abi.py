@@ -87,6 +87,12 @@ def test_host_validation_rejects_bad_calls_without_a_device():
     assert g(0x10000, 0x20000, 0x40004, 0x40000, 4, 4, 4, 1, None) == binding.TG_ERR_INVALID_ARG
     # bad options
     assert binding.tg_gemm_ex(0x1000, 0x2000, None, 0x30000, 4, 4, 4, 9) == binding.TG_ERR_INVALID_ARG
+    assert binding.tg_gemm_ex(0x1000, 0x2000, None, 0x30000, 4, 4, 4, 0, config_id=99) == \
+        binding.TG_ERR_INVALID_ARG
+    assert binding.tg_gemm_ex(0x1000, 0x2000, None, 0x30000, 4, 4, 4, 0, group_m=65) == \
+        binding.TG_ERR_INVALID_ARG
+    assert binding.tg_gemm_ex(0x1000, 0x2000, None, 0x30000, 4, 4, 4, 0, inject=7) == \
+        binding.TG_ERR_INVALID_ARG
 
 
 def test_empty_problems_are_ok_without_a_device():

@@ -97,11 +97,15 @@ def test_rank1_closed_form():
 # ---------------------------------------------------------------- epilogue
 
 def test_gelu_epilogue_within_one_ulp():
-    """A = 0, so C = fp16(GELU(bias)); sweep bias over [-8, 8]."""
-    M, N, K = 128, 4096, 64
+    """A = 0, so C = fp16(GELU(bias)): every finite fp16 value in [-16, 16]
+    as the bias (all inputs the epilogue can see from a zero product)."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = bits.view(np.float16)
+    keep = np.isfinite(vals) & (np.abs(vals.astype(np.float64)) <= 16)
+    bias = torch.from_numpy(vals[keep].copy())
+    M, N, K = 128, bias.numel(), 64
     A = torch.zeros(M, K, dtype=torch.float16)
     B = torch.zeros(K, N, dtype=torch.float16)
-    bias = torch.linspace(-8, 8, N).to(torch.float16)
     C = run_gpu(A, B, bias, GELU)
     ref = run_oracle(A, B, bias, oracle.EPI_BIAS_GELU)
     exp_bits = oracle.double_to_half_rne(ref).astype(np.int32)
@@ -244,10 +248,11 @@ def test_host_entry_matches_device_entry():
     assert torch.equal(c_host, c_dev)
 
 
-def test_bounded_wait_reports_timeout_and_context_survives():
+@pytest.mark.parametrize("config_id", [0, 2])
+def test_bounded_wait_reports_timeout_and_context_survives(config_id):
     """A skipped operand load makes the consumer's bounded wait expire: the
     kernel exits cleanly, the host reads TG_ERR_TIMEOUT, and the next call
-    works."""
+    works (config 0: CTA pair, config 2: single CTA)."""
     dev = torch.device("cuda:0")
     A, B, bias = wl.make_inputs(256, 512, 512, seed=1000, bias=True)
     a, b, bb = A.to(dev), B.to(dev), bias.to(dev)
@@ -255,7 +260,7 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     stream = torch.cuda.current_stream().cuda_stream
     assert binding.tg_gemm_check_error(stream) == binding.TG_OK
     st = binding.tg_gemm_ex(a.data_ptr(), b.data_ptr(), bb.data_ptr(), c.data_ptr(), 256, 512, 512,
-                            GELU, wait_limit_ns=50_000_000,
+                            GELU, config_id=config_id, wait_limit_ns=50_000_000,
                             inject=binding.TG_INJECT_SKIP_FIRST_LOAD, stream=stream)
     assert st == binding.TG_OK
     assert binding.tg_gemm_check_error(stream) == binding.TG_ERR_TIMEOUT

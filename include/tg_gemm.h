@@ -75,7 +75,9 @@ typedef enum {
     TG_ERR_LAUNCH = 4,             /* a kernel launch failed                    */
     TG_ERR_TIMEOUT = 5,            /* a device-side bounded wait expired        */
     TG_ERR_OOM = 6,                /* a temporary could not be allocated        */
-    TG_ERR_CUDA = 7                /* another CUDA runtime error                */
+    TG_ERR_CUDA = 7,               /* another CUDA runtime error                */
+    TG_ERR_SCRATCH_LIMIT = 8       /* tg_gemm_noalloc: the repacking scratch the
+                                      problem needs exceeds TG_NOALLOC_SCRATCH_BYTES */
 } tg_status_t;
 
 /*
@@ -197,6 +199,43 @@ int tg_gemm_launch_count(const void *A, const void *B, const void *bias, const v
  * error, else TG_OK.
  */
 tg_status_t tg_gemm_check_error(void *stream);
+
+/*
+ * tg_gemm_noalloc -- tg_gemm for callers that must not allocate device memory.
+ *
+ * The paper has no counterpart to this entry point; it exists for users of
+ * this library.  tg_gemm repacks operands whose base address or row pitch is
+ * not a multiple of 16 bytes into a temporary taken from a stream-ordered
+ * memory pool.  Some callers cannot have the library allocate at all: a
+ * serving engine that has handed nearly all of HBM to its own allocator (a
+ * KV cache, a caching allocator) and must not see a foreign allocation fail
+ * or fragment its arena, or a latency-critical loop that must not enter the
+ * driver's allocator.  This entry point performs the same computation with
+ * the same arguments, results and conventions as tg_gemm, but takes any
+ * repacking scratch from a fixed array compiled into the library
+ * (file-scope __device__ memory of TG_NOALLOC_SCRATCH_BYTES bytes, which
+ * every GPU that loads the library holds until the process exits).  It
+ * calls no cudaMalloc, cudaFree, memory-pool or other allocating routine.
+ *
+ *   - The scratch a call needs is 2*M*K8 bytes (rounded up to 256) when A
+ *     must be repacked plus 2*K*N8 bytes when B must be repacked (K8, N8 =
+ *     K, N rounded up to a multiple of 8); aligned operands need none.  A
+ *     call needing more than TG_NOALLOC_SCRATCH_BYTES returns
+ *     TG_ERR_SCRATCH_LIMIT and launches nothing.
+ *   - The first call on each device performs a one-time set-up on that
+ *     device (it looks up the device address of the scratch array, which may
+ *     load the library's GPU module); make that first call before any stream
+ *     capture begins on the device.
+ *   - Every call on a device shares the one scratch array and it keeps the
+ *     last call's contents (the repacking kernels rewrite every byte a call
+ *     reads, padding included).  Calls whose kernels can overlap on the GPU,
+ *     e.g. on two streams without ordering between them, race on it: order
+ *     them on one stream or with events.
+ */
+#define TG_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+tg_status_t tg_gemm_noalloc(const void *A, const void *B, const void *bias, void *C,
+                            int64_t M, int64_t N, int64_t K, int epilogue, void *stream);
 
 /* Static, human-readable name of a status code (never NULL). */
 const char *tg_status_string(int status);

@@ -29,6 +29,7 @@ TG_ERR_LAUNCH = 4
 TG_ERR_TIMEOUT = 5
 TG_ERR_OOM = 6
 TG_ERR_CUDA = 7
+TG_ERR_SCRATCH_LIMIT = 8
 
 TG_INJECT_SKIP_FIRST_LOAD = 1
 
@@ -89,6 +90,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.tg_gemm_select_config.restype = c_int
     lib.tg_gemm_launch_count.argtypes = [vp, vp, vp, vp, i64, i64, i64, c_int]
     lib.tg_gemm_launch_count.restype = c_int
+    lib.tg_gemm_noalloc.argtypes = [vp, vp, vp, vp, i64, i64, i64, c_int, vp]
+    lib.tg_gemm_noalloc.restype = c_int
     lib.tg_version.argtypes = []
     lib.tg_version.restype = c_int
     _lib = lib
@@ -107,6 +110,20 @@ def header_symbols(header: str = HEADER):
 def tg_gemm(A: int, B: int, bias: int | None, C: int, M: int, N: int, K: int, epilogue: int,
             stream: int | None = None) -> int:
     return load().tg_gemm(A, B, bias, C, M, N, K, epilogue, stream)
+
+
+def tg_gemm_noalloc(A: int, B: int, bias: int | None, C: int, M: int, N: int, K: int,
+                    epilogue: int, stream: int | None = None) -> int:
+    """tg_gemm without any allocation: repacking scratch comes from the
+    library's fixed device array (see tg_gemm.h)."""
+    return load().tg_gemm_noalloc(A, B, bias, C, M, N, K, epilogue, stream)
+
+
+def noalloc_scratch_bytes(header: str = HEADER) -> int:
+    """TG_NOALLOC_SCRATCH_BYTES as declared in include/tg_gemm.h."""
+    m = re.search(r"#define\s+TG_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)",
+                  open(header).read())
+    return int(m.group(1)) << int(m.group(2))
 
 
 def tg_gemm_ex(A, B, bias, C, M, N, K, epilogue, config_id=-1, wait_limit_ns=0, inject=0,

@@ -524,6 +524,9 @@ const char *tg_status_string(int status)
     case TG_ERR_TIMEOUT: return "TG_ERR_TIMEOUT: a device-side wait expired";
     case TG_ERR_OOM: return "TG_ERR_OOM: temporary allocation failed";
     case TG_ERR_CUDA: return "TG_ERR_CUDA: CUDA runtime error";
+    case TG_ERR_SCRATCH_LIMIT:
+        return "TG_ERR_SCRATCH_LIMIT: tg_gemm_noalloc needs more repacking scratch than "
+               "TG_NOALLOC_SCRATCH_BYTES";
     default: return "unknown tg_status_t";
     }
 }
@@ -531,3 +534,149 @@ const char *tg_status_string(int status)
 int tg_version(void) { return 100; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// tg_gemm_noalloc: the same GEMM with the repacking scratch taken from a fixed
+// file-scope device array instead of a memory pool.  Nothing here allocates.
+
+static __device__ __align__(256) unsigned char g_tg_noalloc_scratch[TG_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+struct NoallocDevice {
+    bool init = false;
+    tg_status_t status = TG_OK;
+    int num_sms = 0;
+    unsigned *error_word = nullptr;
+    unsigned char *scratch = nullptr;   // device address of g_tg_noalloc_scratch
+};
+NoallocDevice g_noalloc_devices[kMaxDevices];
+
+// One-time set-up per device, with that device current: the device checks
+// of device_state() (without its memory pool) plus the device addresses of
+// the error word and of the scratch array.  In host code the array's name is
+// only a host-side stand-in; cudaGetSymbolAddress gives the address to pass.
+tg_status_t noalloc_device(NoallocDevice **out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return TG_ERR_UNSUPPORTED_DEVICE;
+    }
+    std::lock_guard<std::mutex> lock(g_mutex);
+    NoallocDevice &d = g_noalloc_devices[dev];
+    if (!d.init) {
+        d.init = true;
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            major != 10 || minor != 0) {
+            d.status = TG_ERR_UNSUPPORTED_DEVICE;
+        } else if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) !=
+                       cudaSuccess ||
+                   cudaGetSymbolAddress(reinterpret_cast<void **>(&d.error_word),
+                                        g_tg_error_word) != cudaSuccess ||
+                   cudaGetSymbolAddress(reinterpret_cast<void **>(&d.scratch),
+                                        g_tg_noalloc_scratch) != cudaSuccess ||
+                   !d.scratch) {
+            d.status = TG_ERR_CUDA;
+        }
+        if (d.status == TG_OK && !g_encode) {
+            cudaDriverEntryPointQueryResult q;
+            void *fn = nullptr;
+            if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000,
+                                                 cudaEnableDefault, &q) != cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || !fn)
+                d.status = TG_ERR_CUDA;
+            else
+                g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+        cudaGetLastError();
+    }
+    *out = &d;
+    return d.status;
+}
+
+tg_status_t gemm_noalloc_impl(const void *A, const void *B, const void *bias, void *C, int64_t M,
+                              int64_t N, int64_t K, int epilogue, cudaStream_t stream)
+{
+    tg_status_t st = validate(A, B, bias, C, M, N, K, epilogue);
+    if (st != TG_OK || M == 0 || N == 0) return st;
+    // Scratch needed by the repacking step, checked before any device call.
+    const bool a_direct = aligned(A, 16) && (K % 8 == 0);
+    const bool b_direct = aligned(B, 16) && (N % 8 == 0);
+    const int64_t lda = a_direct ? K : (K + 7) / 8 * 8;
+    const int64_t ldb = b_direct ? N : (N + 7) / 8 * 8;
+    const size_t a_bytes = (a_direct || K == 0) ? 0 : static_cast<size_t>(2 * M * lda);
+    const size_t a_pad = (a_bytes + 255) / 256 * 256;
+    const size_t b_bytes = (b_direct || K == 0) ? 0 : static_cast<size_t>(2 * K * ldb);
+    if (a_pad + b_bytes > static_cast<size_t>(TG_NOALLOC_SCRATCH_BYTES)) return TG_ERR_SCRATCH_LIMIT;
+
+    NoallocDevice *dev = nullptr;
+    st = noalloc_device(&dev);
+    if (st != TG_OK) return st;
+    if (epilogue == TG_EPILOGUE_NONE) bias = nullptr;
+    if (K == 0) return launch_k0(bias, C, M, N, epilogue, stream, dev->num_sms);
+
+    const int cfg_id = choose_config(M, N, K, epilogue, dev->num_sms);
+    const KernelConfig &cfg = kConfigs[cfg_id];
+    const void *Aeff = A, *Beff = B;
+    if (!a_direct) {
+        st = launch_pack(A, M, K, dev->scratch, lda, stream, dev->num_sms);
+        if (st != TG_OK) return st;
+        Aeff = dev->scratch;
+    }
+    if (!b_direct) {
+        unsigned char *bdst = dev->scratch + a_pad;
+        st = launch_pack(B, K, N, bdst, ldb, stream, dev->num_sms);
+        if (st != TG_OK) return st;
+        Beff = bdst;
+    }
+
+    const bool c_rows16 = aligned(C, 16) && (N % 8 == 0);
+    const int store = c_rows16 ? cfg.store_pref : tg::kStoreScalar;
+    CUtensorMap ta, tb, tc;
+    std::memset(&tc, 0, sizeof(tc));
+    if (!encode_2d(&ta, Aeff, K, M, 2 * lda, tg::kBlockK, tg::kBlockM,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&tb, Beff, N, K, 2 * ldb, tg::kBChunkN, tg::kBlockK,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        (store == tg::kStoreTma &&
+         !encode_2d(&tc, C, N, M, 2 * N, tg::kStoreCols, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
+        return TG_ERR_CUDA;
+
+    tg::GemmParams p;
+    p.bias = static_cast<const __half *>(bias);
+    p.C = static_cast<__half *>(C);
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.ldc = N;
+    p.num_m_tiles = static_cast<int>(ceil_div(M, cfg.info.block_m));
+    p.num_n_tiles = static_cast<int>(ceil_div(N, cfg.info.block_n));
+    p.num_k_blocks = static_cast<int>(ceil_div(K, tg::kBlockK));
+    p.num_tiles = p.num_m_tiles * p.num_n_tiles;
+    p.group_m = cfg.info.group_m;
+    p.inject = 0;
+    p.bias_vec = (bias && aligned(bias, 16)) ? 1 : 0;
+    p.wait_limit_ns = kDefaultWaitLimitNs;
+    p.error_word = dev->error_word;
+    const int units = cfg.info.cta_pair ? dev->num_sms / 2 : dev->num_sms;
+    const int grid = static_cast<int>(std::min<int64_t>(p.num_tiles, units)) *
+                     (cfg.info.cta_pair ? 2 : 1);
+    if (cfg.fn[epilogue][store == tg::kStoreScalar ? 0 : 1](ta, tb, tc, p, grid, stream) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_LAUNCH;
+    }
+    return TG_OK;
+}
+
+}  // namespace
+
+extern "C" tg_status_t tg_gemm_noalloc(const void *A, const void *B, const void *bias, void *C,
+                                       int64_t M, int64_t N, int64_t K, int epilogue,
+                                       void *stream)
+{
+    return gemm_noalloc_impl(A, B, bias, C, M, N, K, epilogue, static_cast<cudaStream_t>(stream));
+}

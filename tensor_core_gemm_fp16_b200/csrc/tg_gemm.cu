@@ -50,13 +50,13 @@ cudaError_t ensure_smem_attr(Kernel kern, int smem, std::atomic<uint64_t> &attr_
     return cudaSuccess;
 }
 
-template <int BN, int ST_REQ, int EPI, bool PAIR, int EW, int STORE>
+template <int BN, int BK, int ST_REQ, int EPI, bool PAIR, int EW, int STORE>
 cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc,
                         const tg::GemmParams &p, int grid, cudaStream_t stream)
 {
-    constexpr int ST = tg::FittedStages<BN, ST_REQ, PAIR, EW, STORE>::value;
-    using S = tg::KernelShape<BN, ST, PAIR, EW, STORE>;
-    auto kern = tg::gemm_persistent_kernel<BN, ST, EPI, PAIR, EW, STORE>;
+    constexpr int ST = tg::FittedStages<BN, BK, ST_REQ, PAIR, EW, STORE>::value;
+    using S = tg::KernelShape<BN, BK, ST, PAIR, EW, STORE>;
+    auto kern = tg::gemm_persistent_kernel<BN, BK, ST, EPI, PAIR, EW, STORE>;
     static std::atomic<uint64_t> attr_set{0};
     cudaError_t e = ensure_smem_attr(kern, S::kDynamicBytes, attr_set);
     if (e != cudaSuccess) return e;
@@ -86,33 +86,31 @@ struct KernelConfig {
     LaunchFn fn[3][2];    // [epilogue][0: element stores, 1: store_pref]
 };
 
-#define TG_FNS(BN, ST, PAIR, EW, SP)                                                        \
+#define TG_FNS(BN, BK, ST, PAIR, EW, SP)                                                    \
     {                                                                                       \
-        {launch_gemm<BN, ST, 0, PAIR, EW, tg::kStoreScalar>,                                \
-         launch_gemm<BN, ST, 0, PAIR, EW, SP>},                                             \
-            {launch_gemm<BN, ST, 1, PAIR, EW, tg::kStoreScalar>,                            \
-             launch_gemm<BN, ST, 1, PAIR, EW, SP>},                                         \
-            {launch_gemm<BN, ST, 2, PAIR, EW, tg::kStoreScalar>,                            \
-             launch_gemm<BN, ST, 2, PAIR, EW, SP>},                                         \
+        {launch_gemm<BN, BK, ST, 0, PAIR, EW, tg::kStoreScalar>,                            \
+         launch_gemm<BN, BK, ST, 0, PAIR, EW, SP>},                                         \
+            {launch_gemm<BN, BK, ST, 1, PAIR, EW, tg::kStoreScalar>,                        \
+             launch_gemm<BN, BK, ST, 1, PAIR, EW, SP>},                                     \
+            {launch_gemm<BN, BK, ST, 2, PAIR, EW, tg::kStoreScalar>,                        \
+             launch_gemm<BN, BK, ST, 2, PAIR, EW, SP>},                                     \
     }
 
-#define TG_CONFIG(ID, BN, ST, PAIR, EW, SP, GROUP)                                          \
-    {{ID, 128 * ((PAIR) ? 2 : 1), BN, 64, ST, (PAIR) ? 1 : 0, GROUP, EW}, SP,               \
-     TG_FNS(BN, ST, PAIR, EW, SP)}
+#define TG_CONFIG(ID, BN, BK, ST, PAIR, EW, SP, GROUP)                                      \
+    {{ID, 128 * ((PAIR) ? 2 : 1), BN, BK, ST, (PAIR) ? 1 : 0, GROUP, EW}, SP,               \
+     TG_FNS(BN, BK, ST, PAIR, EW, SP)}
 
-// {id, BN, stages, CTA pair, epilogue warps, store mode for aligned C, group_m}
+// {id, BN, BK, stages, CTA pair, epilogue warps, store mode for aligned C, group_m}
 const KernelConfig kConfigs[] = {
-    TG_CONFIG(0, 256, 6, true, 8, tg::kStoreTma, 8),
-    TG_CONFIG(1, 128, 8, true, 8, tg::kStoreTma, 8),
-    TG_CONFIG(2, 256, 4, false, 8, tg::kStoreTma, 8),
-    TG_CONFIG(3, 128, 6, false, 8, tg::kStoreTma, 8),
-    TG_CONFIG(4, 64, 8, false, 4, tg::kStoreTma, 8),
-    TG_CONFIG(5, 256, 6, true, 4, tg::kStoreTma, 8),
-    TG_CONFIG(6, 256, 6, true, 8, tg::kStoreTma, 16),
-    TG_CONFIG(7, 256, 4, false, 4, tg::kStoreVec, 8),
-    TG_CONFIG(8, 256, 7, true, 4, tg::kStoreVec, 8),
-    TG_CONFIG(9, 256, 5, true, 4, tg::kStoreTma, 8),
-    TG_CONFIG(10, 256, 4, true, 4, tg::kStoreTma, 8),
+    TG_CONFIG(0, 256, 128, 3, true, 8, tg::kStoreTma, 8),
+    TG_CONFIG(1, 256, 64, 6, true, 8, tg::kStoreTma, 8),
+    TG_CONFIG(2, 128, 64, 8, true, 8, tg::kStoreTma, 8),
+    TG_CONFIG(3, 256, 64, 4, false, 8, tg::kStoreTma, 8),
+    TG_CONFIG(4, 128, 64, 6, false, 8, tg::kStoreTma, 8),
+    TG_CONFIG(5, 64, 64, 8, false, 4, tg::kStoreTma, 8),
+    TG_CONFIG(6, 256, 128, 3, true, 4, tg::kStoreTma, 8),
+    TG_CONFIG(7, 256, 64, 6, true, 4, tg::kStoreTma, 8),
+    TG_CONFIG(8, 256, 64, 4, false, 4, tg::kStoreVec, 8),
 };
 constexpr int kNumConfigs = sizeof(kConfigs) / sizeof(kConfigs[0]);
 
@@ -132,7 +130,7 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 int rule_config(int64_t M, int64_t N, int num_sms)
 {
     struct Cand { int id; double eff; };
-    const Cand cands[] = {{0, 1.0}, {1, 0.93}, {3, 0.85}, {4, 0.7}};
+    const Cand cands[] = {{0, 1.0}, {2, 0.93}, {4, 0.85}, {5, 0.7}};
     const int sms = num_sms > 1 ? num_sms : 148;
     int best = 0;
     double best_score = 0;
@@ -358,9 +356,9 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
     const int store = c_rows16 ? cfg.store_pref : tg::kStoreScalar;
     CUtensorMap ta, tb, tc;
     std::memset(&tc, 0, sizeof(tc));
-    if (!encode_2d(&ta, Aeff, K, M, 2 * lda, tg::kBlockK, tg::kBlockM,
+    if (!encode_2d(&ta, Aeff, K, M, 2 * lda, tg::kAtomK, tg::kBlockM,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&tb, Beff, N, K, 2 * ldb, tg::kBChunkN, tg::kBlockK,
+        !encode_2d(&tb, Beff, N, K, 2 * ldb, tg::kBChunkN, cfg.info.block_k,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
         (store == tg::kStoreTma &&
          !encode_2d(&tc, C, N, M, 2 * N, tg::kStoreCols, 32, CU_TENSOR_MAP_SWIZZLE_64B))) {
@@ -377,7 +375,7 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
     p.ldc = N;
     p.num_m_tiles = static_cast<int>(ceil_div(M, cfg.info.block_m));
     p.num_n_tiles = static_cast<int>(ceil_div(N, bn));
-    p.num_k_blocks = static_cast<int>(ceil_div(K, tg::kBlockK));
+    p.num_k_blocks = static_cast<int>(ceil_div(K, cfg.info.block_k));
     p.num_tiles = p.num_m_tiles * p.num_n_tiles;
     p.group_m = (opts && opts->group_m > 0) ? opts->group_m : cfg.info.group_m;
     p.inject = opts ? opts->inject : 0;
@@ -637,9 +635,9 @@ tg_status_t gemm_noalloc_impl(const void *A, const void *B, const void *bias, vo
     const int store = c_rows16 ? cfg.store_pref : tg::kStoreScalar;
     CUtensorMap ta, tb, tc;
     std::memset(&tc, 0, sizeof(tc));
-    if (!encode_2d(&ta, Aeff, K, M, 2 * lda, tg::kBlockK, tg::kBlockM,
+    if (!encode_2d(&ta, Aeff, K, M, 2 * lda, tg::kAtomK, tg::kBlockM,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&tb, Beff, N, K, 2 * ldb, tg::kBChunkN, tg::kBlockK,
+        !encode_2d(&tb, Beff, N, K, 2 * ldb, tg::kBChunkN, cfg.info.block_k,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
         (store == tg::kStoreTma &&
          !encode_2d(&tc, C, N, M, 2 * N, tg::kStoreCols, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
@@ -654,7 +652,7 @@ tg_status_t gemm_noalloc_impl(const void *A, const void *B, const void *bias, vo
     p.ldc = N;
     p.num_m_tiles = static_cast<int>(ceil_div(M, cfg.info.block_m));
     p.num_n_tiles = static_cast<int>(ceil_div(N, cfg.info.block_n));
-    p.num_k_blocks = static_cast<int>(ceil_div(K, tg::kBlockK));
+    p.num_k_blocks = static_cast<int>(ceil_div(K, cfg.info.block_k));
     p.num_tiles = p.num_m_tiles * p.num_n_tiles;
     p.group_m = cfg.info.group_m;
     p.inject = 0;

@@ -31,11 +31,10 @@
 namespace tg {
 
 constexpr int kBlockM = 128;   // rows of A (and of C) per CTA: one TMEM lane per row
-constexpr int kBlockK = 64;    // K per stage: 64 fp16 = one 128-byte swizzle row
+constexpr int kAtomK = 64;     // K of one A box: 64 fp16 = one 128-byte swizzle row
 constexpr int kBChunkN = 64;   // B is loaded in 64-column boxes (128 bytes wide)
 constexpr int kUmmaK = 16;     // K of one kind::f16 MMA instruction
-constexpr int kABytesStage = kBlockM * kBlockK * 2;   // 16 KiB
-constexpr int kBChunkBytes = kBChunkN * kBlockK * 2;  // 8 KiB
+constexpr int kAAtomBytes = kBlockM * kAtomK * 2;     // one 128 x 64 A box: 16 KiB
 constexpr int kStoreCols = 32;                        // C columns per TMEM load / TMA store box
 constexpr int kStoreBoxBytes = 32 * kStoreCols * 2;   // 32 rows x 32 fp16 = 2 KiB
 
@@ -68,20 +67,26 @@ struct GemmParams {
 
 // Compile-time shape of one kernel variant.
 //   BN        output columns per tile (the MMA's N)
+//   BK        K per pipeline stage (64 or 128): A arrives as BK/64 boxes of
+//             128 x 64, each B chunk as one 64-column x BK box
 //   STAGES    depth of the shared-memory operand ring
 //   PAIR      two CTAs of a cluster run one cta_group::2 MMA on a 256-row tile;
 //             each loads 128 rows of A and BN/2 columns of B
 //   EPI_WARPS 4 or 8 warps drain TMEM (8: two per lane quarter, halving columns)
-template <int BN, int STAGES, bool PAIR, int EPI_WARPS, int STORE>
+template <int BN, int BK, int STAGES, bool PAIR, int EPI_WARPS, int STORE>
 struct KernelShape {
     static_assert(BN == 64 || BN == 128 || BN == 256, "BN must be 64, 128 or 256");
+    static_assert(BK == 64 || BK == 128, "BK must be 64 or 128");
     static_assert(!PAIR || BN >= 128, "a CTA pair needs BN >= 128");
     static_assert(EPI_WARPS == 4 || EPI_WARPS == 8, "4 or 8 epilogue warps");
     static constexpr int kCG = PAIR ? 2 : 1;
     static constexpr int kTileM = kBlockM * kCG;
     static constexpr int kCtaN = BN / kCG;                       // B columns loaded per CTA
     static constexpr int kBChunks = kCtaN / kBChunkN;
-    static constexpr int kStageBytes = kABytesStage + kBChunks * kBChunkBytes;
+    static constexpr int kAAtoms = BK / kAtomK;
+    static constexpr int kABytes = kAAtoms * kAAtomBytes;       // A part of a stage
+    static constexpr int kBChunkBytes = kBChunkN * BK * 2;      // one B box
+    static constexpr int kStageBytes = kABytes + kBChunks * kBChunkBytes;
     static constexpr uint32_t kTxBytes = kCG * kStageBytes;      // both CTAs land on the leader
     static constexpr int kRingBytes = STAGES * kStageBytes;
     static constexpr int kStagingBytes = STORE != kStoreVec ? EPI_WARPS * 2 * kStoreBoxBytes : 0;
@@ -106,14 +111,15 @@ constexpr int kMaxDynamicSmem = 232448;   // 227 KiB: the sm_100 per-block opt-i
 // STAGES, reduced by one when this store mode's staging buffers would push
 // the block past the shared-memory limit (the element-store fallback of a
 // configuration tuned for direct vector stores).
-template <int BN, int STAGES, bool PAIR, int EPI_WARPS, int STORE>
+template <int BN, int BK, int STAGES, bool PAIR, int EPI_WARPS, int STORE>
 struct FittedStages {
     static constexpr int value =
-        KernelShape<BN, STAGES, PAIR, EPI_WARPS, STORE>::kDynamicBytes <= kMaxDynamicSmem
+        KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, STORE>::kDynamicBytes <= kMaxDynamicSmem
             ? STAGES
             : STAGES - 1;
-    static_assert(KernelShape<BN, value, PAIR, EPI_WARPS, STORE>::kDynamicBytes <= kMaxDynamicSmem,
-                  "shared-memory budget exceeded");
+    static_assert(
+        KernelShape<BN, BK, value, PAIR, EPI_WARPS, STORE>::kDynamicBytes <= kMaxDynamicSmem,
+        "shared-memory budget exceeded");
 };
 
 // Tile index -> (m tile, n tile), walking group_m M-tiles per panel so that
@@ -207,13 +213,13 @@ __device__ __forceinline__ uint4 epilogue8(const uint32_t *r, const float (&b)[8
 //   warp EPI_WARPS        TMA producer (one lane)
 //   warp EPI_WARPS + 1    TMEM allocator; MMA issuer (one lane; the leader CTA
 //                         of a pair issues for both)
-template <int BN, int STAGES, int EPI, bool PAIR, int EPI_WARPS, int STORE>
-__global__ void __launch_bounds__(KernelShape<BN, STAGES, PAIR, EPI_WARPS, STORE>::kThreads, 1)
+template <int BN, int BK, int STAGES, int EPI, bool PAIR, int EPI_WARPS, int STORE>
+__global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, STORE>::kThreads, 1)
     gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmC, const GemmParams p)
 {
-    using S = KernelShape<BN, STAGES, PAIR, EPI_WARPS, STORE>;
+    using S = KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, STORE>;
     constexpr int CG = S::kCG;
     constexpr uint32_t kIdesc = idesc_f16_f32(S::kTileM, BN);
 
@@ -295,24 +301,30 @@ __global__ void __launch_bounds__(KernelShape<BN, STAGES, PAIR, EPI_WARPS, STORE
                         skip_next = false;   // injected fault: this stage never fills
                     } else {
                         const uint32_t a_dst = smem_base + stage * S::kStageBytes;
-                        const uint32_t b_dst = a_dst + kABytesStage;
+                        const uint32_t b_dst = a_dst + S::kABytes;
                         if (leader) {
                             mbar_arrive_expect_tx(&full_bar[stage], S::kTxBytes);
                             pending[stage] = 1u + phase;
                         }
                         if constexpr (PAIR) {
                             const uint32_t bar = map_to_cta(smem_u32(&full_bar[stage]), 0);
-                            tma_load_2d_pair(a_dst, &tmA, bar, kb * kBlockK, a_row);
+#pragma unroll
+                            for (int q = 0; q < S::kAAtoms; ++q)
+                                tma_load_2d_pair(a_dst + q * kAAtomBytes, &tmA, bar,
+                                                 kb * BK + q * kAtomK, a_row);
 #pragma unroll
                             for (int j = 0; j < S::kBChunks; ++j)
-                                tma_load_2d_pair(b_dst + j * kBChunkBytes, &tmB, bar,
-                                                 b_col + j * kBChunkN, kb * kBlockK);
+                                tma_load_2d_pair(b_dst + j * S::kBChunkBytes, &tmB, bar,
+                                                 b_col + j * kBChunkN, kb * BK);
                         } else {
-                            tma_load_2d(a_dst, &tmA, &full_bar[stage], kb * kBlockK, a_row);
+#pragma unroll
+                            for (int q = 0; q < S::kAAtoms; ++q)
+                                tma_load_2d(a_dst + q * kAAtomBytes, &tmA, &full_bar[stage],
+                                            kb * BK + q * kAtomK, a_row);
 #pragma unroll
                             for (int j = 0; j < S::kBChunks; ++j)
-                                tma_load_2d(b_dst + j * kBChunkBytes, &tmB, &full_bar[stage],
-                                            b_col + j * kBChunkN, kb * kBlockK);
+                                tma_load_2d(b_dst + j * S::kBChunkBytes, &tmB, &full_bar[stage],
+                                            b_col + j * kBChunkN, kb * BK);
                         }
                     }
                     if (++stage == STAGES) {
@@ -338,6 +350,19 @@ __global__ void __launch_bounds__(KernelShape<BN, STAGES, PAIR, EPI_WARPS, STORE
             int acc = 0;
             uint32_t acc_phase = 0;
             bool issued_any = false;
+            // Result of a non-blocking probe of full_bar[stage] made while the
+            // previous stage's MMAs were being issued: when it already saw the
+            // data, the blocking wait (and its latency) is skipped.
+            bool ready = false;
+            // Shared-memory descriptors of stage 0; stage s adds s * kStageBytes
+            // to the 14-bit start-address field (units of 16 B, no carry out for
+            // addresses below 256 KiB).
+            // A: K-major, 128-B swizzle; 8-row groups 1024 B apart.
+            const uint64_t a_desc0 = smem_desc_sw128(smem_base, 16, 1024);
+            // B: MN-major, 128-B swizzle; 64-column chunks kBChunkBytes apart
+            // (leading), 8-k-row groups 1024 B apart (stride).
+            const uint64_t b_desc0 =
+                smem_desc_sw128(smem_base + S::kABytes, S::kBChunkBytes, 1024);
             for (int tile = unit; tile < p.num_tiles; tile += num_units) {
                 if (!mbar_wait_bounded(&tmem_empty_bar[acc], acc_phase ^ 1u, abort_flag, limit,
                                        p.error_word, kErrMmaWait))
@@ -346,26 +371,30 @@ __global__ void __launch_bounds__(KernelShape<BN, STAGES, PAIR, EPI_WARPS, STORE
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
                 bool ok = true;
                 for (int kb = 0; kb < p.num_k_blocks; ++kb) {
-                    if (!mbar_wait_bounded(&full_bar[stage], phase, abort_flag, limit,
-                                           p.error_word, kErrMmaWait)) {
+                    if (!ready && !mbar_wait_bounded(&full_bar[stage], phase, abort_flag, limit,
+                                                     p.error_word, kErrMmaWait)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint32_t a_addr = smem_base + stage * S::kStageBytes;
-                    const uint32_t b_addr = a_addr + kABytesStage;
-                    // A: K-major, 128-B swizzle; 8-row groups 1024 B apart.
-                    const uint64_t a_desc = smem_desc_sw128(a_addr, 16, 1024);
-                    // B: MN-major, 128-B swizzle; 64-column chunks kBChunkBytes
-                    // apart (leading), 8-k-row groups 1024 B apart (stride).
-                    const uint64_t b_desc = smem_desc_sw128(b_addr, kBChunkBytes, 1024);
+                    const int next_stage = stage + 1 == STAGES ? 0 : stage + 1;
+                    const uint32_t next_phase = next_stage == 0 ? phase ^ 1u : phase;
+                    ready = mbar_test_wait(&full_bar[next_stage], next_phase);
+                    const uint64_t stage_off =
+                        static_cast<uint64_t>((stage * S::kStageBytes) >> 4);
 #pragma unroll
-                    for (int kk = 0; kk < kBlockK / kUmmaK; ++kk) {
-                        // K step inside the swizzle row: +32 B for A; +16 rows
-                        // (2 KiB) for B, added to the start-address field (16 B units).
-                        const uint64_t a_k = a_desc + static_cast<uint64_t>((kk * kUmmaK * 2) >> 4);
+                    for (int kk = 0; kk < BK / kUmmaK; ++kk) {
+                        // K step: for A, the next 32 B inside a 128-B swizzle row,
+                        // moving to the next 128 x 64 box every 4 steps; for B,
+                        // the next 16 k-rows (2 KiB).
+                        constexpr int kStepsPerAtom = kAtomK / kUmmaK;
+                        const uint64_t a_k =
+                            a_desc0 + stage_off +
+                            static_cast<uint64_t>(((kk / kStepsPerAtom) * kAAtomBytes +
+                                                   (kk % kStepsPerAtom) * kUmmaK * 2) >>
+                                                  4);
                         const uint64_t b_k =
-                            b_desc + static_cast<uint64_t>((kk * kUmmaK * 128) >> 4);
+                            b_desc0 + stage_off + static_cast<uint64_t>((kk * kUmmaK * 128) >> 4);
                         mma_f16_ss<CG>(d_tmem, a_k, b_k, kIdesc, (kb | kk) != 0 ? 1u : 0u);
                     }
                     issued_any = true;
@@ -374,10 +403,8 @@ __global__ void __launch_bounds__(KernelShape<BN, STAGES, PAIR, EPI_WARPS, STORE
                         mma_commit_pair_multicast(&empty_bar[stage], 0x3);
                     else
                         mma_commit<1>(&empty_bar[stage]);
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    stage = next_stage;
+                    phase = next_phase;
                 }
                 if (!ok) break;
                 // accumulator ready for the epilogue (of both CTAs)

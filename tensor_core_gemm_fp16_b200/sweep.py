@@ -97,7 +97,7 @@ def time_library(torch, a, b, bias, epi, reps, warmup, flush):
 
 
 def sweep_shape(torch, binding, name, M, N, K, epi, reps, warmup, configs, group_ms=(0,),
-                context=False):
+                context=False, rounds=5):
     dev = torch.device("cuda")
     g = torch.Generator(device=dev).manual_seed(1234)
     a = torch.randn(M, K, device=dev, generator=g).half()
@@ -110,7 +110,7 @@ def sweep_shape(torch, binding, name, M, N, K, epi, reps, warmup, configs, group
     small = 2 * (M * K + K * N + M * N) <= L2_BYTES
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if small else None
     rows = []
-    lib_ms = time_library(torch, a, b, bias, epi, reps, warmup, flush) if context else None
+    candidates = []
     for cfg, gm in [(c, g) for c in configs for g in group_ms]:
         info = dict(binding.tg_config_info(cfg))
         if gm:
@@ -127,9 +127,25 @@ def sweep_shape(torch, binding, name, M, N, K, epi, reps, warmup, configs, group
         if not rel < 2e-2:
             rows.append({"config": cfg, "error": f"numerically wrong (rel {rel:.2e})"})
             continue
-        ms = time_config(torch, binding, a, b, bias, c, M, N, K, epi, cfg, reps, warmup, flush,
-                         gm)
-        rows.append({"config": cfg, "group_m_override": gm, "ms": ms, "tflops": 2.0 * M * N * K / (ms * 1e-3) / 1e12,
+        candidates.append((cfg, gm, info, rel))
+    # Interleaved rounds: every candidate (and the library context) is timed
+    # once per round, so slow drifts of the GPU's clock (power, temperature)
+    # touch all of them alike; each result is the median over rounds of the
+    # per-round medians.
+    per_round = {i: [] for i in range(len(candidates))}
+    lib_rounds = []
+    per = max(1, reps // rounds)
+    for _ in range(rounds):
+        if context:
+            lib_rounds.append(time_library(torch, a, b, bias, epi, per, warmup, flush))
+        for i, (cfg, gm, info, rel) in enumerate(candidates):
+            per_round[i].append(time_config(torch, binding, a, b, bias, c, M, N, K, epi, cfg,
+                                            per, warmup, flush, gm))
+    lib_ms = statistics.median(lib_rounds) if context else None
+    for i, (cfg, gm, info, rel) in enumerate(candidates):
+        ms = statistics.median(per_round[i])
+        rows.append({"config": cfg, "group_m_override": gm, "ms": ms,
+                     "tflops": 2.0 * M * N * K / (ms * 1e-3) / 1e12,
                      "rel_err": rel, **{k: info[k] for k in ("block_m", "block_n", "stages",
                                                            "cta_pair", "group_m", "epi_warps")}})
     ok = [r for r in rows if "ms" in r]
@@ -168,7 +184,9 @@ def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__,
                                  formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--shapes", nargs="*", default=["all"])
-    ap.add_argument("--reps", type=int, default=20)
+    ap.add_argument("--reps", type=int, default=30, help="launches per candidate in total")
+    ap.add_argument("--rounds", type=int, default=5,
+                    help="interleaved rounds over all candidates (reps are split among them)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--configs", type=int, nargs="*", default=None)
     ap.add_argument("--group-m", type=int, nargs="*", default=[0],
@@ -188,7 +206,7 @@ def main(argv=None):
     for name in names:
         M, N, K, epi = DEFAULT_SHAPES[name]
         r = sweep_shape(torch, binding, name, M, N, K, epi, args.reps, args.warmup, configs,
-                        tuple(args.group_m), args.context)
+                        tuple(args.group_m), args.context, args.rounds)
         results.append(r)
         print(f"== {name} ({M}x{N}x{K}, epilogue {epi}) best config {r['best']} "
               f"group_m {r['best_group_m']}")

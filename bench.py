@@ -142,6 +142,21 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+def max_over_ranks(x: float, world: int, dist=None, device=None) -> float:
+    """Maximum of x over all ranks (the job's time is its slowest rank's)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(flops_per_rank: int, world: int, step_ms: float) -> float:
+    """Whole-job TFLOP/s: every rank's flops over the slowest rank's step time."""
+    return world * flops_per_rank / (step_ms * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------------------- oracle timing
 
 def oracle_rows_for(w, a, b, bb, target_s: float):
@@ -275,12 +290,8 @@ def run_ours(args, w, rank, world):
         if world > 1:
             dist.barrier(device_ids=[local])
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def reduce_max(x: float) -> float:
+        return max_over_ranks(x, world, dist, dev)
 
     # ---------------------------------------------------------------- device-resident timing
     s = time_workload(torch, binding, w, args.steps, args.warmup, dev, stream, flush_buf)
@@ -303,8 +314,8 @@ def run_ours(args, w, rank, world):
     kernel_ms = statistics.mean(launch_ms)
     region_ms = s["t_start"].elapsed_time(s["t_end"])
     step_ms = region_ms / args.steps if s["big"] else sum(launch_ms) / args.steps
-    step_ms = max_over_ranks(step_ms)
-    value = world * w.flops / (step_ms * 1e-3) / 1e12
+    step_ms = reduce_max(step_ms)
+    value = job_value(w.flops, world, step_ms)
     launches_per_step = binding.tg_gemm_launch_count(*s["args"])
     st = binding.tg_gemm_check_error(stream.cuda_stream)
     if st != binding.TG_OK:
@@ -326,7 +337,7 @@ def run_ours(args, w, rank, world):
             s2["launch"]()
             s2["ev"][i][1].record(stream)
         torch.cuda.synchronize(dev)
-        ms2 = max_over_ranks(statistics.mean(e0.elapsed_time(e1) for e0, e1 in s2["ev"]))
+        ms2 = reduce_max(statistics.mean(e0.elapsed_time(e1) for e0, e1 in s2["ev"]))
         also.append({"workload": name, "value": world * w2.flops / (ms2 * 1e-3) / 1e12,
                      "unit": UNIT, "ms_per_step": ms2,
                      "pct_of_fp16_dense_peak_nominal":
@@ -335,7 +346,7 @@ def run_ours(args, w, rank, world):
         del s2
 
     # ---------------------------------------------------------------- end to end (host buffers)
-    e2e = run_e2e(torch, binding, w, s, args, dev, stream, barrier, max_over_ranks, world) \
+    e2e = run_e2e(torch, binding, w, s, args, dev, stream, barrier, reduce_max, world) \
         if not args.no_e2e else None
 
     # ---------------------------------------------------------------- roofline + CPU baseline

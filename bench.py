@@ -241,7 +241,7 @@ def workload_config(w, extra=None):
     return cfg
 
 
-def time_workload(torch, binding, w, steps, warmup, dev, stream, flush_buf):
+def time_workload(torch, binding, w, steps, warmup, dev, stream, flush_buf, config_id=-1):
     """Device-resident inputs; returns dict with per-launch and per-step times."""
     from tensor_core_gemm_fp16_b200 import workloads as wl
     A, B, bias = wl.workload_inputs(w)
@@ -253,7 +253,10 @@ def time_workload(torch, binding, w, steps, warmup, dev, stream, flush_buf):
     big = 2 * (w.M * w.K + w.K * w.N + w.M * w.N) > L2_BYTES
 
     def launch():
-        st = binding.tg_gemm(*args, stream.cuda_stream)
+        if config_id < 0:
+            st = binding.tg_gemm(*args, stream.cuda_stream)
+        else:
+            st = binding.tg_gemm_ex(*args, config_id=config_id, stream=stream.cuda_stream)
         if st != binding.TG_OK:
             raise binding.TgError(st, "tg_gemm")
 
@@ -294,7 +297,8 @@ def run_ours(args, w, rank, world):
         return max_over_ranks(x, world, dist, dev)
 
     # ---------------------------------------------------------------- device-resident timing
-    s = time_workload(torch, binding, w, args.steps, args.warmup, dev, stream, flush_buf)
+    s = time_workload(torch, binding, w, args.steps, args.warmup, dev, stream, flush_buf,
+                      args.config)
     sampler = ClockSampler(torch, local)
     barrier()
     torch.cuda.synchronize(dev)
@@ -424,8 +428,9 @@ def finish(torch, binding, dist, w, s, args, rank, world, dev, step_ms, value, k
         dist.destroy_process_group()
     if rank != 0:
         return 0
-    kcfg = binding.tg_gemm_select_config(w.M, w.N, w.K, w.epilogue,
-                                         torch.cuda.get_device_properties(dev).multi_processor_count)
+    kcfg = binding.tg_config_info(args.config) if args.config >= 0 else \
+        binding.tg_gemm_select_config(w.M, w.N, w.K, w.epilogue,
+                                      torch.cuda.get_device_properties(dev).multi_processor_count)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
@@ -460,6 +465,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--config", type=int, default=-1,
+                    help="force a kernel configuration id for the main workload (profiling)")
     ap.add_argument("--shape", type=int, nargs=3, metavar=("M", "N", "K"),
                     help="custom fused workload (bias + GELU, N(0,1) inputs, B scaled by "
                          "1/sqrt(K), seed 7) instead of --workload; for profiling cases")

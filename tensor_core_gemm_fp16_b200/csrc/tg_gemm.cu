@@ -66,15 +66,23 @@ cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const CUte
     cfg.blockDim = dim3(S::kThreads, 1, 1);
     cfg.dynamicSmemBytes = S::kDynamicBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    // Programmatic stream serialisation: the kernel's prologue may overlap the
+    // previous kernel in the stream; it waits (griddepcontrol.wait) before
+    // touching global memory.
+    cudaLaunchAttribute attr[2];
+    unsigned n_attr = 0;
+    attr[n_attr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n_attr].val.programmaticStreamSerializationAllowed = 1;
+    ++n_attr;
     if (PAIR) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        attr[n_attr].id = cudaLaunchAttributeClusterDimension;
+        attr[n_attr].val.clusterDim.x = 2;
+        attr[n_attr].val.clusterDim.y = 1;
+        attr[n_attr].val.clusterDim.z = 1;
+        ++n_attr;
     }
+    cfg.attrs = attr;
+    cfg.numAttrs = n_attr;
     e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

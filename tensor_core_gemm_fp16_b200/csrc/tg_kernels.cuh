@@ -136,28 +136,45 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int 
     nt = r / rows;
 }
 
-// GELU(v) = v * Phi(v), Phi the standard normal CDF, Phi(v) = erfc(-v/sqrt 2)/2.
-// erfc(z) for z = |v|/sqrt(2) >= 0 is evaluated as t * exp(-z^2 + P(t)),
-// t = 1/(1 + z/2), the Chebyshev-type form of Numerical Recipes (2nd ed.,
-// section 6.2) with our own degree-7 fit of P (csrc/fit_erfc.py: max error
-// of P 6.2e-7 on z in [0, 9]); Phi(-|v|) = erfc(z)/2 and Phi(|v|) = 1 - that.
-// In fp32 the relative error of GELU stays below 6e-6 for |v| <= 8.5 (fp16's
-// half-ulp is 2.4e-4), and the tail keeps full relative accuracy (no 1 + erf
-// cancellation).  About 20 instructions per element.
+__device__ __forceinline__ float rcp_approx(float x)
+{
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ float exp2_approx(float x)
+{
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// GELU(v) = v * Phi(v), Phi the standard normal CDF.  With a = |v| and the
+// tail T = Phi(-a) = erfc(a / sqrt 2) / 2, GELU(v) = max(v, 0) - a * T for
+// either sign of v.  T uses the Chebyshev-type form of erfc of Numerical
+// Recipes (2nd ed., section 6.2), erfc(z) = t exp(-z^2 + P(t)), t = 1/(1+z/2),
+// written with a base-2 exponent and the 1/2 folded into the polynomial:
+//   T = t * 2^(-a^2 log2(e)/2 + Q(t)),  t = 1 / (1 + a / (2 sqrt 2)),
+// Q of degree 6 fitted by csrc/fit_erfc.py (our coefficients; max error of Q
+// 8.2e-6 in log2 units on z in [0, 9]).  In fp32 with the approximate
+// reciprocal and exponential the relative error of GELU stays near 1e-5 for
+// |v| <= 8.5 (fp16's half-ulp is 2.4e-4) and the tail keeps full relative
+// accuracy.  14 instructions per element, two of them MUFU.
 __device__ __forceinline__ float gelu_erf(float v)
 {
-    const float z = fabsf(v) * 0.70710678118654752f;
-    const float t = __fdividef(1.0f, fmaf(0.5f, z, 1.0f));
-    float p = -1.811217638e-01f;
-    p = fmaf(p, t, 7.227813026e-01f);
-    p = fmaf(p, t, -9.495873675e-01f);
-    p = fmaf(p, t, 3.007620395e-01f);
-    p = fmaf(p, t, -1.279667006e-02f);
-    p = fmaf(p, t, 3.855720234e-01f);
-    p = fmaf(p, t, 9.999567273e-01f);
-    p = fmaf(p, t, -1.265566907e+00f);
-    const float tail = 0.5f * t * __expf(fmaf(-z, z, p));   // Phi(-|v|)
-    return v * (v > 0.0f ? 1.0f - tail : tail);
+    const float a = fabsf(v);
+    const float t = rcp_approx(fmaf(a, 0.353553390593273762f, 1.0f));
+    float p = -3.214579429e-02f;
+    p = fmaf(p, t, 4.489113895e-01f);
+    p = fmaf(p, t, -1.198654278e+00f);
+    p = fmaf(p, t, 8.162180034e-01f);
+    p = fmaf(p, t, 3.145696625e-01f);
+    p = fmaf(p, t, 1.479150420e+00f);
+    p = fmaf(p, t, -2.828041197e+00f);
+    const float x = fmaf(-a * 0.721347520444481703f, a, p);   // log2(e)/2 = 0.7213...
+    const float tail = t * exp2_approx(x);
+    return fmaf(-a, tail, fmaxf(v, 0.0f));
 }
 
 template <int EPI>
@@ -169,28 +186,46 @@ __device__ __forceinline__ float apply_epilogue(float acc, float beta)
     return v;
 }
 
-// Eight consecutive bias values as floats (zeros past N or without bias).
+// The 32 bias values of columns [col0, col0 + 32) as packed fp16 (zeros past N
+// or without bias).  Issued ahead of their use so that the load latency
+// overlaps other work: the first chunk's before the accumulator wait, each
+// next chunk's while the current one is processed.
 template <int EPI>
-__device__ __forceinline__ void load_bias8(const __half *bias, int64_t col, int64_t N, bool vec,
-                                           float (&b)[8])
+__device__ __forceinline__ void fetch_bias32(const __half *bias, int64_t col0, int64_t N, bool vec,
+                                             uint4 (&out)[4])
 {
-    if (EPI == kEpiNone || bias == nullptr) {
+    if (EPI == kEpiNone || bias == nullptr || col0 >= N) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) b[e] = 0.f;
+        for (int q = 0; q < 4; ++q) out[q] = make_uint4(0u, 0u, 0u, 0u);
         return;
     }
-    if (vec && col + 8 <= N) {
-        uint4 u = __ldg(reinterpret_cast<const uint4 *>(bias + col));
-        const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+    if (vec && col0 + 32 <= N) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(bias + col0);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 f = __half22float2(h[e]);
-            b[2 * e] = f.x;
-            b[2 * e + 1] = f.y;
-        }
+        for (int q = 0; q < 4; ++q) out[q] = __ldg(src + q);
     } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) b[e] = (col + e < N) ? __half2float(bias[col + e]) : 0.f;
+        for (int q = 0; q < 4; ++q) {
+            __half h[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int64_t col = col0 + q * 8 + e;
+                h[e] = col < N ? bias[col] : __ushort_as_half(static_cast<unsigned short>(0));
+            }
+            out[q] = *reinterpret_cast<const uint4 *>(h);
+        }
+    }
+}
+
+// Eight packed fp16 bias values -> floats.
+__device__ __forceinline__ void unpack_bias8(const uint4 &u, float (&b)[8])
+{
+    const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(h[e]);
+        b[2 * e] = f.x;
+        b[2 * e + 1] = f.y;
     }
 }
 
@@ -271,6 +306,10 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
     if (PAIR) cluster_sync();   // peer barriers initialised before any remote use
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
+    // Everything above touches only this CTA's own resources, so it may overlap
+    // the previous kernel in the stream; A, B, bias and C are touched only after
+    // that kernel has completed.
+    grid_dependency_wait();
 
     const uint32_t smem_base = smem_u32(smem);
     const uint64_t limit = p.wait_limit_ns;
@@ -439,6 +478,9 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
         for (int tile = unit; tile < p.num_tiles; tile += num_units) {
             int mt, nt;
             tile_coords(tile, p.num_m_tiles, p.num_n_tiles, p.group_m, mt, nt);
+            uint4 bias_next[4];
+            fetch_bias32<EPI>(p.bias, static_cast<int64_t>(nt) * BN + chunk0 * kStoreCols, p.N,
+                              bias_vec, bias_next);
             int ok = 0;
             if (lane == 0)
                 ok = mbar_wait_bounded(&tmem_full_bar[acc], acc_phase, abort_flag, limit,
@@ -461,6 +503,11 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                 const int64_t col0 = static_cast<int64_t>(nt) * BN + c * kStoreCols;
                 // warp-uniform: the chunk lies entirely past N, or all 32 rows past M
                 if (col0 >= p.N || row0 >= p.M) break;
+                uint4 bias_cur[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) bias_cur[q] = bias_next[q];
+                if (c + 1 < chunk0 + S::kChunksPerWarp)
+                    fetch_bias32<EPI>(p.bias, col0 + kStoreCols, p.N, bias_vec, bias_next);
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * kStoreCols), r);
                 tmem_wait_ld();
@@ -475,7 +522,7 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         float b[8];
-                        load_bias8<EPI>(p.bias, col0 + q * 8, p.N, bias_vec, b);
+                        unpack_bias8(bias_cur[q], b);
                         const uint4 u = epilogue8<EPI>(r + q * 8, b);
                         const uint32_t phys = static_cast<uint32_t>(q) ^ ((lane >> 1) & 3u);
                         const uint32_t addr = buf + lane * 64u + phys * 16u;
@@ -497,7 +544,7 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             float b[8];
-                            load_bias8<EPI>(p.bias, col0 + q * 8, p.N, bias_vec, b);
+                            unpack_bias8(bias_cur[q], b);
                             const uint4 u = epilogue8<EPI>(r + q * 8, b);
                             if (full) {
                                 *reinterpret_cast<uint4 *>(crow + col0 + q * 8) = u;
@@ -517,7 +564,7 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         float b[8];
-                        load_bias8<EPI>(p.bias, col0 + q * 8, p.N, false, b);
+                        unpack_bias8(bias_cur[q], b);
                         const uint4 u = epilogue8<EPI>(r + q * 8, b);
                         const uint32_t phys = static_cast<uint32_t>(q) ^ ((lane >> 1) & 3u);
                         const uint32_t addr = buf + lane * 64u + phys * 16u;
@@ -564,6 +611,8 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
 
     // Teardown: every role has returned (all waits are bounded), so no thread
     // still reads TMEM and no MMA or copy tracked by this CTA is in flight.
+    // The next kernel in the stream may start its prologue now.
+    grid_launch_dependents();
     tc_fence_before_sync();
     __syncthreads();
     if (PAIR) cluster_sync();   // the leader's MMAs into this CTA's TMEM are done

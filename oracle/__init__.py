@@ -13,7 +13,11 @@ numpy arrays.  Every function cites the passage it follows in the C file:
   (thecryptopost.io), the make_matmul kernel (fp16 A[M,K], B[K,N], C[M,N],
   fp32 accumulator);
 * the bias + GELU epilogue -- the same tutorial (ainovat.com), fused-epilogue
-  section (bias add and GELU on the accumulator before the one output write).
+  section (bias add and GELU on the accumulator before the one output write);
+* the tanh approximation of GELU -- Hendrycks & Gimpel, "Gaussian Error
+  Linear Units", section 2;
+* the row softmax epilogue -- the same tutorial (ainovat.com), row-wise
+  softmax section (per-row max and sum, then normalisation).
 
 Pins (tests/test_oracle_pins.py) hold it to closed forms, exact rational
 arithmetic, exhaustive codec checks against numpy, and scipy's normal CDF.
@@ -29,6 +33,8 @@ import numpy as np
 EPI_NONE = 0
 EPI_BIAS = 1
 EPI_BIAS_GELU = 2
+EPI_BIAS_GELU_TANH = 3
+EPI_BIAS_SOFTMAX = 4
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "tg_oracle.c")
@@ -64,6 +70,7 @@ def _load():
         lib.tgo_half_to_double_n.argtypes = [u16p, i64, f64p]
         lib.tgo_double_to_half_rne_n.argtypes = [f64p, i64, u16p]
         lib.tgo_gelu_n.argtypes = [f64p, i64, f64p]
+        lib.tgo_gelu_tanh_n.argtypes = [f64p, i64, f64p]
         lib.tgo_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -124,7 +131,8 @@ def gemm_int_exact(A, B, bias=None, epilogue: int = EPI_NONE) -> np.ndarray:
     """Exact result for integer-valued inputs, correctly rounded to fp16.
 
     Returns the (M, N) uint16 fp16 bit patterns.  Raises OracleError if any
-    input is not an integer below 2048 in magnitude, or for BIAS_GELU.
+    input is not an integer below 2048 in magnitude, or for an epilogue other
+    than NONE and BIAS.
     """
     A, B, bias = _bits(A), _bits(B), _bits(bias)
     M, K = A.shape
@@ -159,6 +167,14 @@ def gelu(x) -> np.ndarray:
     x = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
     out = np.empty(x.shape, dtype=np.float64)
     _load().tgo_gelu_n(_ptr(x, ctypes.c_double), x.size, _ptr(out, ctypes.c_double))
+    return out
+
+
+def gelu_tanh(x) -> np.ndarray:
+    """The oracle's tanh-approximation GELU in double, elementwise."""
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    out = np.empty(x.shape, dtype=np.float64)
+    _load().tgo_gelu_tanh_n(_ptr(x, ctypes.c_double), x.size, _ptr(out, ctypes.c_double))
     return out
 
 

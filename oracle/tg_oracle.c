@@ -22,6 +22,13 @@
  *     Source: same tutorial (ainovat.com), fused-epilogue section: the bias
  *     add and the GELU are applied to the accumulator before the single
  *     write of the output.
+ *   BIAS_GELU_TANH: g(v) = v/2 (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))),
+ *     the tanh approximation of GELU (Hendrycks & Gimpel, "Gaussian Error
+ *     Linear Units", section 2).
+ *   BIAS_SOFTMAX: row-wise softmax of z = A.B + bias over the N columns of
+ *     each row, ref[i][j] = exp(z_ij - max_j z_ij) / sum_j exp(z_ij - max_j z_ij).
+ *     Source: same tutorial (ainovat.com), the row-wise softmax section (max
+ *     and sum reductions per row, normalisation), here as a GEMM epilogue.
  *
  * Every fp16 x fp16 product is exact in double (11 + 11 significant bits),
  * and a double sum of at most 2^31 such terms keeps an error far below the
@@ -39,6 +46,7 @@
  * Loop order is i-k-j over a double accumulator row; rows are independent
  * and split across OpenMP threads.  No blocking, no reordering beyond that.
  */
+#define _GNU_SOURCE
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -50,6 +58,8 @@
 #define TGO_EPI_NONE 0
 #define TGO_EPI_BIAS 1
 #define TGO_EPI_BIAS_GELU 2
+#define TGO_EPI_BIAS_GELU_TANH 3
+#define TGO_EPI_BIAS_SOFTMAX 4
 
 #define TGO_OK 0
 #define TGO_ERR_ARG 1
@@ -103,10 +113,34 @@ double tgo_gelu(double v)
     return 0.5 * v * erfc(-v / sqrt(2.0));
 }
 
+/* tanh approximation of GELU. */
+double tgo_gelu_tanh(double v)
+{
+    const double c = sqrt(2.0 / M_PI);
+    return 0.5 * v * (1.0 + tanh(c * (v + 0.044715 * v * v * v)));
+}
+
+/* Elementwise epilogues (all but BIAS_SOFTMAX, which needs the whole row). */
 static double apply_epilogue(double acc, double beta, int epilogue)
 {
     double v = acc + beta;
-    return epilogue == TGO_EPI_BIAS_GELU ? tgo_gelu(v) : v;
+    if (epilogue == TGO_EPI_BIAS_GELU) return tgo_gelu(v);
+    if (epilogue == TGO_EPI_BIAS_GELU_TANH) return tgo_gelu_tanh(v);
+    return v;
+}
+
+/* Row softmax in place: z <- exp(z - max z) / sum exp(z - max z). */
+static void softmax_row(double *z, int64_t N)
+{
+    if (N <= 0) return;
+    double m = z[0];
+    for (int64_t j = 1; j < N; ++j) m = z[j] > m ? z[j] : m;
+    double s = 0.0;
+    for (int64_t j = 0; j < N; ++j) {
+        z[j] = exp(z[j] - m);
+        s += z[j];
+    }
+    for (int64_t j = 0; j < N; ++j) z[j] /= s;
 }
 
 static int check_args(const uint16_t *A, const uint16_t *B, const uint16_t *bias,
@@ -114,7 +148,7 @@ static int check_args(const uint16_t *A, const uint16_t *B, const uint16_t *bias
 {
     (void)bias;
     if (M < 0 || N < 0 || K < 0) return TGO_ERR_ARG;
-    if (epilogue < TGO_EPI_NONE || epilogue > TGO_EPI_BIAS_GELU) return TGO_ERR_ARG;
+    if (epilogue < TGO_EPI_NONE || epilogue > TGO_EPI_BIAS_SOFTMAX) return TGO_ERR_ARG;
     if ((M > 0 && K > 0 && !A) || (K > 0 && N > 0 && !B)) return TGO_ERR_ARG;
     return TGO_OK;
 }
@@ -142,6 +176,7 @@ static void one_row(const double *Ad, const double *Bd, const double *biasd,
         double beta = (epilogue != TGO_EPI_NONE && biasd) ? biasd[j] : 0.0;
         ref_row[j] = apply_epilogue(ref_row[j], beta, epilogue);
     }
+    if (epilogue == TGO_EPI_BIAS_SOFTMAX) softmax_row(ref_row, N);
 }
 
 /*
@@ -201,7 +236,7 @@ int tgo_gemm_int_exact(const uint16_t *A, const uint16_t *B, const uint16_t *bia
 {
     int st = check_args(A, B, bias, M, N, K, epilogue);
     if (st) return st;
-    if (epilogue == TGO_EPI_BIAS_GELU) return TGO_ERR_NOT_INTEGER;
+    if (epilogue != TGO_EPI_NONE && epilogue != TGO_EPI_BIAS) return TGO_ERR_NOT_INTEGER;
     if (M == 0 || N == 0) return TGO_OK;
     if (!C_bits) return TGO_ERR_ARG;
     int64_t *Ai = (int64_t *)malloc((size_t)(M * (K > 0 ? K : 1)) * sizeof(int64_t));
@@ -268,4 +303,9 @@ void tgo_double_to_half_rne_n(const double *x, int64_t n, uint16_t *out)
 void tgo_gelu_n(const double *x, int64_t n, double *out)
 {
     for (int64_t t = 0; t < n; ++t) out[t] = tgo_gelu(x[t]);
+}
+
+void tgo_gelu_tanh_n(const double *x, int64_t n, double *out)
+{
+    for (int64_t t = 0; t < n; ++t) out[t] = tgo_gelu_tanh(x[t]);
 }

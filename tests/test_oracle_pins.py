@@ -356,3 +356,100 @@ def test_bad_arguments():
         oracle.gemm(wl.to_bits(A), wl.to_bits(B), None, 7)
     with pytest.raises(oracle.OracleError):
         oracle.gemm(wl.to_bits(A), wl.to_bits(B), None, oracle.EPI_NONE, rows=[4])
+
+
+# ---------------------------------------------------------------------------
+# tanh-approximation GELU and the row-softmax epilogue
+
+
+def test_gelu_tanh_closed_point():
+    """Where sqrt(2/pi)(x + 0.044715 x^3) = atanh(1/2), g(x) = 3x/4 exactly."""
+    from scipy.optimize import brentq
+    c = math.sqrt(2 / math.pi)
+    target = math.atanh(0.5)
+    x = brentq(lambda t: c * (t + 0.044715 * t ** 3) - target, 0.0, 2.0, xtol=1e-15)
+    assert oracle.gelu_tanh([x])[0] == pytest.approx(0.75 * x, rel=1e-14)
+    y = brentq(lambda t: c * (t + 0.044715 * t ** 3) + target, -2.0, 0.0, xtol=1e-15)
+    assert oracle.gelu_tanh([y])[0] == pytest.approx(0.25 * y, rel=1e-14)
+
+
+def test_gelu_tanh_invariants_and_distance_to_erf_form():
+    x = np.linspace(-9, 9, 18001)
+    g = oracle.gelu_tanh(x)
+    assert np.allclose(g - oracle.gelu_tanh(-x), x, rtol=0, atol=1e-14)
+    assert oracle.gelu_tanh([0.0])[0] == 0.0
+    d = np.abs(g - x * ndtr(x))
+    assert d.max() < 5e-4 and d.max() > 1e-4     # close to, and distinct from, erf GELU
+
+
+def _scipy_softmax_rows(z):
+    from scipy.special import softmax
+    return softmax(z, axis=1)
+
+
+def _exact_logits(A, B, bias):
+    a, b, bb = _dec(A), _dec(B), _dec(bias) if bias is not None else None
+    M, K = a.shape
+    N = b.shape[1]
+    z = np.empty((M, N))
+    for i in range(M):
+        for j in range(N):
+            s = sum(Fraction(a[i, k]) * Fraction(b[k, j]) for k in range(K))
+            if bb is not None:
+                s += Fraction(bb[j])
+            z[i, j] = float(s)
+    return z
+
+
+def test_softmax_matches_scipy_on_exact_logits():
+    for (M, N, K, seed) in [(3, 5, 4, 40), (4, 17, 9, 41), (2, 1, 3, 42)]:
+        A, B, bias = wl.make_inputs(M, N, K, seed=seed, bias=True)
+        got = _oracle_gemm(A, B, bias, oracle.EPI_BIAS_SOFTMAX)
+        assert np.allclose(got, _scipy_softmax_rows(_exact_logits(A, B, bias)), rtol=1e-13,
+                           atol=1e-300)
+
+
+def test_softmax_rows_sum_to_one_shift_invariance_and_uniform():
+    A, B, _ = wl.make_inputs(20, 40, 30, seed=43)
+    # bias on a 1/64 grid in [-2, 2): adding 4 keeps every value exact in fp16
+    bias = (torch.arange(40, dtype=torch.float32).mul(37).remainder(256).sub(128) / 64).half()
+    p = _oracle_gemm(A, B, bias, oracle.EPI_BIAS_SOFTMAX)
+    assert np.allclose(p.sum(axis=1), 1.0, rtol=0, atol=1e-14)
+    shifted = (bias.float() + 4.0).half()      # every value stays exact
+    assert np.array_equal(_dec(shifted), _dec(bias) + 4.0)
+    assert np.allclose(_oracle_gemm(A, B, shifted, oracle.EPI_BIAS_SOFTMAX), p, rtol=1e-12,
+                       atol=1e-300)
+    Z = torch.zeros(6, 8, dtype=torch.float16)
+    Bz = torch.zeros(8, 13, dtype=torch.float16)
+    assert np.allclose(_oracle_gemm(Z, Bz, None, oracle.EPI_BIAS_SOFTMAX), 1 / 13, rtol=1e-15)
+
+
+def test_softmax_large_logits_stay_finite():
+    # z up to ~2000: without subtracting the row maximum exp() would overflow
+    A = torch.full((2, 64), 30.0, dtype=torch.float16)
+    B = torch.ones(64, 5, dtype=torch.float16)
+    bias = torch.tensor([0.0, 1.0, 2.0, 3.0, -1.0], dtype=torch.float16)
+    p = _oracle_gemm(A, B, bias, oracle.EPI_BIAS_SOFTMAX)
+    e = np.exp(np.array([0.0, 1.0, 2.0, 3.0, -1.0]))
+    assert np.allclose(p, np.tile(e / e.sum(), (2, 1)), rtol=1e-14)
+
+
+def test_softmax_rank1_closed_form():
+    M, N, K = 4, 9, 32
+    u = np.array([2.0 ** -6, -2.0 ** -5, 2.0 ** -4, 0.0])
+    v = np.array([(-1) ** j * 2.0 ** (j % 4 - 3) for j in range(N)])
+    A = torch.tensor(np.repeat(u[:, None], K, axis=1), dtype=torch.float16)
+    B = torch.tensor(np.repeat(v[None, :], K, axis=0), dtype=torch.float16)
+    z = K * np.outer(u, v)
+    e = np.exp(z - z.max(axis=1, keepdims=True))
+    assert np.allclose(_oracle_gemm(A, B, None, oracle.EPI_BIAS_SOFTMAX),
+                       e / e.sum(axis=1, keepdims=True), rtol=1e-14)
+
+
+def test_softmax_k0_is_softmax_of_bias():
+    bias = torch.tensor([0.5, -1.0, 2.0, 0.0], dtype=torch.float16)
+    A = torch.zeros(3, 0, dtype=torch.float16)
+    B = torch.zeros(0, 4, dtype=torch.float16)
+    e = np.exp(_dec(bias) - 2.0)
+    assert np.allclose(_oracle_gemm(A, B, bias, oracle.EPI_BIAS_SOFTMAX),
+                       np.tile(e / e.sum(), (3, 1)), rtol=1e-15)

@@ -15,13 +15,26 @@
  *   section: float16 A (M,K), B (K,N), C (M,N) with a "float" accumulator
  *   fragment.
  *
- *   beta[j] = bias[j] (converted to fp32) for TG_EPILOGUE_BIAS and
- *   TG_EPILOGUE_BIAS_GELU, 0 for TG_EPILOGUE_NONE.  bias == NULL means a zero
- *   bias.  g is the identity, except for TG_EPILOGUE_BIAS_GELU where
- *   g(v) = v * Phi(v) = 0.5 * v * (1 + erf(v / sqrt(2))) (the erf form of
- *   GELU).  Definition: the same tutorial (ainovat.com), fused-epilogue
- *   section: bias add and GELU applied to the register-resident accumulator
- *   before the single write of the output.
+ *   beta[j] = bias[j] (converted to fp32) for every epilogue except
+ *   TG_EPILOGUE_NONE (beta = 0).  bias == NULL means a zero bias.  g is the
+ *   identity for NONE and BIAS, and for
+ *     TG_EPILOGUE_BIAS_GELU       g(v) = v * Phi(v) = 0.5 v (1 + erf(v / sqrt 2)),
+ *                                 the erf form of GELU.  Definition: the same
+ *                                 tutorial (ainovat.com), fused-epilogue
+ *                                 section: bias add and GELU applied to the
+ *                                 register-resident accumulator before the
+ *                                 single write of the output;
+ *     TG_EPILOGUE_BIAS_GELU_TANH  g(v) = 0.5 v (1 + tanh(sqrt(2/pi)(v + 0.044715 v^3))),
+ *                                 the tanh approximation (Hendrycks & Gimpel,
+ *                                 "Gaussian Error Linear Units", section 2);
+ *     TG_EPILOGUE_BIAS_SOFTMAX    not elementwise: each row of z = A.B + beta is
+ *                                 replaced by softmax(z_i) = exp(z_i - max z_i) /
+ *                                 sum exp(z_i - max z_i) over its N columns.
+ *                                 Definition: the same tutorial (ainovat.com),
+ *                                 row-wise softmax section (per-row max and sum
+ *                                 reductions in registers), here fused as a GEMM
+ *                                 epilogue.  Requires N <= 256 (one tile per
+ *                                 row), else TG_ERR_INVALID_ARG.
  *
  * Conventions shared by every entry point:
  *   - Pointers are DEVICE pointers on the current CUDA device (except where
@@ -62,9 +75,11 @@ extern "C" {
 #endif
 
 typedef enum {
-    TG_EPILOGUE_NONE = 0,      /* C = A.B                      */
-    TG_EPILOGUE_BIAS = 1,      /* C = A.B + bias               */
-    TG_EPILOGUE_BIAS_GELU = 2  /* C = GELU_erf(A.B + bias)     */
+    TG_EPILOGUE_NONE = 0,           /* C = A.B                          */
+    TG_EPILOGUE_BIAS = 1,           /* C = A.B + bias                   */
+    TG_EPILOGUE_BIAS_GELU = 2,      /* C = GELU_erf(A.B + bias)         */
+    TG_EPILOGUE_BIAS_GELU_TANH = 3, /* C = GELU_tanh(A.B + bias)        */
+    TG_EPILOGUE_BIAS_SOFTMAX = 4    /* C = row_softmax(A.B + bias), N <= 256 */
 } tg_epilogue_t;
 
 typedef enum {
@@ -140,7 +155,9 @@ tg_status_t tg_gemm_select_config(int64_t M, int64_t N, int64_t K, int epilogue,
  * tg_gemm_ex -- tg_gemm with explicit options.  `opts` may be NULL (same as
  * tg_gemm).  Used by the offline sweep and the tests.
  *
- *   config_id      -1: table choice; otherwise a configuration id
+ *   config_id      -1: table choice; otherwise a configuration id (for
+ *                  TG_EPILOGUE_BIAS_SOFTMAX it must have 4 epilogue warps and
+ *                  block_n >= N, else TG_ERR_INVALID_ARG)
  *   wait_limit_ns  0: default (2 s); else the limit of every device-side wait
  *   inject         0 normally.  TG_INJECT_SKIP_FIRST_LOAD makes the first CTA
  *                  skip one operand load, so that the consumer's bounded

@@ -20,6 +20,8 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "tg_gemm.h")
 TG_EPILOGUE_NONE = 0
 TG_EPILOGUE_BIAS = 1
 TG_EPILOGUE_BIAS_GELU = 2
+TG_EPILOGUE_BIAS_GELU_TANH = 3
+TG_EPILOGUE_BIAS_SOFTMAX = 4
 
 TG_OK = 0
 TG_ERR_INVALID_ARG = 1
@@ -33,7 +35,8 @@ TG_ERR_SCRATCH_LIMIT = 8
 
 TG_INJECT_SKIP_FIRST_LOAD = 1
 
-EPILOGUES = {"none": TG_EPILOGUE_NONE, "bias": TG_EPILOGUE_BIAS, "bias_gelu": TG_EPILOGUE_BIAS_GELU}
+EPILOGUES = {"none": TG_EPILOGUE_NONE, "bias": TG_EPILOGUE_BIAS, "bias_gelu": TG_EPILOGUE_BIAS_GELU,
+             "bias_gelu_tanh": TG_EPILOGUE_BIAS_GELU_TANH, "bias_softmax": TG_EPILOGUE_BIAS_SOFTMAX}
 
 
 class TgError(RuntimeError):

@@ -88,10 +88,23 @@ cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const CUte
     return cudaGetLastError();
 }
 
+// The row-softmax epilogue needs each epilogue thread to own a whole row,
+// i.e. 4 epilogue warps; other shapes have no softmax kernel.
+template <int BN, int BK, int ST, bool PAIR, int EW, int STORE>
+constexpr LaunchFn softmax_fn()
+{
+    if constexpr (EW == 4)
+        return launch_gemm<BN, BK, ST, TG_EPILOGUE_BIAS_SOFTMAX, PAIR, EW, STORE>;
+    else
+        return nullptr;
+}
+
+constexpr int kNumEpilogues = 5;
+
 struct KernelConfig {
     tg_config_t info;
-    int store_pref;       // store mode when C rows are 16-byte aligned
-    LaunchFn fn[3][2];    // [epilogue][0: element stores, 1: store_pref]
+    int store_pref;                  // store mode when C rows are 16-byte aligned
+    LaunchFn fn[kNumEpilogues][2];   // [epilogue][0: element stores, 1: store_pref]
 };
 
 #define TG_FNS(BN, BK, ST, PAIR, EW, SP)                                                    \
@@ -102,6 +115,10 @@ struct KernelConfig {
              launch_gemm<BN, BK, ST, 1, PAIR, EW, SP>},                                     \
             {launch_gemm<BN, BK, ST, 2, PAIR, EW, tg::kStoreScalar>,                        \
              launch_gemm<BN, BK, ST, 2, PAIR, EW, SP>},                                     \
+            {launch_gemm<BN, BK, ST, 3, PAIR, EW, tg::kStoreScalar>,                        \
+             launch_gemm<BN, BK, ST, 3, PAIR, EW, SP>},                                     \
+            {softmax_fn<BN, BK, ST, PAIR, EW, tg::kStoreScalar>(),                          \
+             softmax_fn<BN, BK, ST, PAIR, EW, SP>()},                                       \
     }
 
 #define TG_CONFIG(ID, BN, BK, ST, PAIR, EW, SP, GROUP)                                      \
@@ -158,8 +175,24 @@ int rule_config(int64_t M, int64_t N, int num_sms)
     return best;
 }
 
+// Softmax rows must fit one tile with whole rows per thread: 4 epilogue
+// warps and block_n >= N (N <= 256).
+bool softmax_capable(const tg_config_t &c, int64_t N) { return c.epi_warps == 4 && c.block_n >= N; }
+
 int choose_config(int64_t M, int64_t N, int64_t K, int epilogue, int num_sms)
 {
+    if (epilogue == TG_EPILOGUE_BIAS_SOFTMAX) {
+        for (const TableRow &r : kShapeTable)
+            if (r.M >= 0 && r.M == M && r.N == N && r.K == K && r.epilogue == epilogue &&
+                r.config >= 0 && r.config < kNumConfigs &&
+                softmax_capable(kConfigs[r.config].info, N))
+                return r.config;
+        // narrow rows: the 64-column single-CTA tile; otherwise the 256-column
+        // CTA pair when it fills the SM pairs, else the 256-column single CTA
+        if (N <= 64) return 5;
+        const int sms = num_sms > 1 ? num_sms : 148;
+        return ceil_div(M, 256) >= sms / 2 ? 6 : 8;
+    }
     for (const TableRow &r : kShapeTable)
         if (r.M >= 0 && r.M == M && r.N == N && r.K == K && (r.epilogue < 0 || r.epilogue == epilogue) &&
             r.config >= 0 && r.config < kNumConfigs)
@@ -260,14 +293,16 @@ bool overlaps(const void *a, int64_t a_bytes, const void *b, int64_t b_bytes)
 bool aligned(const void *p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
 
 constexpr int64_t kDimLimit = (1ll << 31) - 1;
+constexpr int64_t kSoftmaxMaxN = 256;
 
 // Checks that need no device.
 tg_status_t validate(const void *A, const void *B, const void *bias, const void *C, int64_t M,
                      int64_t N, int64_t K, int epilogue)
 {
-    if (epilogue < TG_EPILOGUE_NONE || epilogue > TG_EPILOGUE_BIAS_GELU) return TG_ERR_INVALID_ARG;
+    if (epilogue < TG_EPILOGUE_NONE || epilogue > TG_EPILOGUE_BIAS_SOFTMAX) return TG_ERR_INVALID_ARG;
     if (M < 0 || N < 0 || K < 0 || M > kDimLimit || N > kDimLimit || K > kDimLimit)
         return TG_ERR_INVALID_ARG;
+    if (epilogue == TG_EPILOGUE_BIAS_SOFTMAX && N > kSoftmaxMaxN) return TG_ERR_INVALID_ARG;
     if (M == 0 || N == 0) return TG_OK;
     if (!C || (K > 0 && (!A || !B))) return TG_ERR_INVALID_ARG;
     if (!aligned(C, 2) || (A && !aligned(A, 2)) || (B && !aligned(B, 2)) ||
@@ -292,8 +327,12 @@ tg_status_t launch_k0(const void *bias, void *C, int64_t M, int64_t N, int epilo
         tg::k0_epilogue_kernel<0><<<grid, 256, 0, stream>>>(b, c, M, N);
     else if (epilogue == TG_EPILOGUE_BIAS)
         tg::k0_epilogue_kernel<1><<<grid, 256, 0, stream>>>(b, c, M, N);
-    else
+    else if (epilogue == TG_EPILOGUE_BIAS_GELU)
         tg::k0_epilogue_kernel<2><<<grid, 256, 0, stream>>>(b, c, M, N);
+    else if (epilogue == TG_EPILOGUE_BIAS_GELU_TANH)
+        tg::k0_epilogue_kernel<3><<<grid, 256, 0, stream>>>(b, c, M, N);
+    else
+        tg::k0_epilogue_kernel<4><<<grid, 256, 0, stream>>>(b, c, M, N);
     return cudaGetLastError() == cudaSuccess ? TG_OK : TG_ERR_LAUNCH;
 }
 
@@ -329,6 +368,8 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
                            : choose_config(M, N, K, epilogue, dev->num_sms);
     const KernelConfig &cfg = kConfigs[cfg_id];
     const int bn = cfg.info.block_n;
+    if (epilogue == TG_EPILOGUE_BIAS_SOFTMAX && !softmax_capable(cfg.info, N))
+        return TG_ERR_INVALID_ARG;
 
     // TMA needs 16-byte aligned bases and pitches; otherwise repack.
     const bool a_direct = aligned(A, 16) && (K % 8 == 0);
@@ -437,7 +478,8 @@ tg_status_t tg_gemm_select_config(int64_t M, int64_t N, int64_t K, int epilogue,
                                   tg_config_t *out)
 {
     if (!out || M < 0 || N < 0 || K < 0 || epilogue < TG_EPILOGUE_NONE ||
-        epilogue > TG_EPILOGUE_BIAS_GELU || num_sms <= 0)
+        epilogue > TG_EPILOGUE_BIAS_SOFTMAX || num_sms <= 0 ||
+        (epilogue == TG_EPILOGUE_BIAS_SOFTMAX && N > kSoftmaxMaxN))
         return TG_ERR_INVALID_ARG;
     *out = kConfigs[choose_config(M, N, K, epilogue, num_sms)].info;
     return TG_OK;

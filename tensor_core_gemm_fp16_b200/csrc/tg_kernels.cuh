@@ -44,7 +44,7 @@ constexpr unsigned kErrMmaWait = 2u;
 constexpr unsigned kErrEpilogueWait = 4u;
 constexpr unsigned kErrDrain = 8u;
 
-enum : int { kEpiNone = 0, kEpiBias = 1, kEpiBiasGelu = 2 };
+enum : int { kEpiNone = 0, kEpiBias = 1, kEpiBiasGelu = 2, kEpiBiasGeluTanh = 3, kEpiBiasSoftmax = 4 };
 // How the epilogue writes C: element stores (any pitch), 16-byte stores
 // (16-byte aligned rows), or TMA stores from a swizzled staging tile.
 enum : int { kStoreScalar = 0, kStoreVec = 1, kStoreTma = 2 };
@@ -177,14 +177,27 @@ __device__ __forceinline__ float gelu_erf(float v)
     return fmaf(-a, tail, fmaxf(v, 0.0f));
 }
 
+// tanh approximation of GELU (Hendrycks & Gimpel, "Gaussian Error Linear
+// Units", section 2): v/2 (1 + tanh(u)), u = sqrt(2/pi) (v + 0.044715 v^3),
+// evaluated as v / (1 + exp(-2u)) = v / (1 + 2^(-2 log2(e) u)).
+__device__ __forceinline__ float gelu_tanh(float v)
+{
+    constexpr float k = 2.302208198115997f;   // 2 log2(e) sqrt(2/pi)
+    const float x = v * fmaf(v * v, -k * 0.044715f, -k);
+    return v * rcp_approx(1.0f + exp2_approx(x));
+}
+
 template <int EPI>
 __device__ __forceinline__ float apply_epilogue(float acc, float beta)
 {
     if (EPI == kEpiNone) return acc;
     float v = acc + beta;
     if (EPI == kEpiBiasGelu) v = gelu_erf(v);
+    if (EPI == kEpiBiasGeluTanh) v = gelu_tanh(v);
     return v;
 }
+
+constexpr float kLog2e = 1.4426950408889634f;
 
 // The 32 bias values of columns [col0, col0 + 32) as packed fp16 (zeros past N
 // or without bias).  Issued ahead of their use so that the load latency
@@ -230,15 +243,27 @@ __device__ __forceinline__ void unpack_bias8(const uint4 &u, float (&b)[8])
 }
 
 // Eight fp32 accumulators + bias -> epilogue -> eight fp16 packed in a uint4.
+// For the row softmax, sm_max / sm_scale are the row's maximum and
+// 1 / sum(exp(v - max)).
 template <int EPI>
-__device__ __forceinline__ uint4 epilogue8(const uint32_t *r, const float (&b)[8])
+__device__ __forceinline__ uint4 epilogue8(const uint32_t *r, const float (&b)[8],
+                                           float sm_max = 0.f, float sm_scale = 0.f)
 {
     uint4 u;
     __half2 *h = reinterpret_cast<__half2 *>(&u);
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
-        h[e] = __floats2half2_rn(apply_epilogue<EPI>(__uint_as_float(r[2 * e]), b[2 * e]),
-                                 apply_epilogue<EPI>(__uint_as_float(r[2 * e + 1]), b[2 * e + 1]));
+    for (int e = 0; e < 4; ++e) {
+        float lo, hi;
+        if constexpr (EPI == kEpiBiasSoftmax) {
+            lo = exp2_approx((__uint_as_float(r[2 * e]) + b[2 * e] - sm_max) * kLog2e) * sm_scale;
+            hi = exp2_approx((__uint_as_float(r[2 * e + 1]) + b[2 * e + 1] - sm_max) * kLog2e) *
+                 sm_scale;
+        } else {
+            lo = apply_epilogue<EPI>(__uint_as_float(r[2 * e]), b[2 * e]);
+            hi = apply_epilogue<EPI>(__uint_as_float(r[2 * e + 1]), b[2 * e + 1]);
+        }
+        h[e] = __floats2half2_rn(lo, hi);
+    }
     return u;
 }
 
@@ -498,6 +523,43 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
             __half *crow = p.C + row * p.ldc;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(acc * BN);
+            // Row softmax (4 epilogue warps: each thread owns its whole row): the
+            // row maximum and the sum of exp(v - max) over the valid columns,
+            // from two extra passes over the accumulator in TMEM.
+            float sm_max = 0.f, sm_scale = 0.f;
+            if constexpr (EPI == kEpiBiasSoftmax) {
+                static_assert(EPI_WARPS == 4, "the softmax epilogue needs whole rows per thread");
+                sm_max = -INFINITY;
+                float sum = 0.f;
+#pragma unroll 1
+                for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll 1
+                    for (int c = chunk0; c < chunk0 + S::kChunksPerWarp; ++c) {
+                        const int64_t col0 = static_cast<int64_t>(nt) * BN + c * kStoreCols;
+                        if (col0 >= p.N || row0 >= p.M) break;
+                        uint4 bq[4];
+                        fetch_bias32<EPI>(p.bias, col0, p.N, bias_vec, bq);
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * kStoreCols), r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            float b[8];
+                            unpack_bias8(bq[q], b);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                if (col0 + q * 8 + e >= p.N) continue;
+                                const float v = __uint_as_float(r[q * 8 + e]) + b[e];
+                                if (pass == 0)
+                                    sm_max = fmaxf(sm_max, v);
+                                else
+                                    sum += exp2_approx((v - sm_max) * kLog2e);
+                            }
+                        }
+                    }
+                }
+                sm_scale = rcp_approx(sum);
+            }
 #pragma unroll 1
             for (int c = chunk0; c < chunk0 + S::kChunksPerWarp; ++c) {
                 const int64_t col0 = static_cast<int64_t>(nt) * BN + c * kStoreCols;
@@ -523,7 +585,7 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                     for (int q = 0; q < 4; ++q) {
                         float b[8];
                         unpack_bias8(bias_cur[q], b);
-                        const uint4 u = epilogue8<EPI>(r + q * 8, b);
+                        const uint4 u = epilogue8<EPI>(r + q * 8, b, sm_max, sm_scale);
                         const uint32_t phys = static_cast<uint32_t>(q) ^ ((lane >> 1) & 3u);
                         const uint32_t addr = buf + lane * 64u + phys * 16u;
                         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
@@ -545,7 +607,7 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                         for (int q = 0; q < 4; ++q) {
                             float b[8];
                             unpack_bias8(bias_cur[q], b);
-                            const uint4 u = epilogue8<EPI>(r + q * 8, b);
+                            const uint4 u = epilogue8<EPI>(r + q * 8, b, sm_max, sm_scale);
                             if (full) {
                                 *reinterpret_cast<uint4 *>(crow + col0 + q * 8) = u;
                             } else {
@@ -565,7 +627,7 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                     for (int q = 0; q < 4; ++q) {
                         float b[8];
                         unpack_bias8(bias_cur[q], b);
-                        const uint4 u = epilogue8<EPI>(r + q * 8, b);
+                        const uint4 u = epilogue8<EPI>(r + q * 8, b, sm_max, sm_scale);
                         const uint32_t phys = static_cast<uint32_t>(q) ^ ((lane >> 1) & 3u);
                         const uint32_t addr = buf + lane * 64u + phys * 16u;
                         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
@@ -654,7 +716,16 @@ __global__ void k0_epilogue_kernel(const __half *__restrict__ bias, __half *__re
          t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int64_t j = t % N;
         const float beta = (EPI != kEpiNone && bias != nullptr) ? __half2float(bias[j]) : 0.f;
-        C[t] = __float2half_rn(apply_epilogue<EPI>(0.f, beta));
+        if constexpr (EPI == kEpiBiasSoftmax) {
+            // every row is softmax(bias); N is small (at most 256)
+            float m = -INFINITY, sum = 0.f;
+            for (int64_t q = 0; q < N; ++q) m = fmaxf(m, bias ? __half2float(bias[q]) : 0.f);
+            for (int64_t q = 0; q < N; ++q)
+                sum += exp2_approx(((bias ? __half2float(bias[q]) : 0.f) - m) * kLog2e);
+            C[t] = __float2half_rn(exp2_approx((beta - m) * kLog2e) * rcp_approx(sum));
+        } else {
+            C[t] = __float2half_rn(apply_epilogue<EPI>(0.f, beta));
+        }
     }
 }
 

@@ -63,7 +63,7 @@ def test_select_config_rejects_bad_args():
     with pytest.raises(binding.TgError):
         binding.tg_gemm_select_config(-1, 4, 4, NONE, 148)
     with pytest.raises(binding.TgError):
-        binding.tg_gemm_select_config(4, 4, 4, 3, 148)
+        binding.tg_gemm_select_config(4, 4, 4, 5, 148)
     with pytest.raises(binding.TgError):
         binding.tg_gemm_select_config(4, 4, 4, 0, 0)
 
@@ -127,3 +127,14 @@ def test_binding_checks_tensor_arguments():
     h = torch.zeros(4, 4, dtype=torch.float16)
     with pytest.raises(ValueError):
         binding.gemm(h, h)          # not CUDA tensors
+
+
+def test_softmax_limits_are_checked_on_the_host():
+    assert binding.tg_gemm(0x1000, 0x200000, None, 0x400000, 4, 257, 4, 4, None) == \
+        binding.TG_ERR_INVALID_ARG
+    with pytest.raises(binding.TgError):
+        binding.tg_gemm_select_config(100, 300, 64, 4, 148)
+    c = binding.tg_gemm_select_config(100, 200, 64, 4, 148)
+    assert c["epi_warps"] == 4 and c["block_n"] >= 200
+    assert binding.tg_gemm(0x1000, 0x200000, None, 0x400000, 4, 4, 4, 5, None) == \
+        binding.TG_ERR_INVALID_ARG

@@ -278,3 +278,84 @@ def test_invalid_arguments_on_device():
     assert st == binding.TG_ERR_INVALID_ARG
     with pytest.raises(binding.TgError):
         binding.gemm(a, a, epilogue=NONE, config_id=999)
+
+
+# ---------------------------------------------------------------- tanh GELU and row softmax
+
+TANH, SOFTMAX = binding.TG_EPILOGUE_BIAS_GELU_TANH, binding.TG_EPILOGUE_BIAS_SOFTMAX
+
+
+def _ulp_distance(got_bits, exp_bits):
+    g = got_bits.astype(np.int32)
+    e = exp_bits.astype(np.int32)
+    same = (e & 0x8000) == (g & 0x8000)
+    return np.where(same, np.abs(e - g), (e & 0x7FFF) + (g & 0x7FFF))
+
+
+def test_gelu_tanh_epilogue_within_one_ulp():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = bits.view(np.float16)
+    keep = np.isfinite(vals) & (np.abs(vals.astype(np.float64)) <= 16)
+    bias = torch.from_numpy(vals[keep].copy())
+    M, N, K = 128, bias.numel(), 64
+    A = torch.zeros(M, K, dtype=torch.float16)
+    B = torch.zeros(K, N, dtype=torch.float16)
+    C = run_gpu(A, B, bias, TANH)
+    ref = run_oracle(A, B, bias, oracle.EPI_BIAS_GELU_TANH)
+    dist = _ulp_distance(wl.to_bits(C), oracle.double_to_half_rne(ref))
+    assert dist.max() <= 1, f"max ulp distance {dist.max()}"
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 1), (129, 257, 300), (300, 520, 64)])
+def test_gelu_tanh_epilogue_shapes(M, N, K):
+    A, B, bias = wl.make_inputs(M, N, K, seed=M + N + K, bias=True)
+    assert_close(run_gpu(A, B, bias, TANH), run_oracle(A, B, bias, TANH), f"tanh {M}x{N}x{K}")
+
+
+def _check_softmax(C, ref, what):
+    assert_close(C, ref, what)
+    c = C.to(torch.float64).numpy()
+    # tighter: fp16 rounding of a probability plus fp32 arithmetic
+    err = np.abs(c - ref)
+    assert np.all(err <= 1e-3 * ref + 2e-7), f"{what}: max rel err {np.max(err / (ref + 1e-30)):.2e}"
+    assert np.allclose(c.sum(axis=1), 1.0, atol=2e-2), what
+
+
+SOFTMAX_SHAPES = [(1, 1, 1), (7, 5, 13), (130, 64, 100), (300, 100, 257), (1000, 256, 512),
+                  (257, 200, 64), (64, 33, 2050)]
+
+
+@pytest.mark.parametrize("M,N,K", SOFTMAX_SHAPES)
+def test_softmax_epilogue(M, N, K):
+    A, B, bias = wl.make_inputs(M, N, K, seed=3 * M + N + 7 * K, bias=True)
+    _check_softmax(run_gpu(A, B, bias, SOFTMAX), run_oracle(A, B, bias, SOFTMAX),
+                   f"softmax {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("config_id", [5, 6, 7, 8])
+def test_softmax_every_capable_config(config_id):
+    info = binding.tg_config_info(config_id)
+    N = min(info["block_n"], 200)
+    A, B, bias = wl.make_inputs(517, N, 333, seed=900 + config_id, dist="uniform", bias=True)
+    _check_softmax(run_gpu(A, B, bias, SOFTMAX, config_id=config_id),
+                   run_oracle(A, B, bias, SOFTMAX), f"softmax cfg{config_id}")
+
+
+def test_softmax_without_bias_and_with_k0():
+    A, B, _ = wl.make_inputs(100, 77, 90, seed=950)
+    _check_softmax(run_gpu(A, B, None, SOFTMAX), run_oracle(A, B, None, SOFTMAX), "no bias")
+    bias = torch.linspace(-3, 3, 50).to(torch.float16)
+    A0 = torch.zeros(9, 0, dtype=torch.float16)
+    B0 = torch.zeros(0, 50, dtype=torch.float16)
+    _check_softmax(run_gpu(A0, B0, bias, SOFTMAX), run_oracle(A0, B0, bias, SOFTMAX), "K=0")
+
+
+def test_softmax_rejects_wide_rows_and_incapable_configs():
+    dev = torch.device("cuda:0")
+    a = torch.zeros(64, 64, dtype=torch.float16, device=dev)
+    b = torch.zeros(64, 300, dtype=torch.float16, device=dev)
+    with pytest.raises(binding.TgError):
+        binding.gemm(a, b, epilogue=SOFTMAX)            # N > 256
+    b2 = torch.zeros(64, 128, dtype=torch.float16, device=dev)
+    with pytest.raises(binding.TgError):
+        binding.gemm(a, b2, epilogue=SOFTMAX, config_id=0)   # 8 epilogue warps

@@ -40,7 +40,7 @@ UNIT = "TFLOP/s"
 NOMINAL_FP16_DENSE_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
-EPI_NAMES = {0: "none", 1: "bias", 2: "bias_gelu"}
+EPI_NAMES = {0: "none", 1: "bias", 2: "bias_gelu", 3: "bias_gelu_tanh", 4: "bias_softmax"}
 
 
 # ---------------------------------------------------------------------------- helpers
@@ -459,7 +459,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="fused_8192")
-    ap.add_argument("--also", nargs="*", default=["gemm_2048", "fused_2048"],
+    ap.add_argument("--also", nargs="*",
+                    default=["gemm_2048", "fused_2048", "fused_tanh_2048", "softmax_8192x256x4096",
+                             "deepk_fused_1024x1024x8192"],
                     help="other workloads timed the same way and reported under 'also'")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

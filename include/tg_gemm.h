@@ -109,6 +109,16 @@ typedef enum {
  * rasterisation) comes from a per-shape table built by an offline sweep;
  * see tg_gemm_select_config.  Results are deterministic: the same inputs and
  * configuration give bit-identical C.
+ *
+ * Work split: a problem with at least two waves of output tiles is computed
+ * tile by tile.  A smaller one is computed "stream-K": the tiles' K loops are
+ * divided evenly over all SMs (or SM pairs); a unit that covers the later
+ * part of a tile's K loop writes an fp32 partial tile, and the unit that
+ * covers its start adds those partials (always in the same order) before the
+ * epilogue.  The partials live in a workspace owned by the library, created
+ * once per (device, stream) on first use (a cudaMalloc of about
+ * 148 x 128 KiB plus flags), so stream-K calls on one stream are ordered by
+ * that stream; a first call inside a stream capture cannot create it.
  */
 tg_status_t tg_gemm(const void *A, const void *B, const void *bias, void *C,
                     int64_t M, int64_t N, int64_t K, int epilogue, void *stream);
@@ -118,11 +128,14 @@ tg_status_t tg_gemm(const void *A, const void *B, const void *bias, void *C,
  *   id         index in [0, tg_num_configs())
  *   block_m    output rows per MMA tile (128 per CTA; 256 with a CTA pair)
  *   block_n    output columns per MMA tile (64, 128 or 256)
- *   block_k    K elements per pipeline stage (64)
+ *   block_k    K elements per pipeline stage (64 or 128)
  *   stages     depth of the shared-memory operand ring
  *   cta_pair   1 if two CTAs of a cluster share one 2-SM MMA (cta_group::2)
  *   group_m    M-tiles per rasterisation panel (L2 reuse)
  *   epi_warps  warps that drain the accumulator
+ *   split      from tg_gemm_select_config: how tg_gemm divides that problem
+ *              among the SMs, TG_SPLIT_TILES or TG_SPLIT_STREAM_K; 0 from
+ *              tg_config_info
  */
 typedef struct {
     int id;
@@ -133,6 +146,7 @@ typedef struct {
     int cta_pair;
     int group_m;
     int epi_warps;
+    int split;
 } tg_config_t;
 
 /* Number of compiled tile configurations. */
@@ -145,8 +159,13 @@ tg_status_t tg_config_info(int id, tg_config_t *out);
 /*
  * The configuration tg_gemm would use for this problem (host only, no device
  * call; `num_sms` is the device's SM count, 148 on B200).  The choice comes
- * from the compiled per-shape table (an offline sweep's winners) and falls
- * back to a size rule for shapes the table does not list.
+ * from the compiled per-shape table (an offline sweep's winners, with the
+ * split each was timed with) and falls back to a cost rule for shapes the
+ * table does not list: per configuration, the k-blocks the busiest SM runs
+ * when whole tiles are dealt out in waves, against the k-blocks of an even
+ * stream-K share plus a fixed cost for the partial-sum exchange; the
+ * cheapest (configuration, split) wins.  The softmax epilogue always runs
+ * whole tiles under this rule.
  */
 tg_status_t tg_gemm_select_config(int64_t M, int64_t N, int64_t K, int epilogue,
                                   int num_sms, tg_config_t *out);
@@ -164,15 +183,27 @@ tg_status_t tg_gemm_select_config(int64_t M, int64_t N, int64_t K, int epilogue,
  *                  wait expires; for testing the timeout path only.  The
  *                  kernel then exits cleanly and tg_gemm_check_error returns
  *                  TG_ERR_TIMEOUT.
+ *                  TG_INJECT_SKIP_STREAMK_FLAGS makes stream-K partial
+ *                  results never be flagged, so the units that wait for them
+ *                  time out the same way.
  *   group_m        0: the configuration's rasterisation panel height; else
  *                  the number of M-tiles per panel (1 .. 64)
+ *   split          TG_SPLIT_AUTO: the table's split for a listed shape, else
+ *                  the cost rule of tg_gemm_select_config (for a forced
+ *                  config_id too); TG_SPLIT_TILES: always whole tiles;
+ *                  TG_SPLIT_STREAM_K: always stream-K (see tg_gemm).
  */
 #define TG_INJECT_SKIP_FIRST_LOAD 1
+#define TG_INJECT_SKIP_STREAMK_FLAGS 2
+#define TG_SPLIT_AUTO 0
+#define TG_SPLIT_TILES 1
+#define TG_SPLIT_STREAM_K 2
 typedef struct {
     int config_id;
     uint64_t wait_limit_ns;
     int inject;
     int group_m;
+    int split;
 } tg_options_t;
 
 tg_status_t tg_gemm_ex(const void *A, const void *B, const void *bias, void *C,

@@ -34,6 +34,10 @@ TG_ERR_CUDA = 7
 TG_ERR_SCRATCH_LIMIT = 8
 
 TG_INJECT_SKIP_FIRST_LOAD = 1
+TG_INJECT_SKIP_STREAMK_FLAGS = 2
+TG_SPLIT_AUTO = 0
+TG_SPLIT_TILES = 1
+TG_SPLIT_STREAM_K = 2
 
 EPILOGUES = {"none": TG_EPILOGUE_NONE, "bias": TG_EPILOGUE_BIAS, "bias_gelu": TG_EPILOGUE_BIAS_GELU,
              "bias_gelu_tanh": TG_EPILOGUE_BIAS_GELU_TANH, "bias_softmax": TG_EPILOGUE_BIAS_SOFTMAX}
@@ -48,7 +52,7 @@ class TgError(RuntimeError):
 class tg_config_t(ctypes.Structure):
     _fields_ = [("id", ctypes.c_int), ("block_m", ctypes.c_int), ("block_n", ctypes.c_int),
                 ("block_k", ctypes.c_int), ("stages", ctypes.c_int), ("cta_pair", ctypes.c_int),
-                ("group_m", ctypes.c_int), ("epi_warps", ctypes.c_int)]
+                ("group_m", ctypes.c_int), ("epi_warps", ctypes.c_int), ("split", ctypes.c_int)]
 
     def as_dict(self):
         return {name: getattr(self, name) for name, _ in self._fields_}
@@ -56,7 +60,7 @@ class tg_config_t(ctypes.Structure):
 
 class tg_options_t(ctypes.Structure):
     _fields_ = [("config_id", ctypes.c_int), ("wait_limit_ns", ctypes.c_uint64),
-                ("inject", ctypes.c_int), ("group_m", ctypes.c_int)]
+                ("inject", ctypes.c_int), ("group_m", ctypes.c_int), ("split", ctypes.c_int)]
 
 
 _lib = None
@@ -130,8 +134,8 @@ def noalloc_scratch_bytes(header: str = HEADER) -> int:
 
 
 def tg_gemm_ex(A, B, bias, C, M, N, K, epilogue, config_id=-1, wait_limit_ns=0, inject=0,
-               stream=None, group_m=0) -> int:
-    opts = tg_options_t(config_id, wait_limit_ns, inject, group_m)
+               stream=None, group_m=0, split=0) -> int:
+    opts = tg_options_t(config_id, wait_limit_ns, inject, group_m, split)
     return load().tg_gemm_ex(A, B, bias, C, M, N, K, epilogue, ctypes.byref(opts), stream)
 
 
@@ -194,7 +198,7 @@ def _stream_handle(torch, device):
 
 
 def gemm(a, b, bias=None, epilogue=None, out=None, *, config_id=-1, wait_limit_ns=0, inject=0,
-         group_m=0):
+         group_m=0, split=0):
     """C = g(a @ b + bias) on the GPU through tg_gemm_ex.
 
     a: (M, K) fp16 CUDA, b: (K, N) fp16 CUDA, bias: (N,) fp16 CUDA or None,
@@ -228,7 +232,7 @@ def gemm(a, b, bias=None, epilogue=None, out=None, *, config_id=-1, wait_limit_n
         st = tg_gemm_ex(a.data_ptr(), b.data_ptr(), bias.data_ptr() if bias is not None else None,
                         out.data_ptr(), M, N, K, epi, config_id=config_id,
                         wait_limit_ns=wait_limit_ns, inject=inject,
-                        stream=_stream_handle(torch, a.device), group_m=group_m)
+                        stream=_stream_handle(torch, a.device), group_m=group_m, split=split)
     if st != TG_OK:
         raise TgError(st, "tg_gemm")
     return out

@@ -16,7 +16,9 @@
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "tg_gemm.h"
 #include "tg_kernels.cuh"
@@ -143,32 +145,74 @@ struct TableRow {
     int64_t M, N, K;
     int epilogue;
     int config;
+    int split;   // TG_SPLIT_TILES or TG_SPLIT_STREAM_K, as the sweep timed it
 };
 #include "tg_configs.inc"
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// Size rule for shapes missing from the table: minimise
-// waves * (per-SM tile work) / efficiency, i.e. the finishing time of the
-// last wave in units of one 128 x 64 per-SM tile slice, with wider tiles and
-// CTA pairs credited for their better operand reuse.
-int rule_config(int64_t M, int64_t N, int num_sms)
+// Cost model for choosing a configuration and a work division, in
+// microseconds at the power-capped clock of a busy B200 (about 1.4 GHz).
+//   One k-block of one SM takes max(MMA, operand load): the MMA does
+//   128 x BN x BK multiply-adds at 8192 flops per clock; the loads bring
+//   (128 + BN / CG) x BK fp16 values at about 64 bytes per clock from L2.
+//   Whole tiles: the busiest SM runs ceil(tiles / units) tiles of all k-blocks.
+//   Stream-K: every unit runs ceil(tiles x k-blocks / units) k-blocks, plus a
+//   fixed 6 us for writing, flagging and waiting, plus the head's fold of its
+//   contributors' partials (128 x BN fp32 per CTA each) at about 75 GB/s.
+// The constants were fitted to whole-tile and stream-K timings of the
+// compiled configurations on deep-K and square shapes.
+constexpr double kClockGhz = 1.4;
+constexpr double kStreamKFixedUs = 6.0;
+constexpr double kFoldGBs = 75.0;
+
+struct Choice {
+    int config;
+    int split;   // TG_SPLIT_TILES or TG_SPLIT_STREAM_K
+};
+
+void split_costs(int id, int64_t M, int64_t N, int64_t K, int sms, double *dp, double *sk)
 {
-    struct Cand { int id; double eff; };
-    const Cand cands[] = {{0, 1.0}, {2, 0.93}, {4, 0.85}, {5, 0.7}};
-    const int sms = num_sms > 1 ? num_sms : 148;
-    int best = 0;
-    double best_score = 0;
+    const tg_config_t &ci = kConfigs[id].info;
+    const int cg = ci.cta_pair ? 2 : 1;
+    const int64_t tiles = ceil_div(M, ci.block_m) * ceil_div(N, ci.block_n);
+    const int64_t kb = ceil_div(K, ci.block_k);
+    const int64_t units = ci.cta_pair ? sms / 2 : sms;
+    const double mma_clk = static_cast<double>(ci.block_n) * ci.block_k / 32.0;
+    const double load_clk = (128.0 + static_cast<double>(ci.block_n) / cg) * ci.block_k * 2.0 / 64.0;
+    const double iter_us = (mma_clk > load_clk ? mma_clk : load_clk) / (kClockGhz * 1e3);
+    *dp = static_cast<double>(ceil_div(tiles, units) * kb) * iter_us;
+    const double contributors =
+        units > tiles ? static_cast<double>(units) / static_cast<double>(tiles) : 1.0;
+    const double partial_bytes = 128.0 * ci.block_n * 4.0;
+    *sk = static_cast<double>(ceil_div(tiles * kb, units)) * iter_us + kStreamKFixedUs +
+          contributors * partial_bytes / (kFoldGBs * 1e3);
+}
+
+int rule_split(int id, int64_t M, int64_t N, int64_t K, int epilogue, int sms)
+{
+    if (epilogue == TG_EPILOGUE_BIAS_SOFTMAX) return TG_SPLIT_TILES;
+    double dp, sk;
+    split_costs(id, M, N, K, sms, &dp, &sk);
+    return sk < 0.8 * dp ? TG_SPLIT_STREAM_K : TG_SPLIT_TILES;
+}
+
+// Shapes missing from the table: the cheapest (configuration, split) among
+// the general-purpose tiles.
+Choice rule_choice(int64_t M, int64_t N, int64_t K, int epilogue, int sms)
+{
+    const int cands[] = {0, 2, 4, 5};
+    Choice best{0, TG_SPLIT_TILES};
+    double best_cost = 0;
     bool first = true;
-    for (const Cand &c : cands) {
-        const tg_config_t &ci = kConfigs[c.id].info;
-        const int64_t tiles = ceil_div(M, ci.block_m) * ceil_div(N, ci.block_n);
-        const int64_t units = ci.cta_pair ? sms / 2 : sms;
-        const double waves = static_cast<double>(ceil_div(tiles, units));
-        const double score = waves * (ci.block_n / 64.0) / c.eff;
-        if (first || score < best_score - 1e-9) {
-            best = c.id;
-            best_score = score;
+    for (int id : cands) {
+        const int split = rule_split(id, M, N, K, epilogue, sms);
+        double dp, sk;
+        split_costs(id, M, N, K, sms, &dp, &sk);
+        const double cost = split == TG_SPLIT_STREAM_K ? sk : dp;
+        if (first || cost < best_cost - 1e-9) {
+            best = {id, split};
+            best_cost = cost;
             first = false;
         }
     }
@@ -179,25 +223,24 @@ int rule_config(int64_t M, int64_t N, int num_sms)
 // warps and block_n >= N (N <= 256).
 bool softmax_capable(const tg_config_t &c, int64_t N) { return c.epi_warps == 4 && c.block_n >= N; }
 
-int choose_config(int64_t M, int64_t N, int64_t K, int epilogue, int num_sms)
+Choice choose_config(int64_t M, int64_t N, int64_t K, int epilogue, int num_sms)
 {
+    const int sms = num_sms > 1 ? num_sms : 148;
+    for (const TableRow &r : kShapeTable)
+        if (r.M >= 0 && r.M == M && r.N == N && r.K == K &&
+            (r.epilogue < 0 || r.epilogue == epilogue) && r.config >= 0 &&
+            r.config < kNumConfigs &&
+            (epilogue != TG_EPILOGUE_BIAS_SOFTMAX || softmax_capable(kConfigs[r.config].info, N)))
+            return {r.config, (r.split == TG_SPLIT_TILES || r.split == TG_SPLIT_STREAM_K)
+                                  ? r.split
+                                  : rule_split(r.config, M, N, K, epilogue, sms)};
     if (epilogue == TG_EPILOGUE_BIAS_SOFTMAX) {
-        for (const TableRow &r : kShapeTable)
-            if (r.M >= 0 && r.M == M && r.N == N && r.K == K && r.epilogue == epilogue &&
-                r.config >= 0 && r.config < kNumConfigs &&
-                softmax_capable(kConfigs[r.config].info, N))
-                return r.config;
         // narrow rows: the 64-column single-CTA tile; otherwise the 256-column
         // CTA pair when it fills the SM pairs, else the 256-column single CTA
-        if (N <= 64) return 5;
-        const int sms = num_sms > 1 ? num_sms : 148;
-        return ceil_div(M, 256) >= sms / 2 ? 6 : 8;
+        const int id = N <= 64 ? 5 : (ceil_div(M, 256) >= sms / 2 ? 6 : 8);
+        return {id, TG_SPLIT_TILES};
     }
-    for (const TableRow &r : kShapeTable)
-        if (r.M >= 0 && r.M == M && r.N == N && r.K == K && (r.epilogue < 0 || r.epilogue == epilogue) &&
-            r.config >= 0 && r.config < kNumConfigs)
-            return r.config;
-    return rule_config(M, N, num_sms);
+    return rule_choice(M, N, K, epilogue, sms);
 }
 
 // ------------------------------------------------------------------ devices
@@ -212,6 +255,49 @@ DeviceState g_devices[kMaxDevices];
 std::mutex g_mutex;
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// Stream-K workspace of one (device, stream): an fp32 128 x 256 partial tile
+// per CTA and one completion flag per (CTA, epilogue warp).  Flags hold the
+// epoch of the launch that wrote them, so they never need clearing again.
+struct StreamKWorkspace {
+    float *partials = nullptr;
+    unsigned *flags = nullptr;
+    unsigned epoch = 0;
+};
+constexpr int kMaxEpiWarps = 8;
+std::map<std::pair<int, cudaStream_t>, StreamKWorkspace> g_streamk;   // under g_mutex
+
+// The workspace for (current device, stream) and a fresh epoch; created on
+// first use (cudaMalloc, flags zeroed on `stream`).
+tg_status_t streamk_workspace(int num_sms, cudaStream_t stream, float **partials,
+                              unsigned **flags, unsigned *epoch)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return TG_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    StreamKWorkspace &w = g_streamk[std::make_pair(dev, stream)];
+    if (!w.partials) {
+        const size_t part_bytes = static_cast<size_t>(num_sms) * tg::kBlockM * 256 * sizeof(float);
+        const size_t flag_bytes = static_cast<size_t>(num_sms) * kMaxEpiWarps * sizeof(unsigned);
+        void *mem = nullptr;
+        if (cudaMalloc(&mem, part_bytes + flag_bytes) != cudaSuccess) {
+            cudaGetLastError();
+            g_streamk.erase(std::make_pair(dev, stream));
+            return TG_ERR_OOM;
+        }
+        w.partials = static_cast<float *>(mem);
+        w.flags = reinterpret_cast<unsigned *>(static_cast<char *>(mem) + part_bytes);
+        if (cudaMemsetAsync(w.flags, 0, flag_bytes, stream) != cudaSuccess) {
+            cudaGetLastError();
+            return TG_ERR_CUDA;
+        }
+    }
+    if (++w.epoch == 0) w.epoch = 1;
+    *partials = w.partials;
+    *flags = w.flags;
+    *epoch = w.epoch;
+    return TG_OK;
+}
 
 tg_status_t device_state(DeviceState **out, int *dev_out)
 {
@@ -354,7 +440,10 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
     tg_status_t st = validate(A, B, bias, C, M, N, K, epilogue);
     if (st != TG_OK || M == 0 || N == 0) return st;
     if (opts && (opts->config_id < -1 || opts->config_id >= kNumConfigs)) return TG_ERR_INVALID_ARG;
-    if (opts && (opts->inject != 0 && opts->inject != TG_INJECT_SKIP_FIRST_LOAD))
+    if (opts && (opts->inject != 0 && opts->inject != TG_INJECT_SKIP_FIRST_LOAD &&
+                 opts->inject != TG_INJECT_SKIP_STREAMK_FLAGS))
+        return TG_ERR_INVALID_ARG;
+    if (opts && (opts->split < TG_SPLIT_AUTO || opts->split > TG_SPLIT_STREAM_K))
         return TG_ERR_INVALID_ARG;
     if (opts && (opts->group_m < 0 || opts->group_m > 64)) return TG_ERR_INVALID_ARG;
     DeviceState *dev = nullptr;
@@ -363,9 +452,12 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
     if (epilogue == TG_EPILOGUE_NONE) bias = nullptr;
     if (K == 0) return launch_k0(bias, C, M, N, epilogue, stream, dev->num_sms);
 
-    const int cfg_id = (opts && opts->config_id >= 0)
-                           ? opts->config_id
-                           : choose_config(M, N, K, epilogue, dev->num_sms);
+    Choice choice{0, TG_SPLIT_TILES};
+    if (opts && opts->config_id >= 0)
+        choice = {opts->config_id, rule_split(opts->config_id, M, N, K, epilogue, dev->num_sms)};
+    else
+        choice = choose_config(M, N, K, epilogue, dev->num_sms);
+    const int cfg_id = choice.config;
     const KernelConfig &cfg = kConfigs[cfg_id];
     const int bn = cfg.info.block_n;
     if (epilogue == TG_EPILOGUE_BIAS_SOFTMAX && !softmax_capable(cfg.info, N))
@@ -431,10 +523,26 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
     p.bias_vec = (bias && aligned(bias, 16)) ? 1 : 0;
     p.wait_limit_ns = (opts && opts->wait_limit_ns) ? opts->wait_limit_ns : kDefaultWaitLimitNs;
     p.error_word = dev->error_word;
-    // Persistent grid: one CTA (or CTA pair) per SM (pair of SMs), never
-    // more than there are tiles.
+    // Persistent grid: one CTA (or CTA pair) per SM (pair of SMs).  Whole
+    // tiles: never more units than tiles.
     const int units = cfg.info.cta_pair ? dev->num_sms / 2 : dev->num_sms;
-    const int grid = static_cast<int>(std::min<int64_t>(p.num_tiles, units)) *
+    const int split = (opts && opts->split != TG_SPLIT_AUTO) ? opts->split : choice.split;
+    const int64_t iters = static_cast<int64_t>(p.num_tiles) * p.num_k_blocks;
+    const bool stream_k = split == TG_SPLIT_STREAM_K;
+    p.stream_k = stream_k ? 1 : 0;
+    p.sk_partials = nullptr;
+    p.sk_flags = nullptr;
+    p.sk_epoch = 0;
+    if (stream_k) {
+        st = streamk_workspace(dev->num_sms, stream, &p.sk_partials, &p.sk_flags, &p.sk_epoch);
+        if (st != TG_OK) {
+            if (tmp) cudaFreeAsync(tmp, stream);
+            return st;
+        }
+    }
+    // Stream-K: at most one unit per iteration, so that no unit's range is empty.
+    const int grid = static_cast<int>(stream_k ? std::min<int64_t>(iters, units)
+                                               : std::min<int64_t>(p.num_tiles, units)) *
                      (cfg.info.cta_pair ? 2 : 1);
 
     cudaError_t e = cfg.fn[epilogue][store == tg::kStoreScalar ? 0 : 1](ta, tb, tc, p, grid, stream);
@@ -481,7 +589,9 @@ tg_status_t tg_gemm_select_config(int64_t M, int64_t N, int64_t K, int epilogue,
         epilogue > TG_EPILOGUE_BIAS_SOFTMAX || num_sms <= 0 ||
         (epilogue == TG_EPILOGUE_BIAS_SOFTMAX && N > kSoftmaxMaxN))
         return TG_ERR_INVALID_ARG;
-    *out = kConfigs[choose_config(M, N, K, epilogue, num_sms)].info;
+    const Choice c = choose_config(M, N, K, epilogue, num_sms);
+    *out = kConfigs[c.config].info;
+    out->split = c.split;
     return TG_OK;
 }
 
@@ -666,7 +776,7 @@ tg_status_t gemm_noalloc_impl(const void *A, const void *B, const void *bias, vo
     if (epilogue == TG_EPILOGUE_NONE) bias = nullptr;
     if (K == 0) return launch_k0(bias, C, M, N, epilogue, stream, dev->num_sms);
 
-    const int cfg_id = choose_config(M, N, K, epilogue, dev->num_sms);
+    const int cfg_id = choose_config(M, N, K, epilogue, dev->num_sms).config;
     const KernelConfig &cfg = kConfigs[cfg_id];
     const void *Aeff = A, *Beff = B;
     if (!a_direct) {
@@ -709,6 +819,10 @@ tg_status_t gemm_noalloc_impl(const void *A, const void *B, const void *bias, vo
     p.bias_vec = (bias && aligned(bias, 16)) ? 1 : 0;
     p.wait_limit_ns = kDefaultWaitLimitNs;
     p.error_word = dev->error_word;
+    p.stream_k = 0;   // stream-K needs a workspace; this entry point allocates nothing
+    p.sk_partials = nullptr;
+    p.sk_flags = nullptr;
+    p.sk_epoch = 0;
     const int units = cfg.info.cta_pair ? dev->num_sms / 2 : dev->num_sms;
     const int grid = static_cast<int>(std::min<int64_t>(p.num_tiles, units)) *
                      (cfg.info.cta_pair ? 2 : 1);

@@ -37,12 +37,15 @@ constexpr int kUmmaK = 16;     // K of one kind::f16 MMA instruction
 constexpr int kAAtomBytes = kBlockM * kAtomK * 2;     // one 128 x 64 A box: 16 KiB
 constexpr int kStoreCols = 32;                        // C columns per TMEM load / TMA store box
 constexpr int kStoreBoxBytes = 32 * kStoreCols * 2;   // 32 rows x 32 fp16 = 2 KiB
+constexpr int kFoldSlotBytes = 32 * kStoreCols * 4;   // 32 rows x 32 fp32 columns
 
 // Error word bits (OR-ed into the per-device error word on a wait expiry).
 constexpr unsigned kErrProducerWait = 1u;
 constexpr unsigned kErrMmaWait = 2u;
 constexpr unsigned kErrEpilogueWait = 4u;
 constexpr unsigned kErrDrain = 8u;
+constexpr unsigned kErrStreamKWait = 16u;
+constexpr unsigned kErrFoldWait = 32u;
 
 enum : int { kEpiNone = 0, kEpiBias = 1, kEpiBiasGelu = 2, kEpiBiasGeluTanh = 3, kEpiBiasSoftmax = 4 };
 // How the epilogue writes C: element stores (any pitch), 16-byte stores
@@ -59,10 +62,103 @@ struct GemmParams {
     int num_k_blocks;       // ceil(K / 64)
     int num_tiles;
     int group_m;
-    int inject;             // 1: the first CTA skips its first operand load (timeout test)
+    int inject;             // 1: the first CTA skips its first operand load;
+                            // 2: stream-K partials are never flagged (timeout tests)
     int bias_vec;           // bias is 16-byte aligned: load it 8 values at a time
     uint64_t wait_limit_ns;
     unsigned *error_word;   // device address of the per-device error word
+    // Stream-K: the tiles' k-block iterations are split evenly over the units
+    // (CTAs, or CTA pairs) instead of whole tiles.
+    int stream_k;
+    float *sk_partials;     // per CTA: 128 x BN fp32 partial accumulator, laid out
+                            // so that each warp store is one contiguous 512-B run
+    unsigned *sk_flags;     // per CTA and epilogue warp: epoch at which that warp's
+                            // rows / columns of the CTA's partial are complete
+    unsigned sk_epoch;      // this launch's epoch (never 0)
+};
+
+// The work of one unit, as segments (tile, k-blocks [k0, k1)).
+//   data-parallel: whole tiles unit, unit + num_units, ...
+//   stream-K:      the iterations [unit * I / U, (unit + 1) * I / U) of the
+//                  I = tiles * k-blocks iteration space, cut at tile borders.
+// Roles: kSegFull (whole tile), kSegHead (holds k-block 0 but not the last:
+// adds the later units' partials, then runs the epilogue), kSegPartial (starts
+// after k-block 0: writes its partial for the head).  A unit's partial
+// segment, if any, is its first and its head segment its last, so a head
+// only ever waits on work that the other units do before any waiting.
+enum : int { kSegFull = 0, kSegHead = 1, kSegPartial = 2 };
+
+struct WorkIter {
+    long long cur, end;
+    int kb, step;
+    bool sk;
+
+    __device__ __forceinline__ static long long sk_begin(const GemmParams &p, int unit, int units)
+    {
+        return static_cast<long long>(p.num_tiles) * p.num_k_blocks * unit / units;
+    }
+
+    // The last unit whose range starts before iteration `tile_end` (a head
+    // at `unit` adds the partials of units unit + 1 .. that one).  The range
+    // starts floor(I u / U) are stepped by adding I / U and carrying the
+    // remainder, so the search costs two divisions however long it is.  The
+    // host launches at most I units, so every unit's range is non-empty.
+    __device__ __forceinline__ static int last_contributor(const GemmParams &p, int unit, int units,
+                                                           long long tile_end)
+    {
+        const long long iters = static_cast<long long>(p.num_tiles) * p.num_k_blocks;
+        const long long q_step = iters / units;
+        const long long r_step = iters - q_step * units;
+        const long long num = iters * (unit + 1);
+        long long q = num / units;   // start of unit + 1
+        long long r = num - q * units;
+        int last = unit;
+        while (last + 1 < units && q < tile_end) {
+            ++last;
+            q += q_step;
+            r += r_step;
+            if (r >= units) {
+                r -= units;
+                ++q;
+            }
+        }
+        return last;
+    }
+
+    __device__ __forceinline__ WorkIter(const GemmParams &p, int unit, int units)
+    {
+        kb = p.num_k_blocks;
+        sk = p.stream_k != 0;
+        step = units;
+        if (sk) {
+            cur = sk_begin(p, unit, units);
+            end = sk_begin(p, unit + 1, units);
+        } else {
+            cur = unit;
+            end = p.num_tiles;
+        }
+    }
+
+    __device__ __forceinline__ bool next(int &tile, int &k0, int &k1, int &role)
+    {
+        if (cur >= end) return false;
+        if (!sk) {
+            tile = static_cast<int>(cur);
+            k0 = 0;
+            k1 = kb;
+            role = kSegFull;
+            cur += step;
+            return true;
+        }
+        tile = static_cast<int>(cur / kb);
+        const long long base = static_cast<long long>(tile) * kb;
+        const long long seg_end = end < base + kb ? end : base + kb;
+        k0 = static_cast<int>(cur - base);
+        k1 = static_cast<int>(seg_end - base);
+        role = (k0 == 0 && k1 == kb) ? kSegFull : (k0 == 0 ? kSegHead : kSegPartial);
+        cur = seg_end;
+        return true;
+    }
 };
 
 // Compile-time shape of one kernel variant.
@@ -90,8 +186,18 @@ struct KernelShape {
     static constexpr uint32_t kTxBytes = kCG * kStageBytes;      // both CTAs land on the leader
     static constexpr int kRingBytes = STAGES * kStageBytes;
     static constexpr int kStagingBytes = STORE != kStoreVec ? EPI_WARPS * 2 * kStoreBoxBytes : 0;
-    // barriers: full[STAGES], empty[STAGES], tmem_full[2], tmem_empty[2], drain
-    static constexpr int kNumBars = 2 * STAGES + 5;
+    // Stream-K fold: once a head segment's MMAs are done the operand ring is
+    // idle, and each epilogue warp streams the contributors' partials into its
+    // own kFoldSlots slots of kFoldSlotBytes (one warp's 32 rows x 32 columns
+    // of fp32) there with bulk copies.
+    static constexpr int kFoldSlots =
+        kRingBytes / (EPI_WARPS * kFoldSlotBytes) < 8 ? kRingBytes / (EPI_WARPS * kFoldSlotBytes)
+                                                      : 8;
+    static_assert(kFoldSlots >= 2, "the operand ring must hold two fold slots per epilogue warp");
+    // barriers: full[STAGES], empty[STAGES], tmem_full[2], tmem_empty[2], drain,
+    // fold[EPI_WARPS][kFoldSlots]
+    static constexpr int kFoldBar = 2 * STAGES + 5;
+    static constexpr int kNumBars = kFoldBar + EPI_WARPS * kFoldSlots;
     static constexpr int kStagingOffset = kRingBytes;
     static constexpr int kBarOffset = kRingBytes + kStagingBytes;
     static constexpr int kTmemSlotOffset = kBarOffset + kNumBars * 8;
@@ -314,6 +420,7 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
             mbar_init(&tmem_empty_bar[b], S::kTmemEmptyArrivals);
         }
         mbar_init(drain_bar, 1);
+        for (int f = 0; f < EPI_WARPS * S::kFoldSlots; ++f) mbar_init(&bars[S::kFoldBar + f], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -349,13 +456,15 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
 #pragma unroll
             for (int s = 0; s < STAGES; ++s) pending[s] = 0;
             bool skip_next = (p.inject == 1 && blockIdx.x == 0);
-            for (int tile = unit; tile < p.num_tiles; tile += num_units) {
+            WorkIter work(p, unit, num_units);
+            int tile, k0, k1, role;
+            while (work.next(tile, k0, k1, role)) {
                 int mt, nt;
                 tile_coords(tile, p.num_m_tiles, p.num_n_tiles, p.group_m, mt, nt);
                 const int a_row = mt * S::kTileM + static_cast<int>(cta_rank) * kBlockM;
                 const int b_col = nt * BN + static_cast<int>(cta_rank) * S::kCtaN;
                 bool ok = true;
-                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+                for (int kb = k0; kb < k1; ++kb) {
                     if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, abort_flag, limit,
                                            p.error_word, kErrProducerWait)) {
                         ok = false;
@@ -427,14 +536,16 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
             // (leading), 8-k-row groups 1024 B apart (stride).
             const uint64_t b_desc0 =
                 smem_desc_sw128(smem_base + S::kABytes, S::kBChunkBytes, 1024);
-            for (int tile = unit; tile < p.num_tiles; tile += num_units) {
+            WorkIter work(p, unit, num_units);
+            int tile, k0, k1, role;
+            while (work.next(tile, k0, k1, role)) {
                 if (!mbar_wait_bounded(&tmem_empty_bar[acc], acc_phase ^ 1u, abort_flag, limit,
                                        p.error_word, kErrMmaWait))
                     break;
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
                 bool ok = true;
-                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+                for (int kb = k0; kb < k1; ++kb) {
                     if (!ready && !mbar_wait_bounded(&full_bar[stage], phase, abort_flag, limit,
                                                      p.error_word, kErrMmaWait)) {
                         ok = false;
@@ -459,7 +570,7 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                                                   4);
                         const uint64_t b_k =
                             b_desc0 + stage_off + static_cast<uint64_t>((kk * kUmmaK * 128) >> 4);
-                        mma_f16_ss<CG>(d_tmem, a_k, b_k, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                        mma_f16_ss<CG>(d_tmem, a_k, b_k, kIdesc, (kb != k0 || kk != 0) ? 1u : 0u);
                     }
                     issued_any = true;
                     // the stage is free (in both CTAs) once these MMAs finish
@@ -500,7 +611,9 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
         int acc = 0;
         uint32_t acc_phase = 0;
         uint32_t store_count = 0;
-        for (int tile = unit; tile < p.num_tiles; tile += num_units) {
+        WorkIter work(p, unit, num_units);
+        int tile, k0, k1, role;
+        while (work.next(tile, k0, k1, role)) {
             int mt, nt;
             tile_coords(tile, p.num_m_tiles, p.num_n_tiles, p.group_m, mt, nt);
             uint4 bias_next[4];
@@ -523,42 +636,237 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
             __half *crow = p.C + row * p.ldc;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(acc * BN);
-            // Row softmax (4 epilogue warps: each thread owns its whole row): the
-            // row maximum and the sum of exp(v - max) over the valid columns,
-            // from two extra passes over the accumulator in TMEM.
-            float sm_max = 0.f, sm_scale = 0.f;
-            if constexpr (EPI == kEpiBiasSoftmax) {
-                static_assert(EPI_WARPS == 4, "the softmax epilogue needs whole rows per thread");
-                sm_max = -INFINITY;
-                float sum = 0.f;
-#pragma unroll 1
-                for (int pass = 0; pass < 2; ++pass) {
-#pragma unroll 1
-                    for (int c = chunk0; c < chunk0 + S::kChunksPerWarp; ++c) {
-                        const int64_t col0 = static_cast<int64_t>(nt) * BN + c * kStoreCols;
-                        if (col0 >= p.N || row0 >= p.M) break;
-                        uint4 bq[4];
-                        fetch_bias32<EPI>(p.bias, col0, p.N, bias_vec, bq);
-                        uint32_t r[32];
-                        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * kStoreCols), r);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            float b[8];
-                            unpack_bias8(bq[q], b);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                if (col0 + q * 8 + e >= p.N) continue;
-                                const float v = __uint_as_float(r[q * 8 + e]) + b[e];
-                                if (pass == 0)
-                                    sm_max = fmaxf(sm_max, v);
-                                else
-                                    sum += exp2_approx((v - sm_max) * kLog2e);
-                            }
+            // Stream-K partials of a CTA (slot = unit * CG + rank) hold 128 x BN
+            // fp32 values as uint4 groups indexed ((warp * chunks + chunk) * 8 + q)
+            // * 32 + lane: lane l of warp w keeps columns 4q .. 4q + 3 of its row
+            // of chunk c there, so a warp writes 512 contiguous bytes per store and
+            // each (warp, chunk) block is 4 KiB of contiguous memory.
+            auto partial_group = [&](int slot, int c, int q) {
+                return reinterpret_cast<uint4 *>(p.sk_partials +
+                                                 static_cast<size_t>(slot) * kBlockM * BN) +
+                       ((warp * S::kChunksPerWarp + (c - chunk0)) * 8 + q) * 32 + lane;
+            };
+            int first_contrib = 0, last_contrib = -1;   // units whose partials a head adds
+            if (role == kSegHead) {
+                const long long tile_end = static_cast<long long>(tile + 1) * p.num_k_blocks;
+                first_contrib = unit + 1;
+                last_contrib = WorkIter::last_contributor(p, unit, num_units, tile_end);
+                // Warp w of a head reads exactly the rows and columns that warp w
+                // of each contributing CTA wrote, so it waits for those flags only.
+                for (int v = first_contrib; v <= last_contrib; ++v) {
+                    const unsigned *flag = p.sk_flags + (v * CG + cta_rank) * EPI_WARPS + warp;
+                    if (ld_acquire_gpu(flag) == p.sk_epoch) continue;
+                    const uint64_t t0 = global_timer_ns();
+                    while (ld_acquire_gpu(flag) != p.sk_epoch) {
+                        if (*abort_flag) break;
+                        if (global_timer_ns() - t0 > limit) {
+                            *abort_flag = 1;
+                            atomicOr(p.error_word, kErrStreamKWait);
+                            break;
                         }
                     }
                 }
-                sm_scale = rcp_approx(sum);
+            }
+            __syncwarp();   // reconverge before the warp-collective TMEM loads
+            // The chunks this warp's epilogue visits: up to the first one past N
+            // (none when all 32 rows are past M).
+            int chunk_end = chunk0;
+            if (row0 < p.M)
+                while (chunk_end < chunk0 + S::kChunksPerWarp &&
+                       static_cast<int64_t>(nt) * BN + chunk_end * kStoreCols < p.N)
+                    ++chunk_end;
+            // Fold (heads only).  A head segment is the last of its unit, so its
+            // tmem_full means every MMA of this CTA is done and the operand ring
+            // is idle.  Items (chunk c, contributor v) are visited c-major, v
+            // ascending -- the order the sums are taken in -- and item i is
+            // copied into slot i % kFoldSlots of this warp's part of the ring,
+            // kFoldSlots items ahead of its use.
+            bool folding = first_contrib <= last_contrib && chunk_end > chunk0 && *abort_flag == 0;
+            bool fold_ok = true;
+            uint64_t *fold_bar = bars + S::kFoldBar + warp * S::kFoldSlots;
+            const uint32_t fold_smem =
+                smem_base + static_cast<uint32_t>(warp * S::kFoldSlots * kFoldSlotBytes);
+            int issue_c = chunk0, issue_v = first_contrib;
+            uint32_t issued = 0, waited = 0;
+            auto fold_issue = [&]() {
+                if (!folding || !fold_ok || issue_c >= chunk_end) return;
+                const uint32_t slot = issued % S::kFoldSlots;
+                if (lane == 0) {
+                    // 4 KiB: this warp's 32 rows x 32 columns of chunk issue_c
+                    // in contributor issue_v's partial (the layout below).
+                    const float *src =
+                        p.sk_partials +
+                        static_cast<size_t>(issue_v * CG + cta_rank) * kBlockM * BN +
+                        static_cast<size_t>(warp * S::kChunksPerWarp + (issue_c - chunk0)) *
+                            (kFoldSlotBytes / 4);
+                    mbar_arrive_expect_tx(&fold_bar[slot], kFoldSlotBytes);
+                    bulk_load_g2s(fold_smem + slot * kFoldSlotBytes, src, kFoldSlotBytes,
+                                  &fold_bar[slot]);
+                }
+                ++issued;
+                if (++issue_v > last_contrib) {
+                    issue_v = first_contrib;
+                    ++issue_c;
+                }
+            };
+            if (folding) {
+                // The flags were acquired through the generic proxy; the bulk
+                // copies read the partials through the async proxy.
+                if (lane == 0) fence_proxy_async_all();
+                __syncwarp();
+                for (int i = 0; i < S::kFoldSlots; ++i) fold_issue();
+            }
+            // One 32-column chunk of the accumulator: TMEM, plus (for a head)
+            // the partials of the later units, added in unit order.
+            auto load_acc_chunk = [&](int c, uint32_t (&r)[32]) {
+                tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * kStoreCols), r);
+                tmem_wait_ld();
+                if (!folding) return;
+                for (int v = first_contrib; v <= last_contrib; ++v) {
+                    const uint32_t slot = waited % S::kFoldSlots;
+                    if (fold_ok) {
+                        const int ok = mbar_wait_bounded(&fold_bar[slot],
+                                                         (waited / S::kFoldSlots) & 1u, abort_flag,
+                                                         limit, p.error_word, kErrFoldWait)
+                                           ? 1
+                                           : 0;
+                        fold_ok = __all_sync(0xffffffffu, ok) != 0;
+                    }
+                    if (!fold_ok) return;
+                    const uint32_t src = fold_smem + slot * kFoldSlotBytes + lane * 16u;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        uint32_t u0, u1, u2, u3;
+                        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(u0), "=r"(u1), "=r"(u2), "=r"(u3)
+                                     : "r"(src + static_cast<uint32_t>(q) * 512u)
+                                     : "memory");
+                        r[4 * q + 0] = __float_as_uint(__uint_as_float(r[4 * q + 0]) + __uint_as_float(u0));
+                        r[4 * q + 1] = __float_as_uint(__uint_as_float(r[4 * q + 1]) + __uint_as_float(u1));
+                        r[4 * q + 2] = __float_as_uint(__uint_as_float(r[4 * q + 2]) + __uint_as_float(u2));
+                        r[4 * q + 3] = __float_as_uint(__uint_as_float(r[4 * q + 3]) + __uint_as_float(u3));
+                    }
+                    ++waited;
+                    __syncwarp();   // every lane has read the slot before it is refilled
+                    fold_issue();
+                }
+            };
+            // Copies still in flight after a failed wait land before the ring's
+            // shared memory is released.
+            auto fold_drain = [&]() {
+                if (lane == 0)
+                    for (uint32_t i = waited; i < issued; ++i)
+                        if (!mbar_wait_drain(&fold_bar[i % S::kFoldSlots],
+                                             (i / S::kFoldSlots) & 1u, limit))
+                            atomicOr(p.error_word, kErrDrain);
+                __syncwarp();
+            };
+            if (role == kSegPartial) {
+                // Write this warp's rows / columns of the unit's partial
+                // accumulator; once every lane's stores are fenced, flag them.
+#pragma unroll 1
+                for (int c = chunk0; c < chunk0 + S::kChunksPerWarp; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * kStoreCols), r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        __stcg(partial_group(unit * CG + cta_rank, c, q),
+                               make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]));
+                }
+                __threadfence();
+                __syncwarp();
+                if (lane == 0 && p.inject != 2)
+                    st_release_gpu(p.sk_flags + (unit * CG + cta_rank) * EPI_WARPS + warp,
+                                   p.sk_epoch);
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) {
+                    if (PAIR)
+                        mbar_arrive_cluster(empty_bar_leader + static_cast<uint32_t>(acc * 8));
+                    else
+                        mbar_arrive(&tmem_empty_bar[acc]);
+                }
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+                continue;
+            }
+            // Row softmax (4 epilogue warps: each thread owns its whole row).  One
+            // pass over the accumulator in TMEM gives the row maximum and the sum
+            // of exp(v - max) over the valid columns, kept as a running pair: a
+            // chunk raising the maximum from m to m' rescales the sum by
+            // exp(m - m').  Two chunks are read per TMEM wait, and each chunk's
+            // maximum and sum are taken over eight independent partials.
+            float sm_max = 0.f, sm_scale = 0.f;
+            if constexpr (EPI == kEpiBiasSoftmax) {
+                static_assert(EPI_WARPS == 4, "the softmax epilogue needs whole rows per thread");
+                // The statistics pass and the output pass both read the
+                // accumulator; fold the contributors into it in TMEM once, first.
+                if (folding) {
+#pragma unroll 1
+                    for (int c = chunk0; c < chunk_end; ++c) {
+                        uint32_t r[32];
+                        load_acc_chunk(c, r);
+                        tmem_st_32x32b_x32(t_row + static_cast<uint32_t>(c * kStoreCols), r);
+                    }
+                    tmem_wait_st();
+                    folding = false;
+                }
+                float run_max = -INFINITY, run_sum = 0.f;
+                auto stats_chunk = [&](const uint32_t (&r)[32], const uint4 (&bq)[4], int64_t col0) {
+                    float v[32];
+                    const bool full = col0 + kStoreCols <= p.N;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float b[8];
+                        unpack_bias8(bq[q], b);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float x = __uint_as_float(r[q * 8 + e]) + b[e];
+                            v[q * 8 + e] = (full || col0 + q * 8 + e < p.N) ? x : -INFINITY;
+                        }
+                    }
+                    float m[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        m[j] = fmaxf(fmaxf(v[j], v[j + 8]), fmaxf(v[j + 16], v[j + 24]));
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) m[j] = fmaxf(m[j], m[j + 4]);
+                    const float cmax = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+                    const float new_max = fmaxf(run_max, cmax);   // finite: a chunk has a valid column
+                    const float shift = new_max * kLog2e;
+                    float sp[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) sp[j] = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        sp[e & 7] += exp2_approx(fmaf(v[e], kLog2e, -shift));
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) sp[j] += sp[j + 4];
+                    const float csum = (sp[0] + sp[1]) + (sp[2] + sp[3]);
+                    run_sum = fmaf(run_sum, exp2_approx(fmaf(run_max, kLog2e, -shift)), csum);
+                    run_max = new_max;
+                };
+#pragma unroll 1
+                for (int c = chunk0; c < chunk_end; c += 2) {
+                    const bool two = c + 1 < chunk_end;
+                    const int64_t col0 = static_cast<int64_t>(nt) * BN + c * kStoreCols;
+                    uint32_t ra[32], rb[32];
+                    tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * kStoreCols), ra);
+                    if (two)
+                        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((c + 1) * kStoreCols), rb);
+                    uint4 ba[4], bb[4];
+                    fetch_bias32<EPI>(p.bias, col0, p.N, bias_vec, ba);
+                    if (two) fetch_bias32<EPI>(p.bias, col0 + kStoreCols, p.N, bias_vec, bb);
+                    tmem_wait_ld_dep(ra);
+                    if (two) tmem_wait_ld_dep(rb);
+                    stats_chunk(ra, ba, col0);
+                    if (two) stats_chunk(rb, bb, col0 + kStoreCols);
+                }
+                sm_max = run_max;
+                sm_scale = rcp_approx(run_sum);
             }
 #pragma unroll 1
             for (int c = chunk0; c < chunk0 + S::kChunksPerWarp; ++c) {
@@ -571,8 +879,7 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                 if (c + 1 < chunk0 + S::kChunksPerWarp)
                     fetch_bias32<EPI>(p.bias, col0 + kStoreCols, p.N, bias_vec, bias_next);
                 uint32_t r[32];
-                tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * kStoreCols), r);
-                tmem_wait_ld();
+                load_acc_chunk(c, r);
                 if constexpr (STORE == kStoreTma) {
                     // Stage a 32 x 32 fp16 box (64-B rows, 64-B swizzle) and let
                     // one lane store it with TMA; two boxes alternate.
@@ -653,6 +960,7 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                     ++store_count;
                 }
             }
+            fold_drain();
             // All TMEM reads of this accumulator are complete (wait::ld above).
             tc_fence_before_sync();
             __syncwarp();

@@ -1,8 +1,9 @@
-"""Offline schedule sweep: time every compiled configuration on each shape
-and (optionally) rewrite csrc/tg_configs.inc with the winners.
+"""Offline schedule sweep: time every compiled configuration, dealing out
+whole tiles and with stream-K, on each shape and (optionally) rewrite
+csrc/tg_configs.inc with the winners.
 
     python -m tensor_core_gemm_fp16_b200.sweep [--shapes all|NAME ...]
-        [--reps 20] [--warmup 5] [--write] [--json out.json]
+        [--reps 30] [--splits 1 2] [--context] [--write] [--json out.json]
 
 The tutorial sweeps tile sizes, pipeline stages, thread counts and an L2
 swizzle by hand on its 2048^3 GEMM and keeps the fastest that also passes
@@ -36,16 +37,22 @@ DEFAULT_SHAPES = {
     "ragged_fused": (3000, 1537, 2050, 2),
     "fused_8192": (8192, 8192, 8192, 2),
     "gemm_8192": (8192, 8192, 8192, 0),
+    "fused_tanh_2048": (2048, 2048, 2048, 3),
+    "softmax_8192x256x4096": (8192, 256, 4096, 4),
+    "deepk_fused_1024x1024x8192": (1024, 1024, 8192, 2),
+    "deepk_512x512x16384": (512, 512, 16384, 0),
 }
 
 
-def time_config(torch, binding, a, b, bias, c, M, N, K, epi, cfg, reps, warmup, flush, gm=0):
+def time_config(torch, binding, a, b, bias, c, M, N, K, epi, cfg, reps, warmup, flush, gm=0,
+                split=0):
     stream = torch.cuda.current_stream()
     args = (a.data_ptr(), b.data_ptr(), bias.data_ptr() if bias is not None else None,
             c.data_ptr(), M, N, K, epi)
 
     def launch():
-        st = binding.tg_gemm_ex(*args, config_id=cfg, stream=stream.cuda_stream, group_m=gm)
+        st = binding.tg_gemm_ex(*args, config_id=cfg, stream=stream.cuda_stream, group_m=gm,
+                                split=split)
         if st != binding.TG_OK:
             raise binding.TgError(st, f"config {cfg}")
 
@@ -77,7 +84,13 @@ def time_library(torch, a, b, bias, epi, reps, warmup, flush):
         if epi == 0:
             return a @ b
         y = torch.addmm(bias, a, b)
-        return F.gelu(y) if epi == 2 else y
+        if epi == 2:
+            return F.gelu(y)
+        if epi == 3:
+            return F.gelu(y, approximate="tanh")
+        if epi == 4:
+            return torch.softmax(y, dim=1)
+        return y
 
     for _ in range(warmup):
         run()
@@ -97,7 +110,7 @@ def time_library(torch, a, b, bias, epi, reps, warmup, flush):
 
 
 def sweep_shape(torch, binding, name, M, N, K, epi, reps, warmup, configs, group_ms=(0,),
-                context=False, rounds=5):
+                context=False, rounds=5, splits=(1, 2)):
     dev = torch.device("cuda")
     g = torch.Generator(device=dev).manual_seed(1234)
     a = torch.randn(M, K, device=dev, generator=g).half()
@@ -105,29 +118,39 @@ def sweep_shape(torch, binding, name, M, N, K, epi, reps, warmup, configs, group
     bias = torch.randn(N, device=dev, generator=g).half() if epi else None
     c = torch.empty(M, N, device=dev, dtype=torch.float16)
     ref = a.float() @ b.float()
-    if epi:
-        ref = torch.nn.functional.gelu(ref + bias.float()) if epi == 2 else ref + bias.float()
+    F = torch.nn.functional
+    if epi == 1:
+        ref = ref + bias.float()
+    elif epi == 2:
+        ref = F.gelu(ref + bias.float())
+    elif epi == 3:
+        ref = F.gelu(ref + bias.float(), approximate="tanh")
+    elif epi == 4:
+        ref = torch.softmax(ref + bias.float(), dim=1)
     small = 2 * (M * K + K * N + M * N) <= L2_BYTES
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if small else None
     rows = []
     candidates = []
-    for cfg, gm in [(c, g) for c in configs for g in group_ms]:
+    for cfg, gm, split in [(c, g, sp) for c in configs for g in group_ms for sp in splits]:
         info = dict(binding.tg_config_info(cfg))
+        if epi == 4 and (info["epi_warps"] != 4 or info["block_n"] < N):
+            continue   # the row softmax needs whole rows per epilogue thread
         if gm:
             info["group_m"] = gm
         st = binding.tg_gemm_ex(a.data_ptr(), b.data_ptr(),
                                 bias.data_ptr() if bias is not None else None, c.data_ptr(),
-                                M, N, K, epi, config_id=cfg, group_m=gm,
+                                M, N, K, epi, config_id=cfg, group_m=gm, split=split,
                                 stream=torch.cuda.current_stream().cuda_stream)
         torch.cuda.synchronize()
         if st != binding.TG_OK:
-            rows.append({"config": cfg, "error": binding.tg_status_string(st)})
+            rows.append({"config": cfg, "split": split, "error": binding.tg_status_string(st)})
             continue
         rel = float((c.float() - ref).norm() / ref.norm())
         if not rel < 2e-2:
-            rows.append({"config": cfg, "error": f"numerically wrong (rel {rel:.2e})"})
+            rows.append({"config": cfg, "split": split,
+                         "error": f"numerically wrong (rel {rel:.2e})"})
             continue
-        candidates.append((cfg, gm, info, rel))
+        candidates.append((cfg, gm, split, info, rel))
     # Interleaved rounds: every candidate (and the library context) is timed
     # once per round, so slow drifts of the GPU's clock (power, temperature)
     # touch all of them alike; each result is the median over rounds of the
@@ -138,33 +161,47 @@ def sweep_shape(torch, binding, name, M, N, K, epi, reps, warmup, configs, group
     for _ in range(rounds):
         if context:
             lib_rounds.append(time_library(torch, a, b, bias, epi, per, warmup, flush))
-        for i, (cfg, gm, info, rel) in enumerate(candidates):
+        for i, (cfg, gm, split, info, rel) in enumerate(candidates):
             per_round[i].append(time_config(torch, binding, a, b, bias, c, M, N, K, epi, cfg,
-                                            per, warmup, flush, gm))
+                                            per, warmup, flush, gm, split))
     lib_ms = statistics.median(lib_rounds) if context else None
-    for i, (cfg, gm, info, rel) in enumerate(candidates):
+    for i, (cfg, gm, split, info, rel) in enumerate(candidates):
         ms = statistics.median(per_round[i])
-        rows.append({"config": cfg, "group_m_override": gm, "ms": ms,
+        rows.append({"config": cfg, "group_m_override": gm, "split": split, "ms": ms,
                      "tflops": 2.0 * M * N * K / (ms * 1e-3) / 1e12,
                      "rel_err": rel, **{k: info[k] for k in ("block_m", "block_n", "stages",
                                                            "cta_pair", "group_m", "epi_warps")}})
-    ok = [r for r in rows if "ms" in r]
-    best = min(ok, key=lambda r: r["ms"]) if ok else None
+    best = pick_best(rows)
     return {"shape": name, "M": M, "N": N, "K": K, "epilogue": epi, "rows": rows,
             "best": best["config"] if best else None,
+            "best_split": best["split"] if best else None,
             "best_group_m": best["group_m"] if best else None, "l2_flushed": small,
             "library_ms": lib_ms}
+
+
+# Stream-K must beat whole tiles by this factor to be recorded: the event
+# timer's resolution makes near-ties common, and whole tiles need no
+# workspace and no cross-CTA exchange.
+STREAM_K_MARGIN = 1.03
+
+
+def pick_best(rows):
+    """The fastest timed row, with stream-K handicapped by STREAM_K_MARGIN."""
+    ok = [r for r in rows if "ms" in r]
+    if not ok:
+        return None
+    return min(ok, key=lambda r: r["ms"] * (STREAM_K_MARGIN if r.get("split") == 2 else 1.0))
 
 
 def write_table(results, path=TABLE):
     lines = [
         "// tg_configs.inc -- per-shape configuration table.",
         "//",
-        "// Rows: {M, N, K, epilogue (-1 = any), config id}.  A row matches a problem",
-        "// of exactly that shape.  Rows are the winners of the offline sweep",
-        "// (tensor_core_gemm_fp16_b200/sweep.py), which rewrites this file; shapes it",
-        "// does not list fall back to the size rule in tg_gemm.cu.  The last row is a",
-        "// sentinel (M = -1).",
+        "// Rows: {M, N, K, epilogue (-1 = any), config id, split (1 whole tiles,",
+        "// 2 stream-K)}.  A row matches a problem of exactly that shape.  Rows are",
+        "// the winners of the offline sweep (tensor_core_gemm_fp16_b200/sweep.py),",
+        "// which rewrites this file; shapes it does not list fall back to the cost",
+        "// rule in tg_gemm.cu.  The last row is a sentinel (M = -1).",
         "//",
         "// Written by the sweep on a B200; per row: median ms and TFLOP/s of the winner.",
         "static const TableRow kShapeTable[] = {",
@@ -172,10 +209,12 @@ def write_table(results, path=TABLE):
     for r in results:
         if r["best"] is None:
             continue
-        w = next(x for x in r["rows"] if x["config"] == r["best"])
-        lines.append(f"    {{{r['M']}, {r['N']}, {r['K']}, {r['epilogue']}, {r['best']}}},"
+        w = next(x for x in r["rows"]
+                 if x["config"] == r["best"] and x.get("split") == r["best_split"] and "ms" in x)
+        lines.append(f"    {{{r['M']}, {r['N']}, {r['K']}, {r['epilogue']}, {r['best']}, "
+                     f"{r['best_split']}}},"
                      f"  // {r['shape']}: {w['ms'] * 1e3:.1f} us, {w['tflops']:.0f} TFLOP/s")
-    lines += ["    {-1, -1, -1, -1, -1},", "};", ""]
+    lines += ["    {-1, -1, -1, -1, -1, -1},", "};", ""]
     with open(path, "w") as f:
         f.write("\n".join(lines))
 
@@ -191,11 +230,24 @@ def main(argv=None):
     ap.add_argument("--configs", type=int, nargs="*", default=None)
     ap.add_argument("--group-m", type=int, nargs="*", default=[0],
                     help="rasterisation panel heights to try (0: the configuration's own)")
+    ap.add_argument("--splits", type=int, nargs="*", default=[1, 2],
+                    help="work divisions to try (1 whole tiles, 2 stream-K)")
     ap.add_argument("--context", action="store_true",
                     help="also time torch.matmul (+ eager bias/GELU) on each shape")
     ap.add_argument("--write", action="store_true", help="rewrite csrc/tg_configs.inc")
     ap.add_argument("--json", default=None)
+    ap.add_argument("--from-json", default=None,
+                    help="rewrite the table from a saved sweep (no GPU needed)")
     args = ap.parse_args(argv)
+    if args.from_json:
+        with open(args.from_json) as f:
+            results = json.load(f)
+        for r in results:
+            best = pick_best(r["rows"])
+            r["best"] = best["config"] if best else None
+            r["best_split"] = best["split"] if best else None
+        write_table(results)
+        return 0
     sys.path.insert(0, os.path.dirname(HERE))
     import torch
     from tensor_core_gemm_fp16_b200 import binding
@@ -206,21 +258,22 @@ def main(argv=None):
     for name in names:
         M, N, K, epi = DEFAULT_SHAPES[name]
         r = sweep_shape(torch, binding, name, M, N, K, epi, args.reps, args.warmup, configs,
-                        tuple(args.group_m), args.context, args.rounds)
+                        tuple(args.group_m), args.context, args.rounds, tuple(args.splits))
         results.append(r)
         print(f"== {name} ({M}x{N}x{K}, epilogue {epi}) best config {r['best']} "
-              f"group_m {r['best_group_m']}")
+              f"split {r['best_split']} group_m {r['best_group_m']}")
         if r["library_ms"] is not None:
             print(f"   torch/cuBLAS (context) {r['library_ms'] * 1e3:9.1f} us  "
                   f"{2.0 * M * N * K / (r['library_ms'] * 1e-3) / 1e12:7.1f} TFLOP/s")
         for row in r["rows"]:
             if "ms" in row:
-                print(f"   cfg {row['config']:2d}  BM{row['block_m']:4d} BN{row['block_n']:4d} "
+                print(f"   cfg {row['config']:2d} split{row['split']}  BM{row['block_m']:4d} "
+                      f"BN{row['block_n']:4d} "
                       f"st{row['stages']} pair{row['cta_pair']} g{row['group_m']:2d} "
                       f"ew{row['epi_warps']}  {row['ms'] * 1e3:9.1f} us  "
                       f"{row['tflops']:7.1f} TFLOP/s")
             else:
-                print(f"   cfg {row['config']:2d}  {row['error']}")
+                print(f"   cfg {row['config']:2d} split{row['split']}  {row['error']}")
         sys.stdout.flush()
     if args.json:
         with open(args.json, "w") as f:

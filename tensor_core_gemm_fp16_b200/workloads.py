@@ -28,6 +28,8 @@ import torch
 EPI_NONE = 0
 EPI_BIAS = 1
 EPI_BIAS_GELU = 2
+EPI_BIAS_GELU_TANH = 3
+EPI_BIAS_SOFTMAX = 4
 
 
 @dataclasses.dataclass(frozen=True)
@@ -64,6 +66,20 @@ WORKLOADS = {
                              has_bias=True),
     "fused_8192": Workload("fused_8192", 8192, 8192, 8192, EPI_BIAS_GELU, "normal", 4,
                            b_scale=1.0 / math.sqrt(8192), has_bias=True),
+    # The epilogue variants: the tanh form of GELU on the square shape, and a
+    # row softmax over 256 columns (scores of 8192 queries against 256 keys
+    # with a 4096-wide contraction, B scaled by 1/sqrt(K)).
+    "fused_tanh_2048": Workload("fused_tanh_2048", 2048, 2048, 2048, EPI_BIAS_GELU_TANH, "normal",
+                                5, has_bias=True),
+    "softmax_8192x256x4096": Workload("softmax_8192x256x4096", 8192, 256, 4096, EPI_BIAS_SOFTMAX,
+                                      "normal", 6, b_scale=1.0 / math.sqrt(4096), has_bias=True),
+    # Deep contractions with few output tiles: fewer tiles than SMs, so the
+    # work is divided along K as well (stream-K).  B scaled by 1/sqrt(K).
+    "deepk_fused_1024x1024x8192": Workload("deepk_fused_1024x1024x8192", 1024, 1024, 8192,
+                                           EPI_BIAS_GELU, "normal", 7,
+                                           b_scale=1.0 / math.sqrt(8192), has_bias=True),
+    "deepk_512x512x16384": Workload("deepk_512x512x16384", 512, 512, 16384, EPI_NONE, "normal", 8,
+                                    b_scale=1.0 / math.sqrt(16384)),
     # The same shape with both operands scaled by 1/sqrt(K) (the literal wording
     # of the large-workload description); parity only.
     "fused_8192_literal": Workload("fused_8192_literal", 8192, 8192, 8192, EPI_BIAS_GELU,

@@ -59,6 +59,22 @@ def test_select_config_prefers_more_tiles_for_small_problems():
     assert small["block_n"] <= big["block_n"]
 
 
+def test_select_config_reports_the_split():
+    """Whole tiles when there are enough of them; stream-K for a deep
+    contraction with fewer tiles than SMs; never stream-K for the softmax."""
+    assert binding.tg_gemm_select_config(8192, 8192, 8192, GELU, 148)["split"] == \
+        binding.TG_SPLIT_TILES
+    assert binding.tg_gemm_select_config(512, 512, 16384, NONE, 148)["split"] == \
+        binding.TG_SPLIT_STREAM_K
+    assert binding.tg_gemm_select_config(1024, 1024, 8192, GELU, 148)["split"] == \
+        binding.TG_SPLIT_STREAM_K
+    assert binding.tg_gemm_select_config(256, 256, 256, NONE, 148)["split"] == \
+        binding.TG_SPLIT_TILES
+    assert binding.tg_gemm_select_config(8192, 256, 65536, 4, 148)["split"] == \
+        binding.TG_SPLIT_TILES
+    assert binding.tg_config_info(0)["split"] == 0
+
+
 def test_select_config_rejects_bad_args():
     with pytest.raises(binding.TgError):
         binding.tg_gemm_select_config(-1, 4, 4, NONE, 148)
@@ -92,6 +108,8 @@ def test_host_validation_rejects_bad_calls_without_a_device():
     assert binding.tg_gemm_ex(0x1000, 0x2000, None, 0x30000, 4, 4, 4, 0, group_m=65) == \
         binding.TG_ERR_INVALID_ARG
     assert binding.tg_gemm_ex(0x1000, 0x2000, None, 0x30000, 4, 4, 4, 0, inject=7) == \
+        binding.TG_ERR_INVALID_ARG
+    assert binding.tg_gemm_ex(0x1000, 0x2000, None, 0x30000, 4, 4, 4, 0, split=3) == \
         binding.TG_ERR_INVALID_ARG
 
 

@@ -204,7 +204,9 @@ def test_misaligned_operands_use_the_repacking_path():
 
 # ---------------------------------------------------------------- the workloads
 
-@pytest.mark.parametrize("name", ["gemm_256", "gemm_2048", "fused_2048", "ragged_fused"])
+@pytest.mark.parametrize("name", ["gemm_256", "gemm_2048", "fused_2048", "ragged_fused",
+                                  "fused_tanh_2048", "softmax_8192x256x4096",
+                                  "deepk_fused_1024x1024x8192", "deepk_512x512x16384"])
 def test_workload_full_parity(name):
     w = wl.WORKLOADS[name]
     A, B, bias = wl.workload_inputs(w)

@@ -17,7 +17,10 @@ numpy arrays.  Every function cites the passage it follows in the C file:
 * the tanh approximation of GELU -- Hendrycks & Gimpel, "Gaussian Error
   Linear Units", section 2;
 * the row softmax epilogue -- the same tutorial (ainovat.com), row-wise
-  softmax section (per-row max and sum, then normalisation).
+  softmax section (per-row max and sum, then normalisation);
+* attention forward -- the same tutorial (ainovat.com), FlashAttention
+  section (softmax(scale Q K^T) V, causal and non-causal), as its plain
+  definition.
 
 Pins (tests/test_oracle_pins.py) hold it to closed forms, exact rational
 arithmetic, exhaustive codec checks against numpy, and scipy's normal CDF.
@@ -72,6 +75,9 @@ def _load():
         lib.tgo_gelu_n.argtypes = [f64p, i64, f64p]
         lib.tgo_gelu_tanh_n.argtypes = [f64p, i64, f64p]
         lib.tgo_num_threads.restype = ctypes.c_int
+        lib.tgo_attention.argtypes = [u16p, u16p, u16p, i64, i64, i64, i64, i64, ctypes.c_int,
+                                      ctypes.c_double, i64p, i64, f64p]
+        lib.tgo_attention.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -143,6 +149,37 @@ def gemm_int_exact(A, B, bias=None, epilogue: int = EPI_NONE) -> np.ndarray:
                                     _ptr(out, ctypes.c_uint16))
     if st != 0:
         raise OracleError(f"oracle int-exact gemm failed with status {st}")
+    return out
+
+
+def attention(Q, K, V, causal: bool = False, scale=None, rows=None) -> np.ndarray:
+    """Reference attention forward in float64.
+
+    Q: (B, H, Sq, D), K and V: (B, H, Sk, D), fp16 (or uint16 bits).  ``scale``
+    defaults to 1/sqrt(D).  Returns (B, H, Sq, D); with ``rows`` (flat query
+    indices (b * H + h) * Sq + i) only those rows, as (len(rows), D).
+    """
+    Q, K, V = _bits(Q), _bits(K), _bits(V)
+    if Q.ndim != 4 or K.ndim != 4 or V.ndim != 4:
+        raise ValueError("Q, K, V must be (B, H, S, D)")
+    B, H, Sq, D = Q.shape
+    if K.shape[:2] != (B, H) or K.shape[3] != D or V.shape != K.shape:
+        raise ValueError("K and V must be (B, H, Sk, D) matching Q")
+    Sk = K.shape[2]
+    sc = 1.0 / np.sqrt(D) if scale is None else float(scale)
+    if rows is None:
+        r = None
+        out = np.empty((B, H, Sq, D), dtype=np.float64)
+        n = B * H * Sq
+    else:
+        r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        out = np.empty((r.size, D), dtype=np.float64)
+        n = r.size
+    st = _load().tgo_attention(_ptr(Q, ctypes.c_uint16), _ptr(K, ctypes.c_uint16),
+                               _ptr(V, ctypes.c_uint16), B, H, Sq, Sk, D, 1 if causal else 0, sc,
+                               _ptr(r, ctypes.c_int64), n, _ptr(out, ctypes.c_double))
+    if st != 0:
+        raise OracleError(f"oracle attention failed with status {st}")
     return out
 
 

@@ -30,6 +30,21 @@
  *     Source: same tutorial (ainovat.com), the row-wise softmax section (max
  *     and sum reductions per row, normalisation), here as a GEMM epilogue.
  *
+ * Attention forward (tgo_attention), for the FlashAttention kernel of the same
+ * tutorial (ainovat.com, FlashAttention section: query, key and value tiles,
+ * online softmax with running maxima and sums, causal and non-causal, checked
+ * against PyTorch's scaled dot-product attention), written as its plain
+ * definition rather than the tiled, online algorithm:
+ *
+ *   s_ij = scale * sum_d q(i,d) k(j,d),   visible(i,j) = j < Sk and (!causal or j <= i)
+ *   p_ij = exp(s_ij - max_j' s_ij') / sum_j' exp(s_ij' - max_j' s_ij')  over visible j, j'
+ *   O(i,d) = sum_j p_ij v(j,d)   (0 for a row with no visible key)
+ *
+ *   per (batch, head), Q [Sq, D], K [Sk, D], V [Sk, D], O [Sq, D], all row-major
+ *   slices of [B, H, S, D] tensors.  The causal mask keeps key j <= query i
+ *   (the lower-triangular mask of scaled dot-product attention, aligned at
+ *   the top-left corner when Sq != Sk).
+ *
  * Every fp16 x fp16 product is exact in double (11 + 11 significant bits),
  * and a double sum of at most 2^31 such terms keeps an error far below the
  * fp16 resolution of the result, so the double result is the reference;
@@ -308,4 +323,79 @@ void tgo_gelu_n(const double *x, int64_t n, double *out)
 void tgo_gelu_tanh_n(const double *x, int64_t n, double *out)
 {
     for (int64_t t = 0; t < n; ++t) out[t] = tgo_gelu_tanh(x[t]);
+}
+
+
+/* ---------------------------------------------------------------- attention */
+
+/* One query row r = (b * H + h) * Sq + i of the attention output, from the
+ * decoded K and V (double, [B, H, Sk, D]); scores holds Sk doubles. */
+static void attention_row(const uint16_t *Q, const double *Kd, const double *Vd, int64_t H,
+                          int64_t Sq, int64_t Sk, int64_t D, int causal, double scale, int64_t r,
+                          double *scores, double *q, double *out)
+{
+    const int64_t bh = r / Sq, i = r % Sq;
+    const double *K = Kd + bh * Sk * D, *V = Vd + bh * Sk * D;
+    (void)H;
+    for (int64_t d = 0; d < D; ++d) q[d] = tgo_half_to_double(Q[r * D + d]);
+    const int64_t visible = causal ? (i + 1 < Sk ? i + 1 : Sk) : Sk;
+    for (int64_t d = 0; d < D; ++d) out[d] = 0.0;
+    if (visible <= 0) return;
+    double mx = -INFINITY;
+    for (int64_t j = 0; j < visible; ++j) {
+        double acc = 0.0;
+        for (int64_t d = 0; d < D; ++d) acc += q[d] * K[j * D + d];
+        scores[j] = scale * acc;
+        if (scores[j] > mx) mx = scores[j];
+    }
+    double sum = 0.0;
+    for (int64_t j = 0; j < visible; ++j) {
+        scores[j] = exp(scores[j] - mx);
+        sum += scores[j];
+    }
+    for (int64_t j = 0; j < visible; ++j) {
+        const double w = scores[j] / sum;
+        for (int64_t d = 0; d < D; ++d) out[d] += w * V[j * D + d];
+    }
+}
+
+/* O for the query rows `rows` (flat indices (b * H + h) * Sq + i; NULL: all
+ * B * H * Sq rows in order), each D doubles, into out. */
+int tgo_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int64_t B, int64_t H,
+                  int64_t Sq, int64_t Sk, int64_t D, int causal, double scale, const int64_t *rows,
+                  int64_t nrows, double *out)
+{
+    if (!Q || !K || !V || !out || B < 0 || H < 0 || Sq < 0 || Sk < 0 || D <= 0) return TGO_ERR_ARG;
+    const int64_t total = B * H * Sq;
+    const int64_t n = rows ? nrows : total;
+    for (int64_t t = 0; rows && t < n; ++t)
+        if (rows[t] < 0 || rows[t] >= total) return TGO_ERR_RANGE;
+    if (n == 0) return TGO_OK;
+    double *Kd = decode_all(K, B * H * Sk * D);
+    double *Vd = decode_all(V, B * H * Sk * D);
+    if ((!Kd || !Vd) && B * H * Sk * D > 0) {
+        free(Kd);
+        free(Vd);
+        return TGO_ERR_ARG;
+    }
+    int err = 0;
+#pragma omp parallel
+    {
+        double *scores = malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
+        double *q = malloc(sizeof(double) * (size_t)D);
+        if (!scores || !q) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t t = 0; t < n; ++t)
+                attention_row(Q, Kd, Vd, H, Sq, Sk, D, causal, scale, rows ? rows[t] : t, scores, q,
+                              out + t * D);
+        }
+        free(scores);
+        free(q);
+    }
+    free(Kd);
+    free(Vd);
+    return err ? TGO_ERR_ARG : TGO_OK;
 }

@@ -88,6 +88,61 @@ WORKLOADS = {
 }
 
 
+@dataclasses.dataclass(frozen=True)
+class AttnWorkload:
+    """Attention forward: Q [B, H, Sq, D], K and V [B, H, Sk, D], fp16, row-major."""
+    name: str
+    B: int
+    H: int
+    Sq: int
+    Sk: int
+    D: int
+    causal: bool
+    seed: int
+
+    @property
+    def visible_pairs(self) -> int:
+        """(query, key) pairs the softmax sees: Sq*Sk, or the lower triangle."""
+        if not self.causal:
+            return self.Sq * self.Sk
+        return sum(min(i + 1, self.Sk) for i in range(self.Sq))
+
+    @property
+    def flops(self) -> int:
+        """4*D per visible (query, key) pair and head: Q.K^T and P.V, 2 flops per MAC."""
+        return 4 * self.D * self.B * self.H * self.visible_pairs
+
+    @property
+    def algorithmic_bytes(self) -> int:
+        """Read Q, K, V once and write O once (fp16)."""
+        return 2 * self.B * self.H * self.D * (2 * self.Sq + 2 * self.Sk)
+
+
+# Attention shapes: head width 64 and 128, a sequence of 2048 with 16 heads
+# and batch 4 (the common forward-pass benchmark size), causal and not, and
+# small ragged cases for parity.
+ATTN_WORKLOADS = {
+    "attn_4x16x2048x128": AttnWorkload("attn_4x16x2048x128", 4, 16, 2048, 2048, 128, False, 20),
+    "attn_causal_4x16x2048x128": AttnWorkload("attn_causal_4x16x2048x128", 4, 16, 2048, 2048,
+                                              128, True, 21),
+    "attn_4x16x2048x64": AttnWorkload("attn_4x16x2048x64", 4, 16, 2048, 2048, 64, False, 22),
+    "attn_ragged_2x3x333x64": AttnWorkload("attn_ragged_2x3x333x64", 2, 3, 333, 333, 64, True, 23),
+}
+
+
+def attention_inputs(B: int, H: int, Sq: int, Sk: int, D: int, seed: int, dist: str = "normal"):
+    """Return (Q, K, V) as CPU fp16 tensors, drawn in that order from one generator."""
+    g = torch.Generator().manual_seed(seed)
+    Q = _draw(g, (B, H, Sq, D), dist, 1.0)
+    K = _draw(g, (B, H, Sk, D), dist, 1.0)
+    V = _draw(g, (B, H, Sk, D), dist, 1.0)
+    return Q, K, V
+
+
+def attn_workload_inputs(w: AttnWorkload):
+    return attention_inputs(w.B, w.H, w.Sq, w.Sk, w.D, w.seed)
+
+
 def _draw(g: torch.Generator, shape, dist: str, scale: float) -> torch.Tensor:
     if dist == "normal":
         x = torch.randn(*shape, generator=g, dtype=torch.float32)

@@ -1,4 +1,5 @@
-"""ctypes binding of libtg_gemm.so (include/tg_gemm.h), argument marshalling only.
+"""ctypes binding of libtg_gemm.so (include/tg_gemm.h, include/tg_attention.h),
+argument marshalling only.
 
 The raw entry points keep the C names (``tg_gemm``, ``tg_gemm_ex``, ...) and
 take integers for pointers and the stream.  ``gemm`` / ``gemm_host`` are the
@@ -16,6 +17,7 @@ import re
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libtg_gemm.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "tg_gemm.h")
+HEADERS = [HEADER, os.path.join(os.path.dirname(HERE), "include", "tg_attention.h")]
 
 TG_EPILOGUE_NONE = 0
 TG_EPILOGUE_BIAS = 1
@@ -56,6 +58,10 @@ class tg_config_t(ctypes.Structure):
 
     def as_dict(self):
         return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+class tg_attention_options_t(ctypes.Structure):
+    _fields_ = [("wait_limit_ns", ctypes.c_uint64), ("inject", ctypes.c_int)]
 
 
 class tg_options_t(ctypes.Structure):
@@ -101,15 +107,24 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.tg_gemm_noalloc.restype = c_int
     lib.tg_version.argtypes = []
     lib.tg_version.restype = c_int
+    lib.tg_attention_fwd.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int,
+                                     ctypes.c_float, vp]
+    lib.tg_attention_fwd.restype = c_int
+    lib.tg_attention_fwd_ex.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int,
+                                        ctypes.c_float, ctypes.POINTER(tg_attention_options_t), vp]
+    lib.tg_attention_fwd_ex.restype = c_int
     _lib = lib
     return lib
 
 
-def header_symbols(header: str = HEADER):
-    """Function names declared in include/tg_gemm.h."""
-    text = open(header).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(tg_[a-z0-9_]+)\s*\(", text)))
+def header_symbols(headers=None):
+    """Function names declared in the library's headers (include/*.h)."""
+    names = set()
+    for header in ([headers] if isinstance(headers, str) else (headers or HEADERS)):
+        text = open(header).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names.update(re.findall(r"\b(tg_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
 
 
 # ---------------------------------------------------------------- raw entry points
@@ -235,6 +250,55 @@ def gemm(a, b, bias=None, epilogue=None, out=None, *, config_id=-1, wait_limit_n
                         stream=_stream_handle(torch, a.device), group_m=group_m, split=split)
     if st != TG_OK:
         raise TgError(st, "tg_gemm")
+    return out
+
+
+def tg_attention_fwd(Q, K, V, O, batch, heads, seq_q, seq_k, head_dim, causal, scale,
+                     stream=None) -> int:
+    return load().tg_attention_fwd(Q, K, V, O, batch, heads, seq_q, seq_k, head_dim, int(causal),
+                                   float(scale), stream)
+
+
+def tg_attention_fwd_ex(Q, K, V, O, batch, heads, seq_q, seq_k, head_dim, causal, scale,
+                        wait_limit_ns=0, inject=0, stream=None) -> int:
+    opts = tg_attention_options_t(wait_limit_ns, inject)
+    return load().tg_attention_fwd_ex(Q, K, V, O, batch, heads, seq_q, seq_k, head_dim,
+                                      int(causal), float(scale), ctypes.byref(opts), stream)
+
+
+def attention(q, k, v, causal=False, scale=0.0, out=None, *, wait_limit_ns=0, inject=0):
+    """O = softmax(scale q k^T) v on the GPU through tg_attention_fwd_ex.
+
+    q: (B, H, Sq, D), k and v: (B, H, Sk, D), fp16 contiguous CUDA tensors,
+    D in {64, 128}; scale 0 means 1/sqrt(D).  Returns ``out`` (allocated if
+    None).
+    """
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        if t is None:
+            continue
+        if t.dtype != torch.float16:
+            raise TypeError(f"{name} must be float16, got {t.dtype}")
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape or k.shape[:2] != q.shape[:2] \
+            or k.shape[3] != q.shape[3]:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}, "
+                         f"v {tuple(v.shape)}")
+    B, H, Sq, D = q.shape
+    Sk = k.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape:
+        raise ValueError(f"out must have shape {tuple(q.shape)}")
+    with torch.cuda.device(q.device):
+        st = tg_attention_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H,
+                                 Sq, Sk, D, causal, scale, wait_limit_ns=wait_limit_ns,
+                                 inject=inject, stream=_stream_handle(torch, q.device))
+    if st != TG_OK:
+        raise TgError(st, "tg_attention_fwd")
     return out
 
 

@@ -1,0 +1,593 @@
+// tg_attention.cu -- fused attention forward for sm_100a (tcgen05 + TMEM + TMA)
+// and the host side of include/tg_attention.h.
+//
+// The operation is the FlashAttention forward of "Designing High-Performance
+// GPU Kernels with TileLang" (ainovat.com, FlashAttention section): per
+// (batch, head) and tile of 128 queries, the key/value tiles are visited in
+// order; the scores S = Q K^T of one tile never leave the SM; an online
+// softmax keeps each row's running maximum m and sum l, rescaling the output
+// accumulator when m grows; O += P V; at the end O / l is written once.
+//
+// B200 design, one CTA per (batch x head, query tile), six warps:
+//   warps 0-3  softmax: thread t owns query row t (TMEM lane t).  Reads S from
+//              TMEM, masks, exponentiates, writes P (fp16) to shared memory in
+//              the tensor core's K-major 128-byte-swizzled layout, rescales O
+//              in TMEM when needed, and finally stores O / l.
+//   warp 4     TMA producer (one lane): Q once, then K and V tiles into a ring.
+//   warp 5     TMEM allocator and MMA issuer (one lane): S_j = Q K_j^T into one
+//              of two TMEM score buffers, O += P_j V_j into the TMEM output.
+// S_{j+1} is issued before P_j V_j, so the tensor core computes the next
+// scores while the softmax warps work on the current ones.
+//
+// Lazy rescaling: a row keeps its maximum m until a tile raises it by more
+// than 8 (in log2 units), so exponentials stay below 2^8 and O is rescaled
+// in TMEM only on those tiles; O / l uses the same m, so the result is the
+// same softmax.
+//
+// Every mbarrier wait is bounded by a global-timer limit; on expiry a CTA
+// abort flag is set, a site bit is OR-ed into the library error word, and
+// the CTA tears down after letting its own copies and MMAs land.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "tg_attention.h"
+#include "tg_internal.h"
+#include "tg_ptx.cuh"
+
+namespace tga {
+
+using namespace tg;
+
+constexpr int kTileQ = 128;        // queries per CTA (TMEM lanes)
+constexpr int kTileK = 128;        // keys per tile (score columns)
+constexpr int kAtom = 64;          // head-dim elements per 128-byte swizzle atom
+constexpr int kAtomBytes = 128 * 128;   // one 128-row x 64-element fp16 box
+constexpr int kThreads = 192;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr uint32_t kTmemCols = 512;     // S0 [0,128), S1 [128,256), O [256, 256 + D)
+constexpr uint32_t kOCol = 256;
+
+// Error word bits (shared word with the GEMM kernels; these sites are the
+// attention kernel's).
+constexpr unsigned kErrAttnProducer = 64u;
+constexpr unsigned kErrAttnMma = 128u;
+constexpr unsigned kErrAttnSoftmax = 256u;
+constexpr unsigned kErrAttnDrain = 512u;
+
+struct AttnParams {
+    __half *O;
+    int64_t Sq, Sk;
+    int num_bh;          // batch x heads
+    int num_qt;          // query tiles per (batch, head)
+    int causal;
+    float scale_log2;    // scale * log2(e)
+    int inject;
+    uint64_t wait_limit_ns;
+    unsigned *error_word;
+};
+
+template <int D>
+struct AttnShape {
+    static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+    static constexpr int kAtoms = D / kAtom;
+    static constexpr int kStages = D == 64 ? 4 : 2;     // K/V ring depth
+    static constexpr int kTileBytes = kAtoms * kAtomBytes;   // Q, K or V tile
+    static constexpr int kQOff = 0;
+    static constexpr int kKOff = kQOff + kTileBytes;
+    static constexpr int kVOff = kKOff + kStages * kTileBytes;
+    static constexpr int kPOff = kVOff + kStages * kTileBytes;
+    static constexpr int kPBytes = 2 * kAtomBytes;            // 128 x 128 fp16
+    // barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], s_free[2],
+    // p_full, o_done, drain
+    static constexpr int kNumBars = 1 + 3 * kStages + 4 + 3;
+    static constexpr int kBarOff = kPOff + kPBytes;
+    static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
+    static constexpr int kAbortOff = kTmemSlotOff + 4;
+    static constexpr int kDynamicBytes = kAbortOff + 4 + 1024;
+    static_assert(kDynamicBytes <= 232448, "shared-memory budget");
+};
+
+// Instruction descriptor for kind::f16 with fp32 D and both operands K-major
+// (S = Q K^T: rows of Q and of K are contiguous along the head dimension).
+__host__ __device__ constexpr uint32_t idesc_f16_f32_kk(int m, int n)
+{
+    return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst_smem, const CUtensorMap *tm,
+                                            uint64_t *bar, int32_t x, int32_t y, int32_t z)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst_smem),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x)
+{
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ float rcp(float x)
+{
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi)
+{
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const AttnParams p)
+{
+    using S = AttnShape<D>;
+    constexpr int ST = S::kStages;
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(smem);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S::kBarOff);
+    uint64_t *q_full = bars;
+    uint64_t *k_full = bars + 1;
+    uint64_t *v_full = bars + 1 + ST;
+    uint64_t *kv_empty = bars + 1 + 2 * ST;
+    uint64_t *s_full = bars + 1 + 3 * ST;
+    uint64_t *s_free = bars + 3 + 3 * ST;
+    uint64_t *p_full = bars + 5 + 3 * ST;
+    uint64_t *o_done = bars + 6 + 3 * ST;
+    uint64_t *drain_bar = bars + 7 + 3 * ST;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::kTmemSlotOff);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + S::kAbortOff);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    // Heavier query tiles first (causal: later tiles see more keys).
+    const int qt = p.num_qt - 1 - static_cast<int>(blockIdx.x / p.num_bh);
+    const int bh = static_cast<int>(blockIdx.x % p.num_bh);
+    const int64_t q0 = static_cast<int64_t>(qt) * kTileQ;
+    const int64_t kv_tiles = (p.Sk + kTileK - 1) / kTileK;
+    const int64_t kv_causal = (q0 + kTileQ - 1) / kTileK + 1;
+    const int n_kv = static_cast<int>(p.causal && kv_causal < kv_tiles ? kv_causal : kv_tiles);
+    const uint64_t limit = p.wait_limit_ns;
+
+    if (threadIdx.x == 0) {
+        // s_free and p_full take one arrival from each of the four softmax
+        // warps; every other barrier one arrival (or one commit).
+        for (int b = 0; b < S::kNumBars; ++b) {
+            uint64_t *bar = &bars[b];
+            mbar_init(bar, (bar == &s_free[0] || bar == &s_free[1] || bar == p_full) ? 4u : 1u);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kProducerWarp && lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc<1>(tmem_slot, kTmemCols);
+        tmem_relinquish<1>();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == kProducerWarp) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(q_full, S::kTileBytes);
+            for (int a = 0; a < S::kAtoms; ++a)
+                tma_load_3d(sbase + S::kQOff + a * kAtomBytes, &tmQ, q_full, a * kAtom,
+                            static_cast<int32_t>(q0), bh);
+            int filled[ST];
+            for (int s = 0; s < ST; ++s) filled[s] = 0;
+            for (int j = 0; j < n_kv; ++j) {
+                const int st = j % ST;
+                if (j >= ST && !mbar_wait_bounded(&kv_empty[st], ((j / ST) - 1) & 1, abort_flag,
+                                                  limit, p.error_word, kErrAttnProducer))
+                    break;
+                const int32_t k0 = j * kTileK;
+                const uint32_t kdst = sbase + S::kKOff + st * S::kTileBytes;
+                const uint32_t vdst = sbase + S::kVOff + st * S::kTileBytes;
+                mbar_arrive_expect_tx(&k_full[st], S::kTileBytes);
+                if (!(p.inject == 1 && blockIdx.x == 0 && j == 0))
+                    for (int a = 0; a < S::kAtoms; ++a)
+                        tma_load_3d(kdst + a * kAtomBytes, &tmK, &k_full[st], a * kAtom, k0, bh);
+                mbar_arrive_expect_tx(&v_full[st], S::kTileBytes);
+                for (int a = 0; a < S::kAtoms; ++a)
+                    tma_load_3d(vdst + a * kAtomBytes, &tmV, &v_full[st], a * kAtom, k0, bh);
+                filled[st] = j / ST + 1;
+            }
+            // Let every copy this thread issued land before shared memory goes away.
+            if (!mbar_wait_drain(q_full, 0, limit)) atomicOr(p.error_word, kErrAttnDrain);
+            for (int s = 0; s < ST; ++s)
+                if (filled[s] > 0) {
+                    const uint32_t par = (filled[s] - 1) & 1;
+                    if (!(p.inject == 1 && blockIdx.x == 0 && s == 0 && filled[s] == 1) &&
+                        !mbar_wait_drain(&k_full[s], par, limit))
+                        atomicOr(p.error_word, kErrAttnDrain);
+                    if (!mbar_wait_drain(&v_full[s], par, limit))
+                        atomicOr(p.error_word, kErrAttnDrain);
+                }
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            constexpr uint32_t kIdescS = idesc_f16_f32_kk(kTileQ, kTileK);
+            constexpr uint32_t kIdescO = idesc_f16_f32(kTileQ, D);
+            bool ok = mbar_wait_bounded(q_full, 0, abort_flag, limit, p.error_word, kErrAttnMma);
+            bool issued = false;
+            for (int j = 0; ok && j <= n_kv; ++j) {
+                if (j < n_kv) {
+                    const int st = j % ST;
+                    const int sb = j & 1;
+                    ok = mbar_wait_bounded(&k_full[st], (j / ST) & 1, abort_flag, limit,
+                                           p.error_word, kErrAttnMma);
+                    if (ok && j >= 2)
+                        ok = mbar_wait_bounded(&s_free[sb], ((j >> 1) - 1) & 1, abort_flag, limit,
+                                               p.error_word, kErrAttnMma);
+                    if (!ok) break;
+                    tc_fence_after_sync();
+                    const uint32_t qa = sbase + S::kQOff;
+                    const uint32_t ka = sbase + S::kKOff + st * S::kTileBytes;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * kAtomBytes + (kk & 3) * 32;
+                        mma_f16_ss<1>(tmem_base + sb * kTileK, smem_desc_sw128(qa + off, 16, 1024),
+                                      smem_desc_sw128(ka + off, 16, 1024), kIdescS, kk > 0);
+                    }
+                    mma_commit<1>(&s_full[sb]);
+                    issued = true;
+                }
+                if (j >= 1) {
+                    const int jj = j - 1;
+                    const int st = jj % ST;
+                    ok = mbar_wait_bounded(p_full, jj & 1, abort_flag, limit, p.error_word,
+                                           kErrAttnMma);
+                    if (ok)
+                        ok = mbar_wait_bounded(&v_full[st], (jj / ST) & 1, abort_flag, limit,
+                                               p.error_word, kErrAttnMma);
+                    if (!ok) break;
+                    tc_fence_after_sync();
+                    const uint32_t pa = sbase + S::kPOff;
+                    const uint32_t va = sbase + S::kVOff + st * S::kTileBytes;
+#pragma unroll
+                    for (int kk = 0; kk < kTileK / 16; ++kk) {
+                        const uint32_t aoff = (kk >> 2) * kAtomBytes + (kk & 3) * 32;
+                        mma_f16_ss<1>(tmem_base + kOCol, smem_desc_sw128(pa + aoff, 16, 1024),
+                                      smem_desc_sw128(va + kk * 2048, kAtomBytes, 1024), kIdescO,
+                                      (jj > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit<1>(o_done);
+                    mma_commit<1>(&kv_empty[st]);
+                }
+            }
+            if (issued) {
+                mma_commit<1>(drain_bar);
+                if (!mbar_wait_drain(drain_bar, 0, limit)) atomicOr(p.error_word, kErrAttnDrain);
+            }
+        }
+        __syncwarp();
+    } else {
+        // Softmax warps: row r of the query tile, TMEM lane r.
+        const int row = warp * 32 + lane;
+        const int64_t qi = q0 + row;
+        const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+        const float sl2 = p.scale_log2;
+        float m = -INFINITY;   // running maximum of the scaled scores, log2 units
+        float l = 0.f;         // running sum of 2^(score - m)
+        bool ok = true;
+        uint32_t P_row = sbase + S::kPOff + row * 128;
+        for (int j = 0; j < n_kv; ++j) {
+            const int sb = j & 1;
+            int okw = 1;
+            if (lane == 0)
+                okw = mbar_wait_bounded(&s_full[sb], (j >> 1) & 1, abort_flag, limit, p.error_word,
+                                        kErrAttnSoftmax)
+                          ? 1
+                          : 0;
+            okw = __shfl_sync(0xffffffffu, okw, 0);
+            if (!okw) {
+                ok = false;
+                break;
+            }
+            tc_fence_after_sync();
+            uint32_t s0[32], s1[32], s2[32], s3[32];
+            const uint32_t t_s = t_lane + static_cast<uint32_t>(sb * kTileK);
+            tmem_ld_32x32b_x32(t_s + 0, s0);
+            tmem_ld_32x32b_x32(t_s + 32, s1);
+            tmem_ld_32x32b_x32(t_s + 64, s2);
+            tmem_ld_32x32b_x32(t_s + 96, s3);
+            tmem_wait_ld_dep(s0);
+            tmem_wait_ld_dep(s1);
+            tmem_wait_ld_dep(s2);
+            tmem_wait_ld_dep(s3);
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free[sb]);
+
+            // Scale into log2 units; mask keys past seq_k and, causal, past qi.
+            const int64_t key0 = static_cast<int64_t>(j) * kTileK;
+            const bool need_mask =
+                key0 + kTileK > p.Sk || (p.causal && key0 + kTileK - 1 > q0);
+            float x[128];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                x[c] = __uint_as_float(s0[c]) * sl2;
+                x[32 + c] = __uint_as_float(s1[c]) * sl2;
+                x[64 + c] = __uint_as_float(s2[c]) * sl2;
+                x[96 + c] = __uint_as_float(s3[c]) * sl2;
+            }
+            if (need_mask) {
+                int64_t lim = p.Sk - key0;                     // keys [key0, Sk)
+                if (p.causal && qi + 1 - key0 < lim) lim = qi + 1 - key0;   // keys <= qi
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (c >= lim) x[c] = -INFINITY;
+            }
+            float mx[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) mx[t] = x[t];
+#pragma unroll
+            for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+            float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            // Lazy rescale: move m only when the tile raises it by more than 8.
+            float alpha = 1.f;
+            const bool raise = tmax > m + 8.f;
+            if (raise) {
+                alpha = (m == -INFINITY) ? 0.f : ex2(m - tmax);
+                m = tmax;
+            }
+            const float mu = (m == -INFINITY) ? 0.f : m;
+            float ps[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) ps[t] = 0.f;
+            uint32_t hp[64];
+#pragma unroll
+            for (int c = 0; c < 128; c += 2) {
+                const float e0 = ex2(x[c] - mu);
+                const float e1 = ex2(x[c + 1] - mu);
+                ps[(c >> 1) & 7] += e0 + e1;
+                hp[c >> 1] = pack_half2(e0, e1);
+            }
+            l = fmaf(l, alpha, ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
+
+            // P_{j-1} V_{j-1} must be complete before P is overwritten or O rescaled.
+            if (j > 0) {
+                if (lane == 0)
+                    okw = mbar_wait_bounded(o_done, (j - 1) & 1, abort_flag, limit, p.error_word,
+                                            kErrAttnSoftmax)
+                              ? 1
+                              : 0;
+                okw = __shfl_sync(0xffffffffu, okw, 0);
+                if (!okw) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                if (__any_sync(0xffffffffu, raise)) {
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        const uint32_t t_o = t_lane + kOCol + static_cast<uint32_t>(c * 32);
+                        tmem_ld_32x32b_x32(t_o, o);
+                        tmem_wait_ld_dep(o);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st_32x32b_x32(t_o, o);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            // P row: two 64-key atoms, 8 swizzled 16-byte chunks each.
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t addr =
+                        P_row + a * kAtomBytes + ((static_cast<uint32_t>(k) ^ (row & 7)) * 16u);
+                    const int h = a * 32 + k * 4;
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                                 "r"(hp[h]), "r"(hp[h + 1]), "r"(hp[h + 2]), "r"(hp[h + 3])
+                                 : "memory");
+                }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+        }
+        if (ok && n_kv > 0) {
+            int okw = 1;
+            if (lane == 0)
+                okw = mbar_wait_bounded(o_done, (n_kv - 1) & 1, abort_flag, limit, p.error_word,
+                                        kErrAttnSoftmax)
+                          ? 1
+                          : 0;
+            okw = __shfl_sync(0xffffffffu, okw, 0);
+            if (okw) {
+                tc_fence_after_sync();
+                const float inv_l = l > 0.f ? rcp(l) : 0.f;
+                __half *orow = p.O + (static_cast<int64_t>(bh) * p.Sq + qi) * D;
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld_32x32b_x32(t_lane + kOCol + static_cast<uint32_t>(c * 32), o);
+                    tmem_wait_ld_dep(o);
+                    if (qi < p.Sq) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint4 u;
+                            u.x = pack_half2(__uint_as_float(o[q * 8 + 0]) * inv_l,
+                                             __uint_as_float(o[q * 8 + 1]) * inv_l);
+                            u.y = pack_half2(__uint_as_float(o[q * 8 + 2]) * inv_l,
+                                             __uint_as_float(o[q * 8 + 3]) * inv_l);
+                            u.z = pack_half2(__uint_as_float(o[q * 8 + 4]) * inv_l,
+                                             __uint_as_float(o[q * 8 + 5]) * inv_l);
+                            u.w = pack_half2(__uint_as_float(o[q * 8 + 6]) * inv_l,
+                                             __uint_as_float(o[q * 8 + 7]) * inv_l);
+                            *reinterpret_cast<uint4 *>(orow + c * 32 + q * 8) = u;
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after_sync();
+        tmem_dealloc<1>(tmem_base, kTmemCols);
+    }
+}
+
+}  // namespace tga
+
+namespace {
+
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+
+bool encode_3d(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap *tm, const void *base,
+               uint64_t d, uint64_t s, uint64_t bh)
+{
+    const cuuint64_t dims[3] = {d, s, bh};
+    const cuuint64_t strides[2] = {d * 2, s * d * 2};
+    const cuuint32_t box[3] = {tga::kAtom, tga::kTileQ, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return encode(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb)
+{
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return na && nb && x < y + nb && y < x + na;
+}
+
+template <int D>
+tg_status_t launch_attn(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                        const tga::AttnParams &p, int grid, cudaStream_t stream)
+{
+    constexpr int smem = tga::AttnShape<D>::kDynamicBytes;
+    // One bit per device: the kernel's dynamic shared-memory limit is raised.
+    static std::atomic<uint64_t> attr_set{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return TG_ERR_UNSUPPORTED_DEVICE;
+    }
+    const uint64_t bit = uint64_t(1) << dev;
+    if (!(attr_set.load() & bit)) {
+        if (cudaFuncSetAttribute(tga::attn_fwd_kernel<D>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+            cudaGetLastError();
+            return TG_ERR_LAUNCH;
+        }
+        attr_set.fetch_or(bit);
+    }
+    tga::attn_fwd_kernel<D><<<grid, tga::kThreads, smem, stream>>>(tq, tk, tv, p);
+    if (cudaGetLastError() != cudaSuccess) return TG_ERR_LAUNCH;
+    return TG_OK;
+}
+
+tg_status_t attention_impl(const void *Q, const void *K, const void *V, void *O, int64_t B,
+                           int64_t H, int64_t Sq, int64_t Sk, int64_t D, int causal, float scale,
+                           const tg_attention_options_t *opts, cudaStream_t stream)
+{
+    if (B < 0 || H < 0 || Sq < 0 || Sk < 0 || (D != 64 && D != 128) || (causal != 0 && causal != 1) ||
+        !std::isfinite(scale))
+        return TG_ERR_INVALID_ARG;
+    if (opts && opts->inject != 0 && opts->inject != TG_INJECT_SKIP_FIRST_LOAD)
+        return TG_ERR_INVALID_ARG;
+    const int64_t bh = B * H;
+    if (B > 0 && H > (int64_t(1) << 31) / B) return TG_ERR_INVALID_ARG;
+    if (bh == 0 || Sq == 0) return TG_OK;
+    if (Sq > (int64_t(1) << 31) - tga::kTileQ || Sk > (int64_t(1) << 31) - tga::kTileK)
+        return TG_ERR_INVALID_ARG;
+    if (!Q || !O || (Sk > 0 && (!K || !V))) return TG_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(O) || (Sk > 0 && (!aligned16(K) || !aligned16(V))))
+        return TG_ERR_MISALIGNED;
+    const size_t qbytes = static_cast<size_t>(bh * Sq * D) * 2;
+    const size_t kvbytes = static_cast<size_t>(bh * Sk * D) * 2;
+    if (overlaps(O, qbytes, Q, qbytes) || overlaps(O, qbytes, K, kvbytes) ||
+        overlaps(O, qbytes, V, kvbytes))
+        return TG_ERR_INVALID_ARG;
+    const int64_t num_qt = (Sq + tga::kTileQ - 1) / tga::kTileQ;
+    if (bh * num_qt > 0x7fffffff) return TG_ERR_INVALID_ARG;
+
+    int num_sms = 0;
+    unsigned *error_word = nullptr;
+    PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    tg_status_t st = tg_internal_device(&num_sms, &error_word, &encode);
+    if (st != TG_OK) return st;
+    if (Sk == 0) return cudaMemsetAsync(O, 0, qbytes, stream) == cudaSuccess ? TG_OK : TG_ERR_CUDA;
+
+    CUtensorMap tq, tk, tv;
+    if (!encode_3d(encode, &tq, Q, D, Sq, bh) || !encode_3d(encode, &tk, K, D, Sk, bh) ||
+        !encode_3d(encode, &tv, V, D, Sk, bh))
+        return TG_ERR_CUDA;
+    tga::AttnParams p;
+    p.O = static_cast<__half *>(O);
+    p.Sq = Sq;
+    p.Sk = Sk;
+    p.num_bh = static_cast<int>(bh);
+    p.num_qt = static_cast<int>(num_qt);
+    p.causal = causal;
+    const float sc = scale != 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
+    p.scale_log2 = sc * 1.4426950408889634f;
+    p.inject = opts ? opts->inject : 0;
+    p.wait_limit_ns = (opts && opts->wait_limit_ns) ? opts->wait_limit_ns : kDefaultWaitLimitNs;
+    p.error_word = error_word;
+    const int grid = static_cast<int>(bh * num_qt);
+    return D == 64 ? launch_attn<64>(tq, tk, tv, p, grid, stream)
+                   : launch_attn<128>(tq, tk, tv, p, grid, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+tg_status_t tg_attention_fwd(const void *Q, const void *K, const void *V, void *O, int64_t batch,
+                             int64_t heads, int64_t seq_q, int64_t seq_k, int64_t head_dim,
+                             int causal, float scale, void *stream)
+{
+    return attention_impl(Q, K, V, O, batch, heads, seq_q, seq_k, head_dim, causal, scale, nullptr,
+                          static_cast<cudaStream_t>(stream));
+}
+
+tg_status_t tg_attention_fwd_ex(const void *Q, const void *K, const void *V, void *O,
+                                int64_t batch, int64_t heads, int64_t seq_q, int64_t seq_k,
+                                int64_t head_dim, int causal, float scale,
+                                const tg_attention_options_t *opts, void *stream)
+{
+    return attention_impl(Q, K, V, O, batch, heads, seq_q, seq_k, head_dim, causal, scale, opts,
+                          static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

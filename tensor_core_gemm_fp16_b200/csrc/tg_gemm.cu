@@ -21,6 +21,7 @@
 #include <utility>
 
 #include "tg_gemm.h"
+#include "tg_internal.h"
 #include "tg_kernels.cuh"
 
 // Per-device error word: bounded-wait expiries are OR-ed in here.
@@ -557,6 +558,18 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 }  // namespace
+
+tg_status_t tg_internal_device(int *num_sms, unsigned **error_word,
+                               PFN_cuTensorMapEncodeTiled_v12000 *encode)
+{
+    DeviceState *dev = nullptr;
+    const tg_status_t st = device_state(&dev, nullptr);
+    if (st != TG_OK) return st;
+    *num_sms = dev->num_sms;
+    *error_word = dev->error_word;
+    *encode = g_encode;
+    return g_encode ? TG_OK : TG_ERR_CUDA;
+}
 
 extern "C" {
 

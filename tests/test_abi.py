@@ -16,8 +16,25 @@ def test_library_exports_every_header_symbol():
     lib = binding.load()
     names = binding.header_symbols()
     assert "tg_gemm" in names and "tg_gemm_check_error" in names
+    assert "tg_attention_fwd" in names and "tg_attention_fwd_ex" in names
     for name in names:
-        assert hasattr(lib, name), f"{name} declared in tg_gemm.h but not exported"
+        assert hasattr(lib, name), f"{name} declared in include/*.h but not exported"
+
+
+def test_attention_host_validation_without_a_device():
+    """Every call here is rejected on the host before any device query."""
+    f = binding.tg_attention_fwd
+    q, k, v, o = 0x100000, 0x200000, 0x300000, 0x400000
+    bad = binding.TG_ERR_INVALID_ARG
+    assert f(q, k, v, o, 1, 1, 128, 128, 96, 0, 0.0) == bad            # head_dim
+    assert f(q, k, v, o, 1, 1, 128, 128, 64, 2, 0.0) == bad            # causal flag
+    assert f(q, k, v, o, -1, 1, 128, 128, 64, 0, 0.0) == bad           # negative size
+    assert f(q, k, v, o, 1, 1, 128, 128, 64, 0, float("nan")) == bad   # scale
+    assert f(None, k, v, o, 1, 1, 128, 128, 64, 0, 0.0) == bad         # null pointer
+    assert f(q, k, v, q + 64, 1, 1, 128, 128, 64, 0, 0.0) == bad       # O overlaps Q
+    assert f(q + 8, k, v, o, 1, 1, 128, 128, 64, 0, 0.0) == binding.TG_ERR_MISALIGNED
+    assert f(q, k, v, o, 0, 4, 128, 128, 64, 0, 0.0) == binding.TG_OK   # empty: no-op
+    assert binding.tg_attention_fwd_ex(q, k, v, o, 1, 1, 8, 8, 64, 0, 0.0, inject=9) == bad
 
 
 def test_status_strings():

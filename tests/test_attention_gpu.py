@@ -1,0 +1,167 @@
+"""GPU parity of the fused attention forward (tg_attention_fwd) against the
+fp64 oracle, through the C ABI.
+
+Acceptance is the library's rule: relative Frobenius error <= 2e-3 and every
+element within 1e-2 * max(1, |ref|), no NaN/Inf.  The probabilities enter the
+second product as fp16 (relative rounding 2^-11) and O is rounded to fp16 once,
+so the expected error is a few 1e-4.  Cases the mathematics makes exact are
+compared exactly.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tensor_core_gemm_fp16_b200 import binding
+from tensor_core_gemm_fp16_b200 import workloads as wl
+from gpu_helpers import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+def run_attn(Q, K, V, causal, scale=0.0, **kw):
+    dev = torch.device("cuda:0")
+    o = binding.attention(Q.to(dev), K.to(dev), V.to(dev), causal, scale, **kw)
+    torch.cuda.synchronize()
+    st = binding.tg_gemm_check_error(torch.cuda.current_stream().cuda_stream)
+    assert st == binding.TG_OK, binding.tg_status_string(st)
+    return o.cpu()
+
+
+def oracle_attn(Q, K, V, causal, scale=None, rows=None):
+    return oracle.attention(wl.to_bits(Q), wl.to_bits(K), wl.to_bits(V), causal, scale, rows=rows)
+
+
+def check(Q, K, V, causal, what, scale=0.0):
+    O = run_attn(Q, K, V, causal, scale)
+    ref = oracle_attn(Q, K, V, causal, None if scale == 0.0 else scale)
+    D = Q.shape[-1]
+    return assert_close(O.reshape(-1, D), ref.reshape(-1, D), what)
+
+
+SHAPES = [  # B, H, Sq, Sk, D
+    (1, 1, 128, 128, 64),
+    (1, 1, 128, 128, 128),
+    (2, 3, 200, 333, 64),      # ragged query and key tiles
+    (1, 2, 384, 256, 128),
+    (1, 1, 1, 1, 64),          # one query, one key
+    (1, 1, 257, 129, 128),     # more queries than keys
+    (3, 1, 64, 700, 64),       # a single partial query tile, many key tiles
+]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", SHAPES, ids=["x".join(map(str, s)) for s in SHAPES])
+def test_parity_shapes(shape, causal):
+    B, H, Sq, Sk, D = shape
+    Q, K, V = wl.attention_inputs(B, H, Sq, Sk, D, seed=100 + Sq + Sk + D)
+    check(Q, K, V, causal, f"{shape} causal={causal}")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_explicit_scale_and_large_scores(D):
+    """A large scale makes the softmax nearly one-hot and exercises the lazy
+    rescale (the running maximum moves by far more than 2^8 across tiles)."""
+    Q, K, V = wl.attention_inputs(1, 2, 256, 640, D, seed=150 + D)
+    check(Q, K, V, False, f"scale 1.0 D={D}", scale=1.0)
+    check(Q, K, V, True, f"scale 0.3 causal D={D}", scale=0.3)
+
+
+def test_increasing_scores_force_rescales():
+    """Scores that grow with the key index: every key tile raises each row's
+    maximum by more than 8 (log2 units), so O is rescaled in TMEM on every tile."""
+    B, H, S, D = 1, 1, 128, 64
+    Q = torch.zeros(B, H, S, D, dtype=torch.float16)
+    Q[..., 0] = 1.0
+    K = torch.zeros(B, H, 1024, D, dtype=torch.float16)
+    K[..., 0] = torch.linspace(0, 60, 1024, dtype=torch.float32).half()
+    _, _, V = wl.attention_inputs(B, H, S, 1024, D, seed=160)
+    check(Q, K, V, False, "increasing scores", scale=1.0)
+
+
+def test_uniform_weights_when_q_is_zero():
+    B, H, S, D = 1, 2, 300, 64
+    _, K, V = wl.attention_inputs(B, H, S, S, D, seed=161)
+    Q = torch.zeros(B, H, S, D, dtype=torch.float16)
+    v = V.to(torch.float64).numpy()
+    for causal in (False, True):
+        O = run_attn(Q, K, V, causal).to(torch.float64).numpy()
+        want = np.cumsum(v, axis=2) / np.arange(1, S + 1)[None, None, :, None] if causal else \
+            np.broadcast_to(v.mean(axis=2, keepdims=True), v.shape)
+        assert_close(O.reshape(-1, D), want.reshape(-1, D), f"uniform causal={causal}")
+
+
+def test_first_causal_row_is_v0_exactly():
+    """Query 0 sees only key 0: its weight is exactly 1, so O[0] = V[0] bit for bit."""
+    Q, K, V = wl.attention_inputs(2, 2, 130, 130, 128, seed=162)
+    O = run_attn(Q, K, V, True)
+    assert torch.equal(O[:, :, 0], V[:, :, 0])
+
+
+def test_empty_and_zero_keys():
+    dev = torch.device("cuda:0")
+    q = torch.randn(1, 2, 5, 64, device=dev).half()
+    k = torch.empty(1, 2, 0, 64, device=dev, dtype=torch.float16)
+    o = torch.full_like(q, 7.0)
+    binding.attention(q, k, k, False, out=o)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(o).item() == 0
+    q0 = torch.empty(0, 2, 5, 64, device=dev, dtype=torch.float16)
+    binding.attention(q0, q0, q0, True)
+
+
+def test_deterministic():
+    Q, K, V = wl.attention_inputs(2, 4, 512, 512, 128, seed=163)
+    a = run_attn(Q, K, V, True)
+    b = run_attn(Q, K, V, True)
+    assert torch.equal(a, b)
+
+
+def test_rejects_bad_calls():
+    dev = torch.device("cuda:0")
+    q = torch.randn(1, 1, 8, 96, device=dev).half()
+    with pytest.raises(binding.TgError) as e:
+        binding.attention(q, q.clone(), q.clone())
+    assert e.value.status == binding.TG_ERR_INVALID_ARG
+    q = torch.randn(1, 1, 8, 64, device=dev).half()
+    st = binding.tg_attention_fwd(q.data_ptr(), q.data_ptr(), q.data_ptr(), q.data_ptr(), 1, 1,
+                                  8, 8, 64, 0, 0.0)
+    assert st == binding.TG_ERR_INVALID_ARG          # O overlaps Q
+    buf = torch.zeros(1 + 8 * 64 * 4, device=dev, dtype=torch.float16)
+    st = binding.tg_attention_fwd(buf[1:].data_ptr(), q.data_ptr(), q.data_ptr(),
+                                  torch.empty_like(q).data_ptr(), 1, 1, 8, 8, 64, 0, 0.0)
+    assert st == binding.TG_ERR_MISALIGNED
+
+
+def test_timeout_injection_reports_and_recovers():
+    """The first CTA skips its first key-tile load: the MMA issuer's bounded wait
+    (50 ms) expires, the kernel exits cleanly, the status says so, and the
+    next call is correct.  Nothing faults: the load is simply never issued."""
+    Q, K, V = wl.attention_inputs(1, 2, 256, 256, 64, seed=164)
+    dev = torch.device("cuda:0")
+    binding.attention(Q.to(dev), K.to(dev), V.to(dev), False, wait_limit_ns=50_000_000,
+                      inject=binding.TG_INJECT_SKIP_FIRST_LOAD)
+    torch.cuda.synchronize()
+    st = binding.tg_gemm_check_error(torch.cuda.current_stream().cuda_stream)
+    assert st == binding.TG_ERR_TIMEOUT
+    check(Q, K, V, False, "after timeout")
+
+
+# ---------------------------------------------------------------- full-size workloads
+
+def _sample_rows(n_rows, n, seed):
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, 127, 128, 255, n_rows // 2, n_rows - 129, n_rows - 1]
+    return sorted(set(int(r) for r in fixed + list(rng.choice(n_rows, size=n, replace=False))))
+
+
+@pytest.mark.parametrize("name", list(wl.ATTN_WORKLOADS))
+def test_workload_sampled_rows(name):
+    """The full launch; every element of ~70 sampled query rows against the oracle."""
+    w = wl.ATTN_WORKLOADS[name]
+    Q, K, V = wl.attn_workload_inputs(w)
+    O = run_attn(Q, K, V, w.causal)
+    rows = _sample_rows(w.B * w.H * w.Sq, 60, seed=w.seed)
+    ref = oracle_attn(Q, K, V, w.causal, rows=rows)
+    assert_close(O.reshape(-1, w.D)[rows], ref, f"{name} sampled rows")
+    assert torch.isfinite(O.float()).all()

@@ -45,10 +45,14 @@ EPI_NAMES = {0: "none", 1: "bias", 2: "bias_gelu", 3: "bias_gelu_tanh", 4: "bias
 
 # ---------------------------------------------------------------------------- helpers
 
+GEMM_SOURCES = ("tg_configs.inc", "tg_gemm.cu", "tg_kernels.cuh", "tg_ptx.cuh")
+
+
 def kernel_source_hash() -> str:
-    """Hash of the CUDA sources; ncu traffic figures are valid only for it."""
+    """Hash of the GEMM kernel's sources (device code, launch code and the
+    configuration table); ncu traffic figures are valid only for it."""
     h = hashlib.sha256()
-    files = sorted(glob.glob(os.path.join(ROOT, "tensor_core_gemm_fp16_b200", "csrc", "*")))
+    files = [os.path.join(ROOT, "tensor_core_gemm_fp16_b200", "csrc", f) for f in GEMM_SOURCES]
     for f in files:
         with open(f, "rb") as fh:
             h.update(os.path.basename(f).encode())
@@ -273,6 +277,32 @@ def time_workload(torch, binding, w, steps, warmup, dev, stream, flush_buf, conf
             "big": big, "launch": launch, "ev": ev, "t_start": t_start, "t_end": t_end}
 
 
+def time_attention(torch, binding, w, steps, warmup, dev, stream, flush_buf):
+    """Device-resident inputs for an attention workload; the same dict shape as
+    time_workload (launch closure and per-step events)."""
+    from tensor_core_gemm_fp16_b200 import workloads as wl
+    Q, K, V = wl.attn_workload_inputs(w)
+    q, k, v = Q.to(dev), K.to(dev), V.to(dev)
+    o = torch.empty_like(q)
+    big = 2 * w.B * w.H * w.D * (2 * w.Sq + 2 * w.Sk) > L2_BYTES
+
+    def launch():
+        st = binding.tg_attention_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                      w.B, w.H, w.Sq, w.Sk, w.D, int(w.causal), 0.0,
+                                      stream.cuda_stream)
+        if st != binding.TG_OK:
+            raise binding.TgError(st, "tg_attention_fwd")
+
+    for _ in range(warmup):
+        if not big:
+            flush_buf.zero_()
+        launch()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    return {"q": q, "k": k, "v": v, "o": o, "big": big, "launch": launch, "ev": ev}
+
+
 def run_ours(args, w, rank, world):
     import torch
     import torch.distributed as dist
@@ -330,8 +360,14 @@ def run_ours(args, w, rank, world):
     for name in args.also:
         if name == w.name:
             continue
-        w2 = wl.WORKLOADS[name]
-        s2 = time_workload(torch, binding, w2, args.steps, args.warmup, dev, stream, flush_buf)
+        if name in wl.ATTN_WORKLOADS:
+            w2 = wl.ATTN_WORKLOADS[name]
+            s2 = time_attention(torch, binding, w2, args.steps, args.warmup, dev, stream,
+                                flush_buf)
+        else:
+            w2 = wl.WORKLOADS[name]
+            s2 = time_workload(torch, binding, w2, args.steps, args.warmup, dev, stream,
+                               flush_buf)
         barrier()
         torch.cuda.synchronize(dev)
         for i in range(args.steps):
@@ -344,6 +380,7 @@ def run_ours(args, w, rank, world):
         ms2 = reduce_max(statistics.mean(e0.elapsed_time(e1) for e0, e1 in s2["ev"]))
         also.append({"workload": name, "value": world * w2.flops / (ms2 * 1e-3) / 1e12,
                      "unit": UNIT, "ms_per_step": ms2,
+                     "kind": "attention" if name in wl.ATTN_WORKLOADS else "gemm",
                      "pct_of_fp16_dense_peak_nominal":
                          100.0 * w2.flops / (ms2 * 1e-3) / 1e12 / NOMINAL_FP16_DENSE_TFLOPS,
                      "l2": "flushed between launches" if not s2["big"] else "inputs larger than L2"})
@@ -461,7 +498,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="fused_8192")
     ap.add_argument("--also", nargs="*",
                     default=["gemm_2048", "fused_2048", "fused_tanh_2048", "softmax_8192x256x4096",
-                             "deepk_fused_1024x1024x8192"],
+                             "deepk_fused_1024x1024x8192", "attn_4x16x2048x128",
+                             "attn_causal_4x16x2048x128"],
                     help="other workloads timed the same way and reported under 'also'")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

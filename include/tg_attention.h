@@ -38,7 +38,7 @@ extern "C" {
  *   O        fp16 [batch, heads, seq_q, head_dim], row-major; written
  *   head_dim 64 or 128
  *   causal   0: every key; 1: key j only for query i >= j
- *   scale    factor on the scores; 0 selects 1/sqrt(head_dim)
+ *   scale    factor on the scores (|scale| >= 1e-30); 0 selects 1/sqrt(head_dim)
  *   stream   cudaStream_t (NULL: the legacy default stream)
  *
  * All four are device pointers owned by the caller, 16-byte aligned (else

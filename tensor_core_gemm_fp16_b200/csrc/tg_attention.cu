@@ -8,12 +8,17 @@
 // softmax keeps each row's running maximum m and sum l, rescaling the output
 // accumulator when m grows; O += P V; at the end O / l is written once.
 //
-// B200 design, one CTA per (batch x head, query tile), six warps:
+// B200 design, one CTA per (batch x head, query tile), seven warps:
 //   warps 0-3  softmax: thread t owns query row t (TMEM lane t).  Reads S from
 //              TMEM, masks, exponentiates, writes P (fp16) to shared memory in
 //              the tensor core's K-major 128-byte-swizzled layout, rescales O
 //              in TMEM when needed, and finally stores O / l.
-//   warp 4     TMA producer (one lane): Q once, then K and V tiles into a ring.
+//   warp 4     TMA producer (one lane): Q once, then the K tiles into their ring.
+//   warp 6     TMA producer (one lane): the V tiles into theirs.  A K slot is
+//              released as soon as its score MMA completes, a V slot after its
+//              P V MMA, so keys are fetched well ahead of their use; the two
+//              producers are separate warps so that neither's blocking wait
+//              stalls the other.
 //   warp 5     TMEM allocator and MMA issuer (one lane): S_j = Q K_j^T into one
 //              of two TMEM score buffers, O += P_j V_j into the TMEM output.
 // S_{j+1} is issued before P_j V_j, so the tensor core computes the next
@@ -23,6 +28,12 @@
 // than 8 (in log2 units), so exponentials stay below 2^8 and O is rescaled
 // in TMEM only on those tiles; O / l uses the same m, so the result is the
 // same softmax.
+//
+// Where the time goes (global-timer stamps per phase, 4 x 16 x 2048 x 128):
+// about 1.45 us per 128-key tile, of which 0.7 us are the 16384 exponentials
+// (the SFU rate, 16 per clock per SM, at the power-capped clock), and the
+// rest the row maximum, the P write and the hand-offs, which this one-tile
+// design cannot overlap with the exponentials.
 //
 // Every mbarrier wait is bounded by a global-timer limit; on expiry a CTA
 // abort flag is set, a site bit is OR-ed into the library error word, and
@@ -49,9 +60,11 @@ constexpr int kTileQ = 128;        // queries per CTA (TMEM lanes)
 constexpr int kTileK = 128;        // keys per tile (score columns)
 constexpr int kAtom = 64;          // head-dim elements per 128-byte swizzle atom
 constexpr int kAtomBytes = 128 * 128;   // one 128-row x 64-element fp16 box
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4;
+constexpr int kSoftmaxWarps = 4;
+constexpr int kProducerWarp = 4;   // Q and K
 constexpr int kMmaWarp = 5;
+constexpr int kVProducerWarp = 6;
+constexpr int kThreads = 32 * 7;
 constexpr uint32_t kTmemCols = 512;     // S0 [0,128), S1 [128,256), O [256, 256 + D)
 constexpr uint32_t kOCol = 256;
 
@@ -78,16 +91,17 @@ template <int D>
 struct AttnShape {
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
     static constexpr int kAtoms = D / kAtom;
-    static constexpr int kStages = D == 64 ? 4 : 2;     // K/V ring depth
+    static constexpr int kKStages = D == 64 ? 4 : 3;    // K ring depth
+    static constexpr int kVStages = D == 64 ? 4 : 2;    // V ring depth
     static constexpr int kTileBytes = kAtoms * kAtomBytes;   // Q, K or V tile
     static constexpr int kQOff = 0;
     static constexpr int kKOff = kQOff + kTileBytes;
-    static constexpr int kVOff = kKOff + kStages * kTileBytes;
-    static constexpr int kPOff = kVOff + kStages * kTileBytes;
+    static constexpr int kVOff = kKOff + kKStages * kTileBytes;
+    static constexpr int kPOff = kVOff + kVStages * kTileBytes;
     static constexpr int kPBytes = 2 * kAtomBytes;            // 128 x 128 fp16
-    // barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], s_free[2],
-    // p_full, o_done, drain
-    static constexpr int kNumBars = 1 + 3 * kStages + 4 + 3;
+    // barriers: q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV],
+    // s_full[2], s_free[2], p_full, o_done, drain
+    static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 4 + 3;
     static constexpr int kBarOff = kPOff + kPBytes;
     static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
     static constexpr int kAbortOff = kTmemSlotOff + 4;
@@ -139,7 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p)
 {
     using S = AttnShape<D>;
-    constexpr int ST = S::kStages;
+    constexpr int SK = S::kKStages;
+    constexpr int SV = S::kVStages;
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -148,19 +163,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S::kBarOff);
     uint64_t *q_full = bars;
     uint64_t *k_full = bars + 1;
-    uint64_t *v_full = bars + 1 + ST;
-    uint64_t *kv_empty = bars + 1 + 2 * ST;
-    uint64_t *s_full = bars + 1 + 3 * ST;
-    uint64_t *s_free = bars + 3 + 3 * ST;
-    uint64_t *p_full = bars + 5 + 3 * ST;
-    uint64_t *o_done = bars + 6 + 3 * ST;
-    uint64_t *drain_bar = bars + 7 + 3 * ST;
+    uint64_t *k_empty = k_full + SK;
+    uint64_t *v_full = k_empty + SK;
+    uint64_t *v_empty = v_full + SV;
+    uint64_t *s_full = v_empty + SV;
+    uint64_t *s_free = s_full + 2;
+    uint64_t *p_full = s_free + 2;
+    uint64_t *o_done = p_full + 1;
+    uint64_t *drain_bar = o_done + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::kTmemSlotOff);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + S::kAbortOff);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // Heavier query tiles first (causal: later tiles see more keys).
+    // Heavier query tiles first (causal: later queries see more keys).
     const int qt = p.num_qt - 1 - static_cast<int>(blockIdx.x / p.num_bh);
     const int bh = static_cast<int>(blockIdx.x % p.num_bh);
     const int64_t q0 = static_cast<int64_t>(qt) * kTileQ;
@@ -170,11 +186,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t limit = p.wait_limit_ns;
 
     if (threadIdx.x == 0) {
-        // s_free and p_full take one arrival from each of the four softmax
-        // warps; every other barrier one arrival (or one commit).
+        // s_free and p_full take one arrival from each softmax warp; every
+        // other barrier one arrival (or one commit).
         for (int b = 0; b < S::kNumBars; ++b) {
             uint64_t *bar = &bars[b];
-            mbar_init(bar, (bar == &s_free[0] || bar == &s_free[1] || bar == p_full) ? 4u : 1u);
+            mbar_init(bar, (bar == &s_free[0] || bar == &s_free[1] || bar == p_full)
+                               ? static_cast<uint32_t>(kSoftmaxWarps)
+                               : 1u);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -195,40 +213,56 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kProducerWarp) {
         if (lane == 0) {
+            // Q, then the K ring.
             mbar_arrive_expect_tx(q_full, S::kTileBytes);
             for (int a = 0; a < S::kAtoms; ++a)
                 tma_load_3d(sbase + S::kQOff + a * kAtomBytes, &tmQ, q_full, a * kAtom,
                             static_cast<int32_t>(q0), bh);
-            int filled[ST];
-            for (int s = 0; s < ST; ++s) filled[s] = 0;
+            int filled[SK];
+            for (int st = 0; st < SK; ++st) filled[st] = 0;
             for (int j = 0; j < n_kv; ++j) {
-                const int st = j % ST;
-                if (j >= ST && !mbar_wait_bounded(&kv_empty[st], ((j / ST) - 1) & 1, abort_flag,
+                const int st = j % SK;
+                if (j >= SK && !mbar_wait_bounded(&k_empty[st], ((j / SK) - 1) & 1, abort_flag,
                                                   limit, p.error_word, kErrAttnProducer))
                     break;
-                const int32_t k0 = j * kTileK;
                 const uint32_t kdst = sbase + S::kKOff + st * S::kTileBytes;
-                const uint32_t vdst = sbase + S::kVOff + st * S::kTileBytes;
                 mbar_arrive_expect_tx(&k_full[st], S::kTileBytes);
                 if (!(p.inject == 1 && blockIdx.x == 0 && j == 0))
                     for (int a = 0; a < S::kAtoms; ++a)
-                        tma_load_3d(kdst + a * kAtomBytes, &tmK, &k_full[st], a * kAtom, k0, bh);
+                        tma_load_3d(kdst + a * kAtomBytes, &tmK, &k_full[st], a * kAtom,
+                                    j * kTileK, bh);
+                filled[st] = j / SK + 1;
+            }
+            // Let every copy this thread issued land before shared memory goes away
+            // (the injected test skips one load, whose barrier never completes).
+            if (!mbar_wait_drain(q_full, 0, limit)) atomicOr(p.error_word, kErrAttnDrain);
+            for (int st = 0; st < SK; ++st)
+                if (filled[st] > 0 && !(p.inject == 1 && blockIdx.x == 0 && st == 0 &&
+                                        filled[st] == 1) &&
+                    !mbar_wait_drain(&k_full[st], (filled[st] - 1) & 1, limit))
+                    atomicOr(p.error_word, kErrAttnDrain);
+        }
+        __syncwarp();
+    } else if (warp == kVProducerWarp) {
+        if (lane == 0) {
+            // The V ring.
+            int filled[SV];
+            for (int st = 0; st < SV; ++st) filled[st] = 0;
+            for (int j = 0; j < n_kv; ++j) {
+                const int st = j % SV;
+                if (j >= SV && !mbar_wait_bounded(&v_empty[st], ((j / SV) - 1) & 1, abort_flag,
+                                                  limit, p.error_word, kErrAttnProducer))
+                    break;
+                const uint32_t vdst = sbase + S::kVOff + st * S::kTileBytes;
                 mbar_arrive_expect_tx(&v_full[st], S::kTileBytes);
                 for (int a = 0; a < S::kAtoms; ++a)
-                    tma_load_3d(vdst + a * kAtomBytes, &tmV, &v_full[st], a * kAtom, k0, bh);
-                filled[st] = j / ST + 1;
+                    tma_load_3d(vdst + a * kAtomBytes, &tmV, &v_full[st], a * kAtom, j * kTileK,
+                                bh);
+                filled[st] = j / SV + 1;
             }
-            // Let every copy this thread issued land before shared memory goes away.
-            if (!mbar_wait_drain(q_full, 0, limit)) atomicOr(p.error_word, kErrAttnDrain);
-            for (int s = 0; s < ST; ++s)
-                if (filled[s] > 0) {
-                    const uint32_t par = (filled[s] - 1) & 1;
-                    if (!(p.inject == 1 && blockIdx.x == 0 && s == 0 && filled[s] == 1) &&
-                        !mbar_wait_drain(&k_full[s], par, limit))
-                        atomicOr(p.error_word, kErrAttnDrain);
-                    if (!mbar_wait_drain(&v_full[s], par, limit))
-                        atomicOr(p.error_word, kErrAttnDrain);
-                }
+            for (int st = 0; st < SV; ++st)
+                if (filled[st] > 0 && !mbar_wait_drain(&v_full[st], (filled[st] - 1) & 1, limit))
+                    atomicOr(p.error_word, kErrAttnDrain);
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
@@ -239,9 +273,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool issued = false;
             for (int j = 0; ok && j <= n_kv; ++j) {
                 if (j < n_kv) {
-                    const int st = j % ST;
+                    const int st = j % SK;
                     const int sb = j & 1;
-                    ok = mbar_wait_bounded(&k_full[st], (j / ST) & 1, abort_flag, limit,
+                    ok = mbar_wait_bounded(&k_full[st], (j / SK) & 1, abort_flag, limit,
                                            p.error_word, kErrAttnMma);
                     if (ok && j >= 2)
                         ok = mbar_wait_bounded(&s_free[sb], ((j >> 1) - 1) & 1, abort_flag, limit,
@@ -257,15 +291,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       smem_desc_sw128(ka + off, 16, 1024), kIdescS, kk > 0);
                     }
                     mma_commit<1>(&s_full[sb]);
+                    mma_commit<1>(&k_empty[st]);
                     issued = true;
                 }
                 if (j >= 1) {
                     const int jj = j - 1;
-                    const int st = jj % ST;
+                    const int st = jj % SV;
                     ok = mbar_wait_bounded(p_full, jj & 1, abort_flag, limit, p.error_word,
                                            kErrAttnMma);
                     if (ok)
-                        ok = mbar_wait_bounded(&v_full[st], (jj / ST) & 1, abort_flag, limit,
+                        ok = mbar_wait_bounded(&v_full[st], (jj / SV) & 1, abort_flag, limit,
                                                p.error_word, kErrAttnMma);
                     if (!ok) break;
                     tc_fence_after_sync();
@@ -279,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       (jj > 0 || kk > 0) ? 1u : 0u);
                     }
                     mma_commit<1>(o_done);
-                    mma_commit<1>(&kv_empty[st]);
+                    mma_commit<1>(&v_empty[st]);
                 }
             }
             if (issued) {
@@ -294,10 +329,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t qi = q0 + row;
         const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
         const float sl2 = p.scale_log2;
+        const bool pos = sl2 > 0.f;
         float m = -INFINITY;   // running maximum of the scaled scores, log2 units
         float l = 0.f;         // running sum of 2^(score - m)
         bool ok = true;
-        uint32_t P_row = sbase + S::kPOff + row * 128;
+        const uint32_t P_row = sbase + S::kPOff + row * 128;
         for (int j = 0; j < n_kv; ++j) {
             const int sb = j & 1;
             int okw = 1;
@@ -326,32 +362,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_free[sb]);
 
-            // Scale into log2 units; mask keys past seq_k and, causal, past qi.
+            // Mask keys past seq_k and, causal, past qi, on the raw scores: the
+            // masked value turns into -inf once scaled (the scale's sign decides
+            // which infinity).  The row maximum of the scaled scores is the scale
+            // times the raw maximum (or minimum, for a negative scale), and each
+            // exponent is one fused multiply-add: 2^(s * scale * log2 e - m).
             const int64_t key0 = static_cast<int64_t>(j) * kTileK;
             const bool need_mask =
                 key0 + kTileK > p.Sk || (p.causal && key0 + kTileK - 1 > q0);
             float x[128];
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-                x[c] = __uint_as_float(s0[c]) * sl2;
-                x[32 + c] = __uint_as_float(s1[c]) * sl2;
-                x[64 + c] = __uint_as_float(s2[c]) * sl2;
-                x[96 + c] = __uint_as_float(s3[c]) * sl2;
+                x[c] = __uint_as_float(s0[c]);
+                x[32 + c] = __uint_as_float(s1[c]);
+                x[64 + c] = __uint_as_float(s2[c]);
+                x[96 + c] = __uint_as_float(s3[c]);
             }
             if (need_mask) {
                 int64_t lim = p.Sk - key0;                     // keys [key0, Sk)
                 if (p.causal && qi + 1 - key0 < lim) lim = qi + 1 - key0;   // keys <= qi
+                const float masked = pos ? -INFINITY : INFINITY;
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
-                    if (c >= lim) x[c] = -INFINITY;
+                    if (c >= lim) x[c] = masked;
             }
             float mx[8];
 #pragma unroll
             for (int t = 0; t < 8; ++t) mx[t] = x[t];
+            if (pos) {
 #pragma unroll
-            for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-            float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+            } else {
+#pragma unroll
+                for (int c = 8; c < 128; ++c) mx[c & 7] = fminf(mx[c & 7], x[c]);
+            }
+            const float rext = pos ? fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])))
+                                   : fminf(fminf(fminf(mx[0], mx[1]), fminf(mx[2], mx[3])),
+                                           fminf(fminf(mx[4], mx[5]), fminf(mx[6], mx[7])));
+            const float tmax = rext * sl2;
             // Lazy rescale: move m only when the tile raises it by more than 8.
             float alpha = 1.f;
             const bool raise = tmax > m + 8.f;
@@ -366,8 +415,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t hp[64];
 #pragma unroll
             for (int c = 0; c < 128; c += 2) {
-                const float e0 = ex2(x[c] - mu);
-                const float e1 = ex2(x[c + 1] - mu);
+                const float e0 = ex2(fmaf(x[c], sl2, -mu));
+                const float e1 = ex2(fmaf(x[c + 1], sl2, -mu));
                 ps[(c >> 1) & 7] += e0 + e1;
                 hp[c >> 1] = pack_half2(e0, e1);
             }
@@ -521,7 +570,7 @@ tg_status_t attention_impl(const void *Q, const void *K, const void *V, void *O,
                            const tg_attention_options_t *opts, cudaStream_t stream)
 {
     if (B < 0 || H < 0 || Sq < 0 || Sk < 0 || (D != 64 && D != 128) || (causal != 0 && causal != 1) ||
-        !std::isfinite(scale))
+        !std::isfinite(scale) || (scale != 0.f && std::fabs(scale) < 1e-30f))
         return TG_ERR_INVALID_ARG;
     if (opts && opts->inject != 0 && opts->inject != TG_INJECT_SKIP_FIRST_LOAD)
         return TG_ERR_INVALID_ARG;

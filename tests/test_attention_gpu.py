@@ -65,6 +65,7 @@ def test_explicit_scale_and_large_scores(D):
     Q, K, V = wl.attention_inputs(1, 2, 256, 640, D, seed=150 + D)
     check(Q, K, V, False, f"scale 1.0 D={D}", scale=1.0)
     check(Q, K, V, True, f"scale 0.3 causal D={D}", scale=0.3)
+    check(Q, K, V, True, f"scale -0.2 causal D={D}", scale=-0.2)   # the maximum is -0.2 x min
 
 
 def test_increasing_scores_force_rescales():

@@ -136,6 +136,11 @@ tg_status_t tg_gemm(const void *A, const void *B, const void *bias, void *C,
  *   split      from tg_gemm_select_config: how tg_gemm divides that problem
  *              among the SMs, TG_SPLIT_TILES or TG_SPLIT_STREAM_K; 0 from
  *              tg_config_info
+ *   loader     how operand tiles reach shared memory: 0 TMA (operands whose
+ *              rows are not 16-byte aligned are first repacked into padded
+ *              scratch), 1 plain loads by four loader warps (any row pitch,
+ *              no repacking; latency-bound, so chosen only by config_id or a
+ *              table row -- the default for unaligned rows is the repack)
  */
 typedef struct {
     int id;
@@ -147,6 +152,7 @@ typedef struct {
     int group_m;
     int epi_warps;
     int split;
+    int loader;
 } tg_config_t;
 
 /* Number of compiled tile configurations. */
@@ -232,10 +238,12 @@ tg_status_t tg_gemm_host(const void *A_host, const void *B_host, const void *bia
 
 /*
  * tg_gemm_launch_count -- number of kernels tg_gemm would launch for these
- * arguments (host only, no device call): 0 for an empty problem, 1 for the
- * GEMM kernel (or the K == 0 kernel), plus one repacking kernel for each of
- * A and B whose base address or row pitch is not a multiple of 16 bytes.
- * Returns -1 if the arguments would be rejected.
+ * arguments (host only, no device call; the configuration choice assumes
+ * 148 SMs): 0 for an empty problem, 1 for the GEMM kernel (or the K == 0
+ * kernel), plus one repacking kernel for each of A and B whose base address
+ * or row pitch is not a multiple of 16 bytes when the chosen configuration
+ * loads with TMA (a table row choosing a plain-loader configuration repacks
+ * nothing).  Returns -1 if the arguments would be rejected.
  */
 int tg_gemm_launch_count(const void *A, const void *B, const void *bias, const void *C,
                          int64_t M, int64_t N, int64_t K, int epilogue);

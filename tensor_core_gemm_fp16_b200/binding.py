@@ -54,7 +54,8 @@ class TgError(RuntimeError):
 class tg_config_t(ctypes.Structure):
     _fields_ = [("id", ctypes.c_int), ("block_m", ctypes.c_int), ("block_n", ctypes.c_int),
                 ("block_k", ctypes.c_int), ("stages", ctypes.c_int), ("cta_pair", ctypes.c_int),
-                ("group_m", ctypes.c_int), ("epi_warps", ctypes.c_int), ("split", ctypes.c_int)]
+                ("group_m", ctypes.c_int), ("epi_warps", ctypes.c_int), ("split", ctypes.c_int),
+                ("loader", ctypes.c_int)]
 
     def as_dict(self):
         return {name: getattr(self, name) for name, _ in self._fields_}

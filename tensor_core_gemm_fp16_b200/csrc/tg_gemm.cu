@@ -53,13 +53,13 @@ cudaError_t ensure_smem_attr(Kernel kern, int smem, std::atomic<uint64_t> &attr_
     return cudaSuccess;
 }
 
-template <int BN, int BK, int ST_REQ, int EPI, bool PAIR, int EW, int STORE>
+template <int BN, int BK, int ST_REQ, int EPI, bool PAIR, int EW, int STORE, int LOAD>
 cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc,
                         const tg::GemmParams &p, int grid, cudaStream_t stream)
 {
-    constexpr int ST = tg::FittedStages<BN, BK, ST_REQ, PAIR, EW, STORE>::value;
-    using S = tg::KernelShape<BN, BK, ST, PAIR, EW, STORE>;
-    auto kern = tg::gemm_persistent_kernel<BN, BK, ST, EPI, PAIR, EW, STORE>;
+    constexpr int ST = tg::FittedStages<BN, BK, ST_REQ, PAIR, EW, STORE, LOAD>::value;
+    using S = tg::KernelShape<BN, BK, ST, PAIR, EW, STORE, LOAD>;
+    auto kern = tg::gemm_persistent_kernel<BN, BK, ST, EPI, PAIR, EW, STORE, LOAD>;
     static std::atomic<uint64_t> attr_set{0};
     cudaError_t e = ensure_smem_attr(kern, S::kDynamicBytes, attr_set);
     if (e != cudaSuccess) return e;
@@ -93,11 +93,11 @@ cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const CUte
 
 // The row-softmax epilogue needs each epilogue thread to own a whole row,
 // i.e. 4 epilogue warps; other shapes have no softmax kernel.
-template <int BN, int BK, int ST, bool PAIR, int EW, int STORE>
+template <int BN, int BK, int ST, bool PAIR, int EW, int STORE, int LOAD>
 constexpr LaunchFn softmax_fn()
 {
     if constexpr (EW == 4)
-        return launch_gemm<BN, BK, ST, TG_EPILOGUE_BIAS_SOFTMAX, PAIR, EW, STORE>;
+        return launch_gemm<BN, BK, ST, TG_EPILOGUE_BIAS_SOFTMAX, PAIR, EW, STORE, LOAD>;
     else
         return nullptr;
 }
@@ -110,35 +110,40 @@ struct KernelConfig {
     LaunchFn fn[kNumEpilogues][2];   // [epilogue][0: element stores, 1: store_pref]
 };
 
-#define TG_FNS(BN, BK, ST, PAIR, EW, SP)                                                    \
+#define TG_FNS(BN, BK, ST, PAIR, EW, SP, LD)                                                \
     {                                                                                       \
-        {launch_gemm<BN, BK, ST, 0, PAIR, EW, tg::kStoreScalar>,                            \
-         launch_gemm<BN, BK, ST, 0, PAIR, EW, SP>},                                         \
-            {launch_gemm<BN, BK, ST, 1, PAIR, EW, tg::kStoreScalar>,                        \
-             launch_gemm<BN, BK, ST, 1, PAIR, EW, SP>},                                     \
-            {launch_gemm<BN, BK, ST, 2, PAIR, EW, tg::kStoreScalar>,                        \
-             launch_gemm<BN, BK, ST, 2, PAIR, EW, SP>},                                     \
-            {launch_gemm<BN, BK, ST, 3, PAIR, EW, tg::kStoreScalar>,                        \
-             launch_gemm<BN, BK, ST, 3, PAIR, EW, SP>},                                     \
-            {softmax_fn<BN, BK, ST, PAIR, EW, tg::kStoreScalar>(),                          \
-             softmax_fn<BN, BK, ST, PAIR, EW, SP>()},                                       \
+        {launch_gemm<BN, BK, ST, 0, PAIR, EW, tg::kStoreScalar, LD>,                        \
+         launch_gemm<BN, BK, ST, 0, PAIR, EW, SP, LD>},                                     \
+            {launch_gemm<BN, BK, ST, 1, PAIR, EW, tg::kStoreScalar, LD>,                    \
+             launch_gemm<BN, BK, ST, 1, PAIR, EW, SP, LD>},                                 \
+            {launch_gemm<BN, BK, ST, 2, PAIR, EW, tg::kStoreScalar, LD>,                    \
+             launch_gemm<BN, BK, ST, 2, PAIR, EW, SP, LD>},                                 \
+            {launch_gemm<BN, BK, ST, 3, PAIR, EW, tg::kStoreScalar, LD>,                    \
+             launch_gemm<BN, BK, ST, 3, PAIR, EW, SP, LD>},                                 \
+            {softmax_fn<BN, BK, ST, PAIR, EW, tg::kStoreScalar, LD>(),                      \
+             softmax_fn<BN, BK, ST, PAIR, EW, SP, LD>()},                                   \
     }
 
-#define TG_CONFIG(ID, BN, BK, ST, PAIR, EW, SP, GROUP)                                      \
-    {{ID, 128 * ((PAIR) ? 2 : 1), BN, BK, ST, (PAIR) ? 1 : 0, GROUP, EW}, SP,               \
-     TG_FNS(BN, BK, ST, PAIR, EW, SP)}
+#define TG_CONFIG(ID, BN, BK, ST, PAIR, EW, SP, GROUP, LD)                                  \
+    {{ID, 128 * ((PAIR) ? 2 : 1), BN, BK, ST, (PAIR) ? 1 : 0, GROUP, EW, 0, LD}, SP,        \
+     TG_FNS(BN, BK, ST, PAIR, EW, SP, LD)}
 
-// {id, BN, BK, stages, CTA pair, epilogue warps, store mode for aligned C, group_m}
+// {id, BN, BK, stages, CTA pair, epilogue warps, store mode for aligned C, group_m, loader}
+// Configurations 9 and 10 load operands with plain loads (any row pitch, no
+// repacking); the others use TMA and repack operands whose rows are not
+// 16-byte aligned.
 const KernelConfig kConfigs[] = {
-    TG_CONFIG(0, 256, 128, 3, true, 8, tg::kStoreTma, 8),
-    TG_CONFIG(1, 256, 64, 6, true, 8, tg::kStoreTma, 8),
-    TG_CONFIG(2, 128, 64, 8, true, 8, tg::kStoreTma, 8),
-    TG_CONFIG(3, 256, 64, 4, false, 8, tg::kStoreTma, 8),
-    TG_CONFIG(4, 128, 64, 6, false, 8, tg::kStoreTma, 8),
-    TG_CONFIG(5, 64, 64, 8, false, 4, tg::kStoreTma, 8),
-    TG_CONFIG(6, 256, 128, 3, true, 4, tg::kStoreTma, 8),
-    TG_CONFIG(7, 256, 64, 6, true, 4, tg::kStoreTma, 8),
-    TG_CONFIG(8, 256, 64, 4, false, 4, tg::kStoreVec, 8),
+    TG_CONFIG(0, 256, 128, 3, true, 8, tg::kStoreTma, 8, tg::kLoadTma),
+    TG_CONFIG(1, 256, 64, 6, true, 8, tg::kStoreTma, 8, tg::kLoadTma),
+    TG_CONFIG(2, 128, 64, 8, true, 8, tg::kStoreTma, 8, tg::kLoadTma),
+    TG_CONFIG(3, 256, 64, 4, false, 8, tg::kStoreTma, 8, tg::kLoadTma),
+    TG_CONFIG(4, 128, 64, 6, false, 8, tg::kStoreTma, 8, tg::kLoadTma),
+    TG_CONFIG(5, 64, 64, 8, false, 4, tg::kStoreTma, 8, tg::kLoadTma),
+    TG_CONFIG(6, 256, 128, 3, true, 4, tg::kStoreTma, 8, tg::kLoadTma),
+    TG_CONFIG(7, 256, 64, 6, true, 4, tg::kStoreTma, 8, tg::kLoadTma),
+    TG_CONFIG(8, 256, 64, 4, false, 4, tg::kStoreVec, 8, tg::kLoadTma),
+    TG_CONFIG(9, 256, 64, 4, false, 4, tg::kStoreTma, 8, tg::kLoadPlain),
+    TG_CONFIG(10, 128, 64, 6, false, 4, tg::kStoreTma, 8, tg::kLoadPlain),
 };
 constexpr int kNumConfigs = sizeof(kConfigs) / sizeof(kConfigs[0]);
 
@@ -199,14 +204,19 @@ int rule_split(int id, int64_t M, int64_t N, int64_t K, int epilogue, int sms)
 }
 
 // Shapes missing from the table: the cheapest (configuration, split) among
-// the general-purpose tiles.
+// the general-purpose TMA tiles.  Operands whose rows are not 16-byte aligned
+// are repacked for them: on B200 the repacking pass plus TMA is 8 to 20 times
+// faster than the plain loader (whose loads are latency-bound), so the plain
+// loader runs only when chosen explicitly or by a table row.
 Choice rule_choice(int64_t M, int64_t N, int64_t K, int epilogue, int sms)
 {
-    const int cands[] = {0, 2, 4, 5};
-    Choice best{0, TG_SPLIT_TILES};
+    static const int cands[] = {0, 2, 4, 5};
+    const int n_cands = 4;
+    Choice best{cands[0], TG_SPLIT_TILES};
     double best_cost = 0;
     bool first = true;
-    for (int id : cands) {
+    for (int c = 0; c < n_cands; ++c) {
+        const int id = cands[c];
         const int split = rule_split(id, M, N, K, epilogue, sms);
         double dp, sk;
         split_costs(id, M, N, K, sms, &dp, &sk);
@@ -224,13 +234,17 @@ Choice rule_choice(int64_t M, int64_t N, int64_t K, int epilogue, int sms)
 // warps and block_n >= N (N <= 256).
 bool softmax_capable(const tg_config_t &c, int64_t N) { return c.epi_warps == 4 && c.block_n >= N; }
 
-Choice choose_config(int64_t M, int64_t N, int64_t K, int epilogue, int num_sms)
+// `allow_plain`: a table row may select a plain-loader configuration (not for
+// the allocation-free entry point, which keeps its repacking scratch).
+Choice choose_config(int64_t M, int64_t N, int64_t K, int epilogue, int num_sms,
+                     bool allow_plain = true)
 {
     const int sms = num_sms > 1 ? num_sms : 148;
     for (const TableRow &r : kShapeTable)
         if (r.M >= 0 && r.M == M && r.N == N && r.K == K &&
             (r.epilogue < 0 || r.epilogue == epilogue) && r.config >= 0 &&
             r.config < kNumConfigs &&
+            (allow_plain || kConfigs[r.config].info.loader == tg::kLoadTma) &&
             (epilogue != TG_EPILOGUE_BIAS_SOFTMAX || softmax_capable(kConfigs[r.config].info, N)))
             return {r.config, (r.split == TG_SPLIT_TILES || r.split == TG_SPLIT_STREAM_K)
                                   ? r.split
@@ -453,6 +467,10 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
     if (epilogue == TG_EPILOGUE_NONE) bias = nullptr;
     if (K == 0) return launch_k0(bias, C, M, N, epilogue, stream, dev->num_sms);
 
+    // TMA needs 16-byte aligned bases and pitches; otherwise repack, or load
+    // with the plain loader.
+    const bool a_aligned = aligned(A, 16) && (K % 8 == 0);
+    const bool b_aligned = aligned(B, 16) && (N % 8 == 0);
     Choice choice{0, TG_SPLIT_TILES};
     if (opts && opts->config_id >= 0)
         choice = {opts->config_id, rule_split(opts->config_id, M, N, K, epilogue, dev->num_sms)};
@@ -463,10 +481,9 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
     const int bn = cfg.info.block_n;
     if (epilogue == TG_EPILOGUE_BIAS_SOFTMAX && !softmax_capable(cfg.info, N))
         return TG_ERR_INVALID_ARG;
-
-    // TMA needs 16-byte aligned bases and pitches; otherwise repack.
-    const bool a_direct = aligned(A, 16) && (K % 8 == 0);
-    const bool b_direct = aligned(B, 16) && (N % 8 == 0);
+    const bool plain = cfg.info.loader == tg::kLoadPlain;
+    const bool a_direct = plain || a_aligned;
+    const bool b_direct = plain || b_aligned;
     const int64_t lda = a_direct ? K : (K + 7) / 8 * 8;
     const int64_t ldb = b_direct ? N : (N + 7) / 8 * 8;
     void *tmp = nullptr;
@@ -497,11 +514,13 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
     const bool c_rows16 = aligned(C, 16) && (N % 8 == 0);
     const int store = c_rows16 ? cfg.store_pref : tg::kStoreScalar;
     CUtensorMap ta, tb, tc;
+    std::memset(&ta, 0, sizeof(ta));
+    std::memset(&tb, 0, sizeof(tb));
     std::memset(&tc, 0, sizeof(tc));
-    if (!encode_2d(&ta, Aeff, K, M, 2 * lda, tg::kAtomK, tg::kBlockM,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&tb, Beff, N, K, 2 * ldb, tg::kBChunkN, cfg.info.block_k,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+    if ((!plain && (!encode_2d(&ta, Aeff, K, M, 2 * lda, tg::kAtomK, tg::kBlockM,
+                               CU_TENSOR_MAP_SWIZZLE_128B) ||
+                    !encode_2d(&tb, Beff, N, K, 2 * ldb, tg::kBChunkN, cfg.info.block_k,
+                               CU_TENSOR_MAP_SWIZZLE_128B))) ||
         (store == tg::kStoreTma &&
          !encode_2d(&tc, C, N, M, 2 * N, tg::kStoreCols, 32, CU_TENSOR_MAP_SWIZZLE_64B))) {
         if (tmp) cudaFreeAsync(tmp, stream);
@@ -509,6 +528,10 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
     }
 
     tg::GemmParams p;
+    p.A = static_cast<const __half *>(Aeff);
+    p.B = static_cast<const __half *>(Beff);
+    p.lda = lda;
+    p.ldb = ldb;
     p.bias = static_cast<const __half *>(bias);
     p.C = static_cast<__half *>(C);
     p.M = M;
@@ -659,6 +682,8 @@ int tg_gemm_launch_count(const void *A, const void *B, const void *bias, const v
     if (K == 0) return 1;
     const bool a_direct = aligned(A, 16) && (K % 8 == 0);
     const bool b_direct = aligned(B, 16) && (N % 8 == 0);
+    const Choice c = choose_config(M, N, K, epilogue, 148);
+    if (kConfigs[c.config].info.loader == tg::kLoadPlain) return 1;
     return 1 + (a_direct ? 0 : 1) + (b_direct ? 0 : 1);
 }
 
@@ -789,7 +814,8 @@ tg_status_t gemm_noalloc_impl(const void *A, const void *B, const void *bias, vo
     if (epilogue == TG_EPILOGUE_NONE) bias = nullptr;
     if (K == 0) return launch_k0(bias, C, M, N, epilogue, stream, dev->num_sms);
 
-    const int cfg_id = choose_config(M, N, K, epilogue, dev->num_sms).config;
+    const int cfg_id =
+        choose_config(M, N, K, epilogue, dev->num_sms, false).config;
     const KernelConfig &cfg = kConfigs[cfg_id];
     const void *Aeff = A, *Beff = B;
     if (!a_direct) {
@@ -817,6 +843,10 @@ tg_status_t gemm_noalloc_impl(const void *A, const void *B, const void *bias, vo
         return TG_ERR_CUDA;
 
     tg::GemmParams p;
+    p.A = static_cast<const __half *>(Aeff);
+    p.B = static_cast<const __half *>(Beff);
+    p.lda = lda;
+    p.ldb = ldb;
     p.bias = static_cast<const __half *>(bias);
     p.C = static_cast<__half *>(C);
     p.M = M;

@@ -51,8 +51,14 @@ enum : int { kEpiNone = 0, kEpiBias = 1, kEpiBiasGelu = 2, kEpiBiasGeluTanh = 3,
 // How the epilogue writes C: element stores (any pitch), 16-byte stores
 // (16-byte aligned rows), or TMA stores from a swizzled staging tile.
 enum : int { kStoreScalar = 0, kStoreVec = 1, kStoreTma = 2 };
+// How operand tiles reach shared memory: TMA (16-byte aligned bases and row
+// pitches), or plain loads by four loader warps (any pitch; 2-byte alignment).
+enum : int { kLoadTma = 0, kLoadPlain = 1 };
 
 struct GemmParams {
+    const __half *A;        // [M, lda], read by the plain loader only
+    const __half *B;        // [K, ldb], read by the plain loader only
+    int64_t lda, ldb;
     const __half *bias;     // [N] or nullptr
     __half *C;              // [M, ldc]
     int64_t M, N, K;
@@ -169,12 +175,16 @@ struct WorkIter {
 //   PAIR      two CTAs of a cluster run one cta_group::2 MMA on a 256-row tile;
 //             each loads 128 rows of A and BN/2 columns of B
 //   EPI_WARPS 4 or 8 warps drain TMEM (8: two per lane quarter, halving columns)
-template <int BN, int BK, int STAGES, bool PAIR, int EPI_WARPS, int STORE>
+//   LOAD      kLoadTma (one producer lane) or kLoadPlain (four loader warps;
+//             single CTA with 4 epilogue warps only)
+template <int BN, int BK, int STAGES, bool PAIR, int EPI_WARPS, int STORE, int LOAD = kLoadTma>
 struct KernelShape {
     static_assert(BN == 64 || BN == 128 || BN == 256, "BN must be 64, 128 or 256");
     static_assert(BK == 64 || BK == 128, "BK must be 64 or 128");
     static_assert(!PAIR || BN >= 128, "a CTA pair needs BN >= 128");
     static_assert(EPI_WARPS == 4 || EPI_WARPS == 8, "4 or 8 epilogue warps");
+    static_assert(LOAD == kLoadTma || (!PAIR && EPI_WARPS == 4),
+                  "the plain loader runs single CTAs with 4 epilogue warps");
     static constexpr int kCG = PAIR ? 2 : 1;
     static constexpr int kTileM = kBlockM * kCG;
     static constexpr int kCtaN = BN / kCG;                       // B columns loaded per CTA
@@ -205,9 +215,10 @@ struct KernelShape {
     static constexpr int kUsedBytes = kAbortOffset + 4;
     static constexpr int kDynamicBytes = kUsedBytes + 1024;     // slack for 1024-B alignment
     static constexpr uint32_t kTmemCols = 2 * BN;               // double-buffered accumulator
-    static constexpr int kProducerWarp = EPI_WARPS;
-    static constexpr int kMmaWarp = EPI_WARPS + 1;
-    static constexpr int kThreads = 32 * (EPI_WARPS + 2);
+    static constexpr int kLoaderWarps = LOAD == kLoadPlain ? 4 : 1;
+    static constexpr int kProducerWarp = EPI_WARPS;             // the first loader warp
+    static constexpr int kMmaWarp = EPI_WARPS + kLoaderWarps;
+    static constexpr int kThreads = 32 * (EPI_WARPS + kLoaderWarps + 1);
     static constexpr int kChunksPerWarp = (BN / kStoreCols) / (EPI_WARPS / 4);
     static constexpr uint32_t kTmemEmptyArrivals = kCG * EPI_WARPS;
 };
@@ -217,16 +228,41 @@ constexpr int kMaxDynamicSmem = 232448;   // 227 KiB: the sm_100 per-block opt-i
 // STAGES, reduced by one when this store mode's staging buffers would push
 // the block past the shared-memory limit (the element-store fallback of a
 // configuration tuned for direct vector stores).
-template <int BN, int BK, int STAGES, bool PAIR, int EPI_WARPS, int STORE>
+template <int BN, int BK, int STAGES, bool PAIR, int EPI_WARPS, int STORE, int LOAD = kLoadTma>
 struct FittedStages {
     static constexpr int value =
-        KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, STORE>::kDynamicBytes <= kMaxDynamicSmem
+        KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, STORE, LOAD>::kDynamicBytes <= kMaxDynamicSmem
             ? STAGES
             : STAGES - 1;
-    static_assert(
-        KernelShape<BN, BK, value, PAIR, EPI_WARPS, STORE>::kDynamicBytes <= kMaxDynamicSmem,
-        "shared-memory budget exceeded");
+    static_assert(KernelShape<BN, BK, value, PAIR, EPI_WARPS, STORE, LOAD>::kDynamicBytes <=
+                      kMaxDynamicSmem,
+                  "shared-memory budget exceeded");
 };
+
+// Eight consecutive fp16 values src[0 .. 8) of a row with `valid` of them in
+// bounds (the rest read as zero), by the widest loads their alignment allows:
+// one 16-byte load, four 4-byte loads, or element loads.  Nothing outside the
+// valid range is read.
+__device__ __forceinline__ uint4 load8_any(const __half *src, int64_t valid)
+{
+    if (valid <= 0) return make_uint4(0u, 0u, 0u, 0u);
+    const uintptr_t addr = reinterpret_cast<uintptr_t>(src);
+    if (valid >= 8) {
+        if ((addr & 15u) == 0) return __ldg(reinterpret_cast<const uint4 *>(src));
+        if ((addr & 3u) == 0) {
+            const unsigned *w = reinterpret_cast<const unsigned *>(src);
+            return make_uint4(__ldg(w), __ldg(w + 1), __ldg(w + 2), __ldg(w + 3));
+        }
+    }
+    const unsigned short *h = reinterpret_cast<const unsigned short *>(src);
+    unsigned short e[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) e[i] = i < valid ? __ldg(h + i) : static_cast<unsigned short>(0);
+    return make_uint4(e[0] | (static_cast<unsigned>(e[1]) << 16),
+                      e[2] | (static_cast<unsigned>(e[3]) << 16),
+                      e[4] | (static_cast<unsigned>(e[5]) << 16),
+                      e[6] | (static_cast<unsigned>(e[7]) << 16));
+}
 
 // Tile index -> (m tile, n tile), walking group_m M-tiles per panel so that
 // CTAs running at the same time share A rows and B columns in L2.
@@ -379,13 +415,14 @@ __device__ __forceinline__ uint4 epilogue8(const uint32_t *r, const float (&b)[8
 //   warp EPI_WARPS        TMA producer (one lane)
 //   warp EPI_WARPS + 1    TMEM allocator; MMA issuer (one lane; the leader CTA
 //                         of a pair issues for both)
-template <int BN, int BK, int STAGES, int EPI, bool PAIR, int EPI_WARPS, int STORE>
-__global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, STORE>::kThreads, 1)
+template <int BN, int BK, int STAGES, int EPI, bool PAIR, int EPI_WARPS, int STORE, int LOAD>
+__global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, STORE, LOAD>::kThreads,
+                                  1)
     gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmC, const GemmParams p)
 {
-    using S = KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, STORE>;
+    using S = KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, STORE, LOAD>;
     constexpr int CG = S::kCG;
     constexpr uint32_t kIdesc = idesc_f16_f32(S::kTileM, BN);
 
@@ -412,7 +449,7 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full_bar[s], 1);
+            mbar_init(&full_bar[s], LOAD == kLoadPlain ? 32 * S::kLoaderWarps : 1);
             mbar_init(&empty_bar[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -425,8 +462,10 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
         fence_mbar_init();
     }
     if (warp == S::kProducerWarp && lane == 0) {
-        tma_prefetch_desc(&tmA);
-        tma_prefetch_desc(&tmB);
+        if (LOAD == kLoadTma) {
+            tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB);
+        }
         if (STORE == kStoreTma) tma_prefetch_desc(&tmC);
     }
     if (warp == S::kMmaWarp) {
@@ -446,7 +485,79 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
     const uint32_t smem_base = smem_u32(smem);
     const uint64_t limit = p.wait_limit_ns;
 
-    if (warp == S::kProducerWarp) {
+    if (LOAD == kLoadPlain && warp >= S::kProducerWarp && warp < S::kMmaWarp) {
+        // Plain loader: 128 threads copy each stage's A and B tiles with global
+        // loads into the same 128-byte-swizzled layout TMA would produce (16-byte
+        // chunk c of row r at chunk c ^ (r % 8)), zero-filling past M, N and K,
+        // then publish them to the tensor core (each thread: proxy fence, then
+        // its arrival on the stage's full barrier).  Consecutive threads take
+        // consecutive chunks of one 128-byte row: coalesced reads.
+        const int lt = (warp - S::kProducerWarp) * 32 + lane;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool skip_next = (p.inject == 1 && blockIdx.x == 0 && warp == S::kProducerWarp);
+        WorkIter work(p, unit, num_units);
+        int tile, k0, k1, role;
+        bool ok = true;
+        while (ok && work.next(tile, k0, k1, role)) {
+            int mt, nt;
+            tile_coords(tile, p.num_m_tiles, p.num_n_tiles, p.group_m, mt, nt);
+            const int64_t a_row0 = static_cast<int64_t>(mt) * kBlockM;
+            const int64_t b_col0 = static_cast<int64_t>(nt) * BN;
+            for (int kb = k0; kb < k1; ++kb) {
+                int okw = 1;
+                if (lane == 0)
+                    okw = mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, abort_flag, limit,
+                                            p.error_word, kErrProducerWait)
+                              ? 1
+                              : 0;
+                okw = __shfl_sync(0xffffffffu, okw, 0);
+                if (!okw) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t a_dst = smem_base + stage * S::kStageBytes;
+                const uint32_t b_dst = a_dst + S::kABytes;
+                const int64_t kbase = static_cast<int64_t>(kb) * BK;
+#pragma unroll 2
+                for (int i = lt; i < S::kAAtoms * kBlockM * 8; i += 128) {
+                    const int q = i >> 10, r = (i >> 3) & 127, c = i & 7;
+                    const int64_t gm = a_row0 + r;
+                    const int64_t gk = kbase + q * kAtomK + c * 8;
+                    const uint4 v = gm < p.M ? load8_any(p.A + gm * p.lda + gk, p.K - gk)
+                                             : make_uint4(0u, 0u, 0u, 0u);
+                    const uint32_t addr = a_dst + q * kAAtomBytes + r * 128 +
+                                          ((static_cast<uint32_t>(c) ^ (r & 7)) * 16u);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                                 "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                                 : "memory");
+                }
+#pragma unroll 2
+                for (int i = lt; i < S::kBChunks * BK * 8; i += 128) {
+                    const int j = i / (BK * 8), rem = i % (BK * 8), r = rem >> 3, c = rem & 7;
+                    const int64_t gk = kbase + r;
+                    const int64_t gn = b_col0 + j * kBChunkN + c * 8;
+                    const uint4 v = gk < p.K ? load8_any(p.B + gk * p.ldb + gn, p.N - gn)
+                                             : make_uint4(0u, 0u, 0u, 0u);
+                    const uint32_t addr = b_dst + j * S::kBChunkBytes + r * 128 +
+                                          ((static_cast<uint32_t>(c) ^ (r & 7)) * 16u);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                                 "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                                 : "memory");
+                }
+                fence_proxy_async_smem();
+                if (skip_next)
+                    skip_next = false;   // injected fault: this stage never fills
+                else
+                    mbar_arrive(&full_bar[stage]);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        __syncwarp();
+    } else if (LOAD == kLoadTma && warp == S::kProducerWarp) {
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;

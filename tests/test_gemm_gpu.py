@@ -180,8 +180,11 @@ def test_empty_m_or_n_is_a_no_op():
         assert c.shape == (M, N)
 
 
-def test_misaligned_operands_use_the_repacking_path():
-    """Views one element off a 16-byte boundary for A, B, bias and C."""
+@pytest.mark.parametrize("config_id", [-1, 0, 3, 9])
+def test_misaligned_operands(config_id):
+    """Views one element off a 16-byte boundary for A, B, bias and C: the
+    default choice and forced TMA configurations (which repack A and B
+    first), and the plain loader (which reads them in place)."""
     dev = torch.device("cuda:0")
     M, N, K = 300, 260, 200
     A, B, bias = wl.make_inputs(M, N, K, seed=700, bias=True)
@@ -196,10 +199,10 @@ def test_misaligned_operands_use_the_repacking_path():
     a.copy_(A.to(dev))
     b.copy_(B.to(dev))
     bb.copy_(bias.to(dev))
-    binding.gemm(a, b, bb, epilogue=GELU, out=c)
+    binding.gemm(a, b, bb, epilogue=GELU, out=c, config_id=config_id)
     torch.cuda.synchronize()
     assert c_buf[0].item() == 0.0, "wrote before C"
-    assert_close(c.cpu(), run_oracle(A, B, bias, GELU), "misaligned views")
+    assert_close(c.cpu(), run_oracle(A, B, bias, GELU), f"misaligned views, config {config_id}")
 
 
 # ---------------------------------------------------------------- the workloads
@@ -250,7 +253,7 @@ def test_host_entry_matches_device_entry():
     assert torch.equal(c_host, c_dev)
 
 
-@pytest.mark.parametrize("config_id", [0, 3])
+@pytest.mark.parametrize("config_id", [0, 3, 9])
 def test_bounded_wait_reports_timeout_and_context_survives(config_id):
     """A skipped operand load makes the consumer's bounded wait expire: the
     kernel exits cleanly, the host reads TG_ERR_TIMEOUT, and the next call

@@ -3,37 +3,38 @@
 //
 // The operation is the FlashAttention forward of "Designing High-Performance
 // GPU Kernels with TileLang" (ainovat.com, FlashAttention section): per
-// (batch, head) and tile of 128 queries, the key/value tiles are visited in
+// (batch, head) and tile of queries, the key/value tiles are visited in
 // order; the scores S = Q K^T of one tile never leave the SM; an online
 // softmax keeps each row's running maximum m and sum l, rescaling the output
 // accumulator when m grows; O += P V; at the end O / l is written once.
 //
-// B200 design, one CTA per (batch x head, query tile), seven warps:
-//   warps 0-3  softmax: thread t owns query row t (TMEM lane t).  Reads S from
-//              TMEM, masks, exponentiates, writes P (fp16) to shared memory in
-//              the tensor core's K-major 128-byte-swizzled layout, rescales O
-//              in TMEM when needed, and finally stores O / l.
-//   warp 4     TMA producer (one lane): Q once, then the K tiles into their ring.
-//   warp 6     TMA producer (one lane): the V tiles into theirs.  A K slot is
-//              released as soon as its score MMA completes, a V slot after its
-//              P V MMA, so keys are fetched well ahead of their use; the two
-//              producers are separate warps so that neither's blocking wait
-//              stalls the other.
-//   warp 5     TMEM allocator and MMA issuer (one lane): S_j = Q K_j^T into one
-//              of two TMEM score buffers, O += P_j V_j into the TMEM output.
-// S_{j+1} is issued before P_j V_j, so the tensor core computes the next
-// scores while the softmax warps work on the current ones.
+// B200 design: one CTA per (batch x head, pair of 128-query tiles t = 0, 1),
+// ten warps.
+//   warps 4t .. 4t+3  softmax of tile t: thread r owns query row r of the tile
+//              (TMEM lane r).  Reads S_t from TMEM, masks, exponentiates, and
+//              writes P_t (fp16, two values per 32-bit column) back into the
+//              first 64 columns of S_t, where the tensor core reads it as the
+//              A operand of P_t V; rescales O_t in TMEM when needed; stores
+//              O_t / l at the end.
+//   warp 8     TMA producer (one lane): Q for both tiles, then the K and V
+//              tiles into their rings, polling both rings' empty barriers
+//              without blocking so neither ring waits on the other.
+//   warp 9     TMEM allocator and MMA issuer (one lane).
+// TMEM: tile t owns columns [256 t, 256 t + 128) for S_t (and P_t) and
+// [256 t + 128, 256 t + 128 + D) for O_t.  The two tiles' softmax phases
+// alternate on the SM: while one group's exponentials occupy the SFU, the
+// other's hand-offs and the tensor core's products proceed.
+//
+// Order of the MMA issuer per key tile j (each wait bounded):
+//   P_0,j V_j  ->  S_0,j+1 (after P_0,j V_j completed: it overwrites P_0,j)
+//   P_1,j V_j  ->  S_1,j+1 (likewise)
+// so a softmax group that sees S_t,j+1 complete knows P_t,j V_j is done and
+// may rescale O_t and overwrite P_t.
 //
 // Lazy rescaling: a row keeps its maximum m until a tile raises it by more
 // than 8 (in log2 units), so exponentials stay below 2^8 and O is rescaled
 // in TMEM only on those tiles; O / l uses the same m, so the result is the
 // same softmax.
-//
-// Where the time goes (global-timer stamps per phase, 4 x 16 x 2048 x 128):
-// about 1.45 us per 128-key tile, of which 0.7 us are the 16384 exponentials
-// (the SFU rate, 16 per clock per SM, at the power-capped clock), and the
-// rest the row maximum, the P write and the hand-offs, which this one-tile
-// design cannot overlap with the exponentials.
 //
 // Every mbarrier wait is bounded by a global-timer limit; on expiry a CTA
 // abort flag is set, a site bit is OR-ed into the library error word, and
@@ -56,17 +57,17 @@ namespace tga {
 
 using namespace tg;
 
-constexpr int kTileQ = 128;        // queries per CTA (TMEM lanes)
+constexpr int kTileQ = 128;        // queries per tile (TMEM lanes)
+constexpr int kTilesPerCta = 2;
 constexpr int kTileK = 128;        // keys per tile (score columns)
 constexpr int kAtom = 64;          // head-dim elements per 128-byte swizzle atom
 constexpr int kAtomBytes = 128 * 128;   // one 128-row x 64-element fp16 box
-constexpr int kSoftmaxWarps = 4;
-constexpr int kProducerWarp = 4;   // Q and K
-constexpr int kMmaWarp = 5;
-constexpr int kVProducerWarp = 6;
-constexpr int kThreads = 32 * 7;
-constexpr uint32_t kTmemCols = 512;     // S0 [0,128), S1 [128,256), O [256, 256 + D)
-constexpr uint32_t kOCol = 256;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 32 * 10;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTileCols = 256;     // per tile: S (and P) [0, 128), O [128, 128 + D)
+constexpr uint32_t kOCol = 128;
 
 // Error word bits (shared word with the GEMM kernels; these sites are the
 // attention kernel's).
@@ -79,7 +80,7 @@ struct AttnParams {
     __half *O;
     int64_t Sq, Sk;
     int num_bh;          // batch x heads
-    int num_qt;          // query tiles per (batch, head)
+    int num_qp;          // pairs of query tiles per (batch, head)
     int causal;
     float scale_log2;    // scale * log2(e)
     int inject;
@@ -93,16 +94,14 @@ struct AttnShape {
     static constexpr int kAtoms = D / kAtom;
     static constexpr int kKStages = D == 64 ? 4 : 3;    // K ring depth
     static constexpr int kVStages = D == 64 ? 4 : 2;    // V ring depth
-    static constexpr int kTileBytes = kAtoms * kAtomBytes;   // Q, K or V tile
-    static constexpr int kQOff = 0;
-    static constexpr int kKOff = kQOff + kTileBytes;
+    static constexpr int kTileBytes = kAtoms * kAtomBytes;   // one 128-row Q, K or V tile
+    static constexpr int kQOff = 0;                          // Q of both query tiles
+    static constexpr int kKOff = kQOff + kTilesPerCta * kTileBytes;
     static constexpr int kVOff = kKOff + kKStages * kTileBytes;
-    static constexpr int kPOff = kVOff + kVStages * kTileBytes;
-    static constexpr int kPBytes = 2 * kAtomBytes;            // 128 x 128 fp16
     // barriers: q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV],
-    // s_full[2], s_free[2], p_full, o_done, drain
-    static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 4 + 3;
-    static constexpr int kBarOff = kPOff + kPBytes;
+    // s_full[2], p_full[2], pv_done[2], drain
+    static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 6 + 1;
+    static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
     static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
     static constexpr int kAbortOff = kTmemSlotOff + 4;
     static constexpr int kDynamicBytes = kAbortOff + 4 + 1024;
@@ -115,6 +114,19 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32_kk(int m, int n)
 {
     return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) |
            (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// D (TMEM) += A (TMEM: 128 lanes x 16 fp16, two per 32-bit column) x B (shared
+// memory descriptor).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst_smem, const CUtensorMap *tm,
@@ -147,6 +159,17 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// Keys visible to query tile (pair qp, tile t): all key tiles, or with the
+// causal mask those up to the one holding the tile's last query; 0 for a tile
+// that lies entirely past seq_q.
+__device__ __forceinline__ int tile_key_tiles(const AttnParams &p, int64_t q0)
+{
+    if (q0 >= p.Sq) return 0;
+    const int64_t kv_tiles = (p.Sk + kTileK - 1) / kTileK;
+    const int64_t kv_causal = (q0 + kTileQ - 1) / kTileK + 1;
+    return static_cast<int>(p.causal && kv_causal < kv_tiles ? kv_causal : kv_tiles);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -166,33 +189,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *k_empty = k_full + SK;
     uint64_t *v_full = k_empty + SK;
     uint64_t *v_empty = v_full + SV;
-    uint64_t *s_full = v_empty + SV;
-    uint64_t *s_free = s_full + 2;
-    uint64_t *p_full = s_free + 2;
-    uint64_t *o_done = p_full + 1;
-    uint64_t *drain_bar = o_done + 1;
+    uint64_t *s_full = v_empty + SV;     // [2]: S_t of the current key tile is in TMEM
+    uint64_t *p_full = s_full + 2;       // [2]: P_t written to TMEM (4 arrivals)
+    uint64_t *pv_done = p_full + 2;      // [2]: P_t V complete
+    uint64_t *drain_bar = pv_done + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::kTmemSlotOff);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + S::kAbortOff);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // Heavier query tiles first (causal: later queries see more keys).
-    const int qt = p.num_qt - 1 - static_cast<int>(blockIdx.x / p.num_bh);
+    // Heavier query pairs first (causal: later queries see more keys).
+    const int qp = p.num_qp - 1 - static_cast<int>(blockIdx.x / p.num_bh);
     const int bh = static_cast<int>(blockIdx.x % p.num_bh);
-    const int64_t q0 = static_cast<int64_t>(qt) * kTileQ;
-    const int64_t kv_tiles = (p.Sk + kTileK - 1) / kTileK;
-    const int64_t kv_causal = (q0 + kTileQ - 1) / kTileK + 1;
-    const int n_kv = static_cast<int>(p.causal && kv_causal < kv_tiles ? kv_causal : kv_tiles);
+    const int64_t qbase = static_cast<int64_t>(qp) * kTilesPerCta * kTileQ;
+    const int n0 = tile_key_tiles(p, qbase);
+    const int n1 = tile_key_tiles(p, qbase + kTileQ);
+    const int n_all = n0 > n1 ? n0 : n1;
     const uint64_t limit = p.wait_limit_ns;
 
     if (threadIdx.x == 0) {
-        // s_free and p_full take one arrival from each softmax warp; every
-        // other barrier one arrival (or one commit).
         for (int b = 0; b < S::kNumBars; ++b) {
             uint64_t *bar = &bars[b];
-            mbar_init(bar, (bar == &s_free[0] || bar == &s_free[1] || bar == p_full)
-                               ? static_cast<uint32_t>(kSoftmaxWarps)
-                               : 1u);
+            mbar_init(bar, (bar == &p_full[0] || bar == &p_full[1]) ? 4u : 1u);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -212,110 +230,139 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == kProducerWarp) {
-        if (lane == 0) {
-            // Q, then the K ring.
-            mbar_arrive_expect_tx(q_full, S::kTileBytes);
-            for (int a = 0; a < S::kAtoms; ++a)
-                tma_load_3d(sbase + S::kQOff + a * kAtomBytes, &tmQ, q_full, a * kAtom,
-                            static_cast<int32_t>(q0), bh);
-            int filled[SK];
-            for (int st = 0; st < SK; ++st) filled[st] = 0;
-            for (int j = 0; j < n_kv; ++j) {
-                const int st = j % SK;
-                if (j >= SK && !mbar_wait_bounded(&k_empty[st], ((j / SK) - 1) & 1, abort_flag,
-                                                  limit, p.error_word, kErrAttnProducer))
-                    break;
-                const uint32_t kdst = sbase + S::kKOff + st * S::kTileBytes;
-                mbar_arrive_expect_tx(&k_full[st], S::kTileBytes);
-                if (!(p.inject == 1 && blockIdx.x == 0 && j == 0))
+        if (lane == 0 && n_all > 0) {
+            // Q of both tiles (rows past seq_q read as zero), then both rings.
+            mbar_arrive_expect_tx(q_full, kTilesPerCta * S::kTileBytes);
+            for (int t = 0; t < kTilesPerCta; ++t)
+                for (int a = 0; a < S::kAtoms; ++a)
+                    tma_load_3d(sbase + S::kQOff + t * S::kTileBytes + a * kAtomBytes, &tmQ,
+                                q_full, a * kAtom, static_cast<int32_t>(qbase + t * kTileQ), bh);
+            int jk = 0, jv = 0;
+            int k_filled[SK], v_filled[SV];
+            for (int st = 0; st < SK; ++st) k_filled[st] = 0;
+            for (int st = 0; st < SV; ++st) v_filled[st] = 0;
+            uint64_t t_idle = 0;
+            bool ok = true;
+            while (ok && (jk < n_all || jv < n_all)) {
+                bool progress = false;
+                if (jk < n_all &&
+                    (jk < SK || mbar_test_wait(&k_empty[jk % SK], ((jk / SK) - 1) & 1))) {
+                    const int st = jk % SK;
+                    const uint32_t kdst = sbase + S::kKOff + st * S::kTileBytes;
+                    mbar_arrive_expect_tx(&k_full[st], S::kTileBytes);
+                    if (!(p.inject == 1 && blockIdx.x == 0 && jk == 0))
+                        for (int a = 0; a < S::kAtoms; ++a)
+                            tma_load_3d(kdst + a * kAtomBytes, &tmK, &k_full[st], a * kAtom,
+                                        jk * kTileK, bh);
+                    k_filled[st] = jk / SK + 1;
+                    ++jk;
+                    progress = true;
+                }
+                if (jv < n_all &&
+                    (jv < SV || mbar_test_wait(&v_empty[jv % SV], ((jv / SV) - 1) & 1))) {
+                    const int st = jv % SV;
+                    const uint32_t vdst = sbase + S::kVOff + st * S::kTileBytes;
+                    mbar_arrive_expect_tx(&v_full[st], S::kTileBytes);
                     for (int a = 0; a < S::kAtoms; ++a)
-                        tma_load_3d(kdst + a * kAtomBytes, &tmK, &k_full[st], a * kAtom,
-                                    j * kTileK, bh);
-                filled[st] = j / SK + 1;
+                        tma_load_3d(vdst + a * kAtomBytes, &tmV, &v_full[st], a * kAtom,
+                                    jv * kTileK, bh);
+                    v_filled[st] = jv / SV + 1;
+                    ++jv;
+                    progress = true;
+                }
+                if (progress) {
+                    t_idle = 0;
+                } else {
+                    // Bounded: give up after the wait limit without progress.
+                    if (*abort_flag) break;
+                    const uint64_t now = global_timer_ns();
+                    if (t_idle == 0) {
+                        t_idle = now;
+                    } else if (now - t_idle > limit) {
+                        *abort_flag = 1;
+                        atomicOr(p.error_word, kErrAttnProducer);
+                        ok = false;
+                    }
+                }
             }
             // Let every copy this thread issued land before shared memory goes away
             // (the injected test skips one load, whose barrier never completes).
             if (!mbar_wait_drain(q_full, 0, limit)) atomicOr(p.error_word, kErrAttnDrain);
             for (int st = 0; st < SK; ++st)
-                if (filled[st] > 0 && !(p.inject == 1 && blockIdx.x == 0 && st == 0 &&
-                                        filled[st] == 1) &&
-                    !mbar_wait_drain(&k_full[st], (filled[st] - 1) & 1, limit))
+                if (k_filled[st] > 0 && !(p.inject == 1 && blockIdx.x == 0 && st == 0 &&
+                                          k_filled[st] == 1) &&
+                    !mbar_wait_drain(&k_full[st], (k_filled[st] - 1) & 1, limit))
                     atomicOr(p.error_word, kErrAttnDrain);
-        }
-        __syncwarp();
-    } else if (warp == kVProducerWarp) {
-        if (lane == 0) {
-            // The V ring.
-            int filled[SV];
-            for (int st = 0; st < SV; ++st) filled[st] = 0;
-            for (int j = 0; j < n_kv; ++j) {
-                const int st = j % SV;
-                if (j >= SV && !mbar_wait_bounded(&v_empty[st], ((j / SV) - 1) & 1, abort_flag,
-                                                  limit, p.error_word, kErrAttnProducer))
-                    break;
-                const uint32_t vdst = sbase + S::kVOff + st * S::kTileBytes;
-                mbar_arrive_expect_tx(&v_full[st], S::kTileBytes);
-                for (int a = 0; a < S::kAtoms; ++a)
-                    tma_load_3d(vdst + a * kAtomBytes, &tmV, &v_full[st], a * kAtom, j * kTileK,
-                                bh);
-                filled[st] = j / SV + 1;
-            }
             for (int st = 0; st < SV; ++st)
-                if (filled[st] > 0 && !mbar_wait_drain(&v_full[st], (filled[st] - 1) & 1, limit))
+                if (v_filled[st] > 0 && !mbar_wait_drain(&v_full[st], (v_filled[st] - 1) & 1, limit))
                     atomicOr(p.error_word, kErrAttnDrain);
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
-        if (lane == 0) {
+        if (lane == 0 && n_all > 0) {
             constexpr uint32_t kIdescS = idesc_f16_f32_kk(kTileQ, kTileK);
             constexpr uint32_t kIdescO = idesc_f16_f32(kTileQ, D);
+            const int nt[2] = {n0, n1};
             bool ok = mbar_wait_bounded(q_full, 0, abort_flag, limit, p.error_word, kErrAttnMma);
             bool issued = false;
-            for (int j = 0; ok && j <= n_kv; ++j) {
-                if (j < n_kv) {
-                    const int st = j % SK;
-                    const int sb = j & 1;
-                    ok = mbar_wait_bounded(&k_full[st], (j / SK) & 1, abort_flag, limit,
-                                           p.error_word, kErrAttnMma);
-                    if (ok && j >= 2)
-                        ok = mbar_wait_bounded(&s_free[sb], ((j >> 1) - 1) & 1, abort_flag, limit,
-                                               p.error_word, kErrAttnMma);
-                    if (!ok) break;
-                    tc_fence_after_sync();
-                    const uint32_t qa = sbase + S::kQOff;
-                    const uint32_t ka = sbase + S::kKOff + st * S::kTileBytes;
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * kAtomBytes + (kk & 3) * 32;
-                        mma_f16_ss<1>(tmem_base + sb * kTileK, smem_desc_sw128(qa + off, 16, 1024),
-                                      smem_desc_sw128(ka + off, 16, 1024), kIdescS, kk > 0);
-                    }
-                    mma_commit<1>(&s_full[sb]);
-                    mma_commit<1>(&k_empty[st]);
-                    issued = true;
-                }
-                if (j >= 1) {
-                    const int jj = j - 1;
-                    const int st = jj % SV;
-                    ok = mbar_wait_bounded(p_full, jj & 1, abort_flag, limit, p.error_word,
+            auto wait = [&](uint64_t *bar, uint32_t parity) {
+                if (ok)
+                    ok = mbar_wait_bounded(bar, parity, abort_flag, limit, p.error_word,
                                            kErrAttnMma);
-                    if (ok)
-                        ok = mbar_wait_bounded(&v_full[st], (jj / SV) & 1, abort_flag, limit,
-                                               p.error_word, kErrAttnMma);
-                    if (!ok) break;
-                    tc_fence_after_sync();
-                    const uint32_t pa = sbase + S::kPOff;
-                    const uint32_t va = sbase + S::kVOff + st * S::kTileBytes;
+                return ok;
+            };
+            // S_t,j = Q_t K_j^T into tile t's score columns.
+            auto issue_s = [&](int t, int j) {
+                const uint32_t qa = sbase + S::kQOff + t * S::kTileBytes;
+                const uint32_t ka = sbase + S::kKOff + (j % SK) * S::kTileBytes;
+                tc_fence_after_sync();
 #pragma unroll
-                    for (int kk = 0; kk < kTileK / 16; ++kk) {
-                        const uint32_t aoff = (kk >> 2) * kAtomBytes + (kk & 3) * 32;
-                        mma_f16_ss<1>(tmem_base + kOCol, smem_desc_sw128(pa + aoff, 16, 1024),
-                                      smem_desc_sw128(va + kk * 2048, kAtomBytes, 1024), kIdescO,
-                                      (jj > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    mma_commit<1>(o_done);
-                    mma_commit<1>(&v_empty[st]);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kAtomBytes + (kk & 3) * 32;
+                    mma_f16_ss<1>(tmem_base + t * kTileCols, smem_desc_sw128(qa + off, 16, 1024),
+                                  smem_desc_sw128(ka + off, 16, 1024), kIdescS, kk > 0);
                 }
+                mma_commit<1>(&s_full[t]);
+                issued = true;
+            };
+            // O_t += P_t,j V_j, P_t from TMEM (8 columns per 16 keys).
+            auto issue_pv = [&](int t, int j) {
+                const uint32_t va = sbase + S::kVOff + (j % SV) * S::kTileBytes;
+                tc_fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < kTileK / 16; ++kk)
+                    mma_f16_ts(tmem_base + t * kTileCols + kOCol,
+                               tmem_base + t * kTileCols + static_cast<uint32_t>(kk * 8),
+                               smem_desc_sw128(va + kk * 2048, kAtomBytes, 1024), kIdescO,
+                               (j > 0 || kk > 0) ? 1u : 0u);
+                mma_commit<1>(&pv_done[t]);
+                issued = true;
+            };
+            if (wait(&k_full[0], 0)) {
+                for (int t = 0; t < 2; ++t)
+                    if (nt[t] > 0) issue_s(t, 0);
+                mma_commit<1>(&k_empty[0]);
+            }
+            for (int j = 0; ok && j < n_all; ++j) {
+                if (!wait(&v_full[j % SV], (j / SV) & 1)) break;
+                const bool next = j + 1 < n_all;
+                bool k_next = false;   // K_j+1 waited for
+                for (int t = 0; t < 2 && ok; ++t) {
+                    if (j < nt[t]) {
+                        if (!wait(&p_full[t], j & 1)) break;
+                        issue_pv(t, j);
+                    }
+                    if (j + 1 < nt[t]) {
+                        if (!k_next && !wait(&k_full[(j + 1) % SK], ((j + 1) / SK) & 1)) break;
+                        k_next = true;
+                        // S_t,j+1 overwrites P_t,j: only after P_t,j V_j completed.
+                        if (!wait(&pv_done[t], j & 1)) break;
+                        issue_s(t, j + 1);
+                    }
+                }
+                if (!ok) break;
+                mma_commit<1>(&v_empty[j % SV]);
+                if (next) mma_commit<1>(&k_empty[(j + 1) % SK]);
             }
             if (issued) {
                 mma_commit<1>(drain_bar);
@@ -324,21 +371,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else {
-        // Softmax warps: row r of the query tile, TMEM lane r.
-        const int row = warp * 32 + lane;
+        // Softmax group t = warp / 4: row r = 32 (warp % 4) + lane of query tile t.
+        const int t = warp >> 2;
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const int64_t q0 = qbase + static_cast<int64_t>(t) * kTileQ;
         const int64_t qi = q0 + row;
-        const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+        const int n_kv = t == 0 ? n0 : n1;
+        const uint32_t t_lane =
+            tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + t * kTileCols;
         const float sl2 = p.scale_log2;
         const bool pos = sl2 > 0.f;
         float m = -INFINITY;   // running maximum of the scaled scores, log2 units
         float l = 0.f;         // running sum of 2^(score - m)
         bool ok = true;
-        const uint32_t P_row = sbase + S::kPOff + row * 128;
         for (int j = 0; j < n_kv; ++j) {
-            const int sb = j & 1;
             int okw = 1;
             if (lane == 0)
-                okw = mbar_wait_bounded(&s_full[sb], (j >> 1) & 1, abort_flag, limit, p.error_word,
+                okw = mbar_wait_bounded(&s_full[t], j & 1, abort_flag, limit, p.error_word,
                                         kErrAttnSoftmax)
                           ? 1
                           : 0;
@@ -349,18 +399,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after_sync();
             uint32_t s0[32], s1[32], s2[32], s3[32];
-            const uint32_t t_s = t_lane + static_cast<uint32_t>(sb * kTileK);
-            tmem_ld_32x32b_x32(t_s + 0, s0);
-            tmem_ld_32x32b_x32(t_s + 32, s1);
-            tmem_ld_32x32b_x32(t_s + 64, s2);
-            tmem_ld_32x32b_x32(t_s + 96, s3);
+            tmem_ld_32x32b_x32(t_lane + 0, s0);
+            tmem_ld_32x32b_x32(t_lane + 32, s1);
+            tmem_ld_32x32b_x32(t_lane + 64, s2);
+            tmem_ld_32x32b_x32(t_lane + 96, s3);
             tmem_wait_ld_dep(s0);
             tmem_wait_ld_dep(s1);
             tmem_wait_ld_dep(s2);
             tmem_wait_ld_dep(s3);
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_free[sb]);
 
             // Mask keys past seq_k and, causal, past qi, on the raw scores: the
             // masked value turns into -inf once scaled (the scale's sign decides
@@ -388,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             float mx[8];
 #pragma unroll
-            for (int t = 0; t < 8; ++t) mx[t] = x[t];
+            for (int u = 0; u < 8; ++u) mx[u] = x[u];
             if (pos) {
 #pragma unroll
                 for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
@@ -409,69 +455,49 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m = tmax;
             }
             const float mu = (m == -INFINITY) ? 0.f : m;
+            // P_t,j-1 V_j-1 is complete (S_t,j was issued after it): O_t may be
+            // rescaled and P_t overwritten.
+            if (j > 0 && __any_sync(0xffffffffu, raise)) {
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    const uint32_t t_o = t_lane + kOCol + static_cast<uint32_t>(c * 32);
+                    tmem_ld_32x32b_x32(t_o, o);
+                    tmem_wait_ld_dep(o);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st_32x32b_x32(t_o, o);
+                }
+            }
+            // P row into TMEM columns [0, 64): two halves of 64 keys, 32 packed
+            // columns each.
             float ps[8];
 #pragma unroll
-            for (int t = 0; t < 8; ++t) ps[t] = 0.f;
-            uint32_t hp[64];
+            for (int u = 0; u < 8; ++u) ps[u] = 0.f;
 #pragma unroll
-            for (int c = 0; c < 128; c += 2) {
-                const float e0 = ex2(fmaf(x[c], sl2, -mu));
-                const float e1 = ex2(fmaf(x[c + 1], sl2, -mu));
-                ps[(c >> 1) & 7] += e0 + e1;
-                hp[c >> 1] = pack_half2(e0, e1);
+            for (int h = 0; h < 2; ++h) {
+                uint32_t hp[32];
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) {
+                    const float e0 = ex2(fmaf(x[h * 64 + c], sl2, -mu));
+                    const float e1 = ex2(fmaf(x[h * 64 + c + 1], sl2, -mu));
+                    ps[(c >> 1) & 7] += e0 + e1;
+                    hp[c >> 1] = pack_half2(e0, e1);
+                }
+                tmem_st_32x32b_x32(t_lane + static_cast<uint32_t>(h * 32), hp);
             }
             l = fmaf(l, alpha, ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
-
-            // P_{j-1} V_{j-1} must be complete before P is overwritten or O rescaled.
-            if (j > 0) {
-                if (lane == 0)
-                    okw = mbar_wait_bounded(o_done, (j - 1) & 1, abort_flag, limit, p.error_word,
-                                            kErrAttnSoftmax)
-                              ? 1
-                              : 0;
-                okw = __shfl_sync(0xffffffffu, okw, 0);
-                if (!okw) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after_sync();
-                if (__any_sync(0xffffffffu, raise)) {
-#pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t o[32];
-                        const uint32_t t_o = t_lane + kOCol + static_cast<uint32_t>(c * 32);
-                        tmem_ld_32x32b_x32(t_o, o);
-                        tmem_wait_ld_dep(o);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st_32x32b_x32(t_o, o);
-                    }
-                    tmem_wait_st();
-                }
-            }
-            // P row: two 64-key atoms, 8 swizzled 16-byte chunks each.
-#pragma unroll
-            for (int a = 0; a < 2; ++a)
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint32_t addr =
-                        P_row + a * kAtomBytes + ((static_cast<uint32_t>(k) ^ (row & 7)) * 16u);
-                    const int h = a * 32 + k * 4;
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                                 "r"(hp[h]), "r"(hp[h + 1]), "r"(hp[h + 2]), "r"(hp[h + 3])
-                                 : "memory");
-                }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(&p_full[t]);
         }
         if (ok && n_kv > 0) {
             int okw = 1;
             if (lane == 0)
-                okw = mbar_wait_bounded(o_done, (n_kv - 1) & 1, abort_flag, limit, p.error_word,
-                                        kErrAttnSoftmax)
+                okw = mbar_wait_bounded(&pv_done[t], (n_kv - 1) & 1, abort_flag, limit,
+                                        p.error_word, kErrAttnSoftmax)
                           ? 1
                           : 0;
             okw = __shfl_sync(0xffffffffu, okw, 0);
@@ -587,8 +613,9 @@ tg_status_t attention_impl(const void *Q, const void *K, const void *V, void *O,
     if (overlaps(O, qbytes, Q, qbytes) || overlaps(O, qbytes, K, kvbytes) ||
         overlaps(O, qbytes, V, kvbytes))
         return TG_ERR_INVALID_ARG;
-    const int64_t num_qt = (Sq + tga::kTileQ - 1) / tga::kTileQ;
-    if (bh * num_qt > 0x7fffffff) return TG_ERR_INVALID_ARG;
+    const int64_t pair_rows = static_cast<int64_t>(tga::kTilesPerCta) * tga::kTileQ;
+    const int64_t num_qp = (Sq + pair_rows - 1) / pair_rows;
+    if (bh * num_qp > 0x7fffffff) return TG_ERR_INVALID_ARG;
 
     int num_sms = 0;
     unsigned *error_word = nullptr;
@@ -606,14 +633,14 @@ tg_status_t attention_impl(const void *Q, const void *K, const void *V, void *O,
     p.Sq = Sq;
     p.Sk = Sk;
     p.num_bh = static_cast<int>(bh);
-    p.num_qt = static_cast<int>(num_qt);
+    p.num_qp = static_cast<int>(num_qp);
     p.causal = causal;
     const float sc = scale != 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
     p.scale_log2 = sc * 1.4426950408889634f;
     p.inject = opts ? opts->inject : 0;
     p.wait_limit_ns = (opts && opts->wait_limit_ns) ? opts->wait_limit_ns : kDefaultWaitLimitNs;
     p.error_word = error_word;
-    const int grid = static_cast<int>(bh * num_qt);
+    const int grid = static_cast<int>(bh * num_qp);
     return D == 64 ? launch_attn<64>(tq, tk, tv, p, grid, stream)
                    : launch_attn<128>(tq, tk, tv, p, grid, stream);
 }

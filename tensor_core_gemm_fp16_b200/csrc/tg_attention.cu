@@ -20,16 +20,21 @@
 //              tiles into their rings, polling both rings' empty barriers
 //              without blocking so neither ring waits on the other.
 //   warp 9     TMEM allocator and MMA issuer (one lane).
-// TMEM: tile t owns columns [256 t, 256 t + 128) for S_t (and P_t) and
-// [256 t + 128, 256 t + 128 + D) for O_t.  The two tiles' softmax phases
+// TMEM: tile t owns columns [256 t, 256 t + 256).  Head width 128: S_t (and
+// P_t, written over it) in the first 128, O_t in the next 128.  Head width
+// 64: S_t in the first 128, P_t in the next 64, O_t in the last 64; P no
+// longer overwrites S, so S_t,j+1 can be issued as soon as the softmax group
+// has read S_t,j, while it still exponentiates.  The two tiles' softmax phases
 // alternate on the SM: while one group's exponentials occupy the SFU, the
 // other's hand-offs and the tensor core's products proceed.
 //
-// Order of the MMA issuer per key tile j (each wait bounded):
+// Order of the MMA issuer per key tile j (each wait bounded), head width 128:
 //   P_0,j V_j  ->  S_0,j+1 (after P_0,j V_j completed: it overwrites P_0,j)
 //   P_1,j V_j  ->  S_1,j+1 (likewise)
 // so a softmax group that sees S_t,j+1 complete knows P_t,j V_j is done and
-// may rescale O_t and overwrite P_t.
+// may rescale O_t and overwrite P_t.  Head width 64: S_0,j+1 and S_1,j+1 as
+// soon as the groups have read S_t,j (s_free), then the P_t,j V_j; a group
+// waits for P_t,j-1 V_j-1 itself before it rescales O_t or writes P_t.
 //
 // Lazy rescaling: a row keeps its maximum m until a tile raises it by more
 // than 8 (in log2 units), so exponentials stay below 2^8 and O is rescaled
@@ -66,8 +71,7 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kThreads = 32 * 10;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTileCols = 256;     // per tile: S (and P) [0, 128), O [128, 128 + D)
-constexpr uint32_t kOCol = 128;
+constexpr uint32_t kTileCols = 256;     // per tile, see the layout above
 
 // Error word bits (shared word with the GEMM kernels; these sites are the
 // attention kernel's).
@@ -94,13 +98,17 @@ struct AttnShape {
     static constexpr int kAtoms = D / kAtom;
     static constexpr int kKStages = D == 64 ? 4 : 3;    // K ring depth
     static constexpr int kVStages = D == 64 ? 4 : 2;    // V ring depth
+    // P in its own TMEM columns (head width 64), or written over S (128)
+    static constexpr bool kSepP = D == 64;
+    static constexpr uint32_t kPCol = kSepP ? 128u : 0u;
+    static constexpr uint32_t kOCol = kSepP ? 192u : 128u;
     static constexpr int kTileBytes = kAtoms * kAtomBytes;   // one 128-row Q, K or V tile
     static constexpr int kQOff = 0;                          // Q of both query tiles
     static constexpr int kKOff = kQOff + kTilesPerCta * kTileBytes;
     static constexpr int kVOff = kKOff + kKStages * kTileBytes;
     // barriers: q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV],
-    // s_full[2], p_full[2], pv_done[2], drain
-    static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 6 + 1;
+    // s_full[2], p_full[2], pv_done[2], s_free[2], drain
+    static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 8 + 1;
     static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
     static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
     static constexpr int kAbortOff = kTmemSlotOff + 4;
@@ -153,6 +161,34 @@ __device__ __forceinline__ float rcp(float x)
     return r;
 }
 
+// Two fp32 values in one 64-bit register, and the packed f32x2 arithmetic of
+// sm_100 (one instruction for both halves).
+__device__ __forceinline__ uint64_t f2(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void f2split(uint64_t v, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi)
 {
     __half2 h = __floats2half2_rn(lo, hi);
@@ -192,7 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *s_full = v_empty + SV;     // [2]: S_t of the current key tile is in TMEM
     uint64_t *p_full = s_full + 2;       // [2]: P_t written to TMEM (4 arrivals)
     uint64_t *pv_done = p_full + 2;      // [2]: P_t V complete
-    uint64_t *drain_bar = pv_done + 2;
+    uint64_t *s_free = pv_done + 2;      // [2]: S_t read (4 arrivals; head width 64)
+    uint64_t *drain_bar = s_free + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::kTmemSlotOff);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + S::kAbortOff);
 
@@ -210,7 +247,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int b = 0; b < S::kNumBars; ++b) {
             uint64_t *bar = &bars[b];
-            mbar_init(bar, (bar == &p_full[0] || bar == &p_full[1]) ? 4u : 1u);
+            mbar_init(bar, (bar == &p_full[0] || bar == &p_full[1] || bar == &s_free[0] ||
+                            bar == &s_free[1])
+                               ? 4u
+                               : 1u);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -331,8 +371,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < kTileK / 16; ++kk)
-                    mma_f16_ts(tmem_base + t * kTileCols + kOCol,
-                               tmem_base + t * kTileCols + static_cast<uint32_t>(kk * 8),
+                    mma_f16_ts(tmem_base + t * kTileCols + S::kOCol,
+                               tmem_base + t * kTileCols + S::kPCol + static_cast<uint32_t>(kk * 8),
                                smem_desc_sw128(va + kk * 2048, kAtomBytes, 1024), kIdescO,
                                (j > 0 || kk > 0) ? 1u : 0u);
                 mma_commit<1>(&pv_done[t]);
@@ -344,9 +384,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_commit<1>(&k_empty[0]);
             }
             for (int j = 0; ok && j < n_all; ++j) {
-                if (!wait(&v_full[j % SV], (j / SV) & 1)) break;
                 const bool next = j + 1 < n_all;
                 bool k_next = false;   // K_j+1 waited for
+                if constexpr (S::kSepP) {
+                    // S_t,j+1 as soon as group t has read S_t,j.
+                    for (int t = 0; t < 2 && ok; ++t) {
+                        if (j + 1 < nt[t]) {
+                            if (!k_next && !wait(&k_full[(j + 1) % SK], ((j + 1) / SK) & 1)) break;
+                            k_next = true;
+                            if (!wait(&s_free[t], j & 1)) break;
+                            issue_s(t, j + 1);
+                        }
+                    }
+                    if (!ok || !wait(&v_full[j % SV], (j / SV) & 1)) break;
+                    for (int t = 0; t < 2 && ok; ++t)
+                        if (j < nt[t]) {
+                            if (!wait(&p_full[t], j & 1)) break;
+                            issue_pv(t, j);
+                        }
+                    if (!ok) break;
+                    mma_commit<1>(&v_empty[j % SV]);
+                    if (next) mma_commit<1>(&k_empty[(j + 1) % SK]);
+                    continue;
+                }
+                if (!wait(&v_full[j % SV], (j / SV) & 1)) break;
                 for (int t = 0; t < 2 && ok; ++t) {
                     if (j < nt[t]) {
                         if (!wait(&p_full[t], j & 1)) break;
@@ -398,49 +459,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after_sync();
-            uint32_t s0[32], s1[32], s2[32], s3[32];
-            tmem_ld_32x32b_x32(t_lane + 0, s0);
-            tmem_ld_32x32b_x32(t_lane + 32, s1);
-            tmem_ld_32x32b_x32(t_lane + 64, s2);
-            tmem_ld_32x32b_x32(t_lane + 96, s3);
-            tmem_wait_ld_dep(s0);
-            tmem_wait_ld_dep(s1);
-            tmem_wait_ld_dep(s2);
-            tmem_wait_ld_dep(s3);
-
             // Mask keys past seq_k and, causal, past qi, on the raw scores: the
             // masked value turns into -inf once scaled (the scale's sign decides
             // which infinity).  The row maximum of the scaled scores is the scale
             // times the raw maximum (or minimum, for a negative scale), and each
             // exponent is one fused multiply-add: 2^(s * scale * log2 e - m).
+            // Two passes over the row in TMEM, 64 columns at a time (registers
+            // for a whole row would spill): the maximum, then the exponentials.
             const int64_t key0 = static_cast<int64_t>(j) * kTileK;
             const bool need_mask =
                 key0 + kTileK > p.Sk || (p.causal && key0 + kTileK - 1 > q0);
-            float x[128];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                x[c] = __uint_as_float(s0[c]);
-                x[32 + c] = __uint_as_float(s1[c]);
-                x[64 + c] = __uint_as_float(s2[c]);
-                x[96 + c] = __uint_as_float(s3[c]);
-            }
+            int64_t lim = kTileK;   // valid columns: keys [key0, Sk) and, causal, <= qi
             if (need_mask) {
-                int64_t lim = p.Sk - key0;                     // keys [key0, Sk)
-                if (p.causal && qi + 1 - key0 < lim) lim = qi + 1 - key0;   // keys <= qi
-                const float masked = pos ? -INFINITY : INFINITY;
-#pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (c >= lim) x[c] = masked;
+                lim = p.Sk - key0;
+                if (p.causal && qi + 1 - key0 < lim) lim = qi + 1 - key0;
             }
+            const float masked = pos ? -INFINITY : INFINITY;
+            auto load_half = [&](int h, float (&x)[64]) {
+                uint32_t sa[32], sb[32];
+                tmem_ld_32x32b_x32(t_lane + static_cast<uint32_t>(h * 64), sa);
+                tmem_ld_32x32b_x32(t_lane + static_cast<uint32_t>(h * 64 + 32), sb);
+                tmem_wait_ld_dep(sa);
+                tmem_wait_ld_dep(sb);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    x[c] = __uint_as_float(sa[c]);
+                    x[32 + c] = __uint_as_float(sb[c]);
+                }
+                if (need_mask) {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (h * 64 + c >= lim) x[c] = masked;
+                }
+            };
             float mx[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) mx[u] = x[u];
-            if (pos) {
+            for (int u = 0; u < 8; ++u) mx[u] = masked;
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+                float x[64];
+                load_half(h, x);
+                if (pos) {
 #pragma unroll
-                for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-            } else {
+                    for (int c = 0; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+                } else {
 #pragma unroll
-                for (int c = 8; c < 128; ++c) mx[c & 7] = fminf(mx[c & 7], x[c]);
+                    for (int c = 0; c < 64; ++c) mx[c & 7] = fminf(mx[c & 7], x[c]);
+                }
             }
             const float rext = pos ? fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                            fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])))
@@ -455,13 +520,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m = tmax;
             }
             const float mu = (m == -INFINITY) ? 0.f : m;
-            // P_t,j-1 V_j-1 is complete (S_t,j was issued after it): O_t may be
-            // rescaled and P_t overwritten.
+            // Head width 128: P_t,j-1 V_j-1 is complete (S_t,j was issued after
+            // it).  Head width 64: wait for it here.  Then O_t may be rescaled
+            // and P_t overwritten.
+            if constexpr (S::kSepP) {
+                if (j > 0) {
+                    int okv = 1;
+                    if (lane == 0)
+                        okv = mbar_wait_bounded(&pv_done[t], (j - 1) & 1, abort_flag, limit,
+                                                p.error_word, kErrAttnSoftmax)
+                                  ? 1
+                                  : 0;
+                    okv = __shfl_sync(0xffffffffu, okv, 0);
+                    if (!okv) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                }
+            }
             if (j > 0 && __any_sync(0xffffffffu, raise)) {
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t o[32];
-                    const uint32_t t_o = t_lane + kOCol + static_cast<uint32_t>(c * 32);
+                    const uint32_t t_o = t_lane + S::kOCol + static_cast<uint32_t>(c * 32);
                     tmem_ld_32x32b_x32(t_o, o);
                     tmem_wait_ld_dep(o);
 #pragma unroll
@@ -470,24 +552,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_st_32x32b_x32(t_o, o);
                 }
             }
-            // P row into TMEM columns [0, 64): two halves of 64 keys, 32 packed
-            // columns each.
-            float ps[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) ps[u] = 0.f;
-#pragma unroll
+            // P row into TMEM columns [0, 64), half h (keys 64h .. 64h + 63) into
+            // columns [32h, 32h + 32): half 0's P overwrites scores that half 0
+            // has already read, half 1's the rest of half 0.  Arguments and
+            // partial sums use the packed f32x2 FMA and add.
+            const uint64_t sl2x2 = f2(sl2, sl2);
+            const uint64_t nmu2 = f2(-mu, -mu);
+            uint64_t ps2[4] = {0, 0, 0, 0};
+#pragma unroll 1
             for (int h = 0; h < 2; ++h) {
+                float x[64];
+                load_half(h, x);
+                if (S::kSepP && h == 1) {
+                    // All of S_t,j is in registers or consumed: S_t,j+1 may land.
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s_free[t]);
+                }
                 uint32_t hp[32];
 #pragma unroll
                 for (int c = 0; c < 64; c += 2) {
-                    const float e0 = ex2(fmaf(x[h * 64 + c], sl2, -mu));
-                    const float e1 = ex2(fmaf(x[h * 64 + c + 1], sl2, -mu));
-                    ps[(c >> 1) & 7] += e0 + e1;
-                    hp[c >> 1] = pack_half2(e0, e1);
+                    const int pr = c >> 1;
+                    const uint64_t a2 = ffma2(f2(x[c], x[c + 1]), sl2x2, nmu2);
+                    float a0, a1;
+                    f2split(a2, a0, a1);
+                    const float e0 = ex2(a0);
+                    const float e1 = ex2(a1);
+                    ps2[pr & 3] = fadd2(ps2[pr & 3], f2(e0, e1));
+                    hp[pr] = pack_half2(e0, e1);
                 }
-                tmem_st_32x32b_x32(t_lane + static_cast<uint32_t>(h * 32), hp);
+                tmem_st_32x32b_x32(t_lane + S::kPCol + static_cast<uint32_t>(h * 32), hp);
             }
-            l = fmaf(l, alpha, ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
+            float q0, q1, q2, q3;
+            f2split(fadd2(ps2[0], ps2[1]), q0, q1);
+            f2split(fadd2(ps2[2], ps2[3]), q2, q3);
+            l = fmaf(l, alpha, (q0 + q1) + (q2 + q3));
             tmem_wait_st();
             tc_fence_before_sync();
             __syncwarp();
@@ -508,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t o[32];
-                    tmem_ld_32x32b_x32(t_lane + kOCol + static_cast<uint32_t>(c * 32), o);
+                    tmem_ld_32x32b_x32(t_lane + S::kOCol + static_cast<uint32_t>(c * 32), o);
                     tmem_wait_ld_dep(o);
                     if (qi < p.Sq) {
 #pragma unroll

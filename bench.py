@@ -381,6 +381,7 @@ def run_ours(args, w, rank, world):
         also.append({"workload": name, "value": world * w2.flops / (ms2 * 1e-3) / 1e12,
                      "unit": UNIT, "ms_per_step": ms2,
                      "kind": "attention" if name in wl.ATTN_WORKLOADS else "gemm",
+                     "gbs": w2.algorithmic_bytes / (ms2 * 1e-3) / 1e9,
                      "pct_of_fp16_dense_peak_nominal":
                          100.0 * w2.flops / (ms2 * 1e-3) / 1e12 / NOMINAL_FP16_DENSE_TFLOPS,
                      "l2": "flushed between launches" if not s2["big"] else "inputs larger than L2"})
@@ -497,7 +498,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="fused_8192")
     ap.add_argument("--also", nargs="*",
-                    default=["gemm_2048", "fused_2048", "fused_tanh_2048", "softmax_8192x256x4096",
+                    default=["gemm_256", "gemm_2048", "fused_2048", "ragged_fused",
+                             "fused_tanh_2048", "softmax_8192x256x4096",
                              "deepk_fused_1024x1024x8192", "attn_4x16x2048x128",
                              "attn_causal_4x16x2048x128"],
                     help="other workloads timed the same way and reported under 'also'")

@@ -226,9 +226,16 @@ tg_status_t tg_gemm_ex(const void *A, const void *B, const void *bias, void *C,
  *                                        tg_gemm_host_workspace_size(M, N, K, has_bias)
  *                                        bytes, 256-byte aligned; owned by the caller
  *
- * Enqueues on `stream`: host-to-device copies of the inputs into the
- * workspace, tg_gemm, and the device-to-host copy of C.  Returns after
- * enqueueing; synchronise `stream` before reading C_host.  Allocates nothing.
+ * Enqueues host-to-device copies of the inputs into the workspace, tg_gemm,
+ * and the device-to-host copy of C, overlapped: B and the bias go up first,
+ * then A in panels of about 2048 rows (at most 8 panels); each panel's GEMM
+ * runs on `stream` as soon as its rows are up, and its rows of C go down
+ * while later panels are uploaded and computed.  The copies run on two
+ * library streams (created once per device and caller stream) that are
+ * joined back into `stream` before the call returns, so the call is ordered
+ * on `stream` like any other work.  Returns after enqueueing; synchronise
+ * `stream` before reading C_host.  Allocates no memory (the first call on a
+ * stream creates the two streams and their events).
  */
 size_t tg_gemm_host_workspace_size(int64_t M, int64_t N, int64_t K, int has_bias);
 

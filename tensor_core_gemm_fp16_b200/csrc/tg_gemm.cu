@@ -13,6 +13,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -580,6 +581,53 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
+// The end-to-end entry point overlaps its copies with the GEMM: B (and the
+// bias) go up first, then A in row panels on an internal copy-in stream;
+// panel i's GEMM runs on the caller's stream as soon as its rows have
+// arrived, and its rows of C go down on an internal copy-out stream while the
+// next panels are uploaded and computed.  Streams and events are created once
+// per (device, caller stream) and reused; everything joins back into the
+// caller's stream before the call returns.
+constexpr int kMaxHostPanels = 8;
+constexpr int64_t kHostPanelRows = 2048;
+
+struct HostPipe {
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaEvent_t entry = nullptr, b_ready = nullptr, out_done = nullptr;
+    cudaEvent_t a_ready[kMaxHostPanels] = {}, c_ready[kMaxHostPanels] = {};
+};
+std::map<std::pair<int, cudaStream_t>, HostPipe> g_host_pipes;
+
+tg_status_t host_pipe(cudaStream_t caller, HostPipe **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lock(g_mutex);
+    auto it = g_host_pipes.find(std::make_pair(dev, caller));
+    if (it != g_host_pipes.end()) {
+        *out = &it->second;
+        return TG_OK;
+    }
+    HostPipe hp;
+    bool ok = cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.entry, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.b_ready, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.out_done, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; ok && i < kMaxHostPanels; ++i)
+        ok = cudaEventCreateWithFlags(&hp.a_ready[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&hp.c_ready[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+        cudaGetLastError();
+        return TG_ERR_CUDA;
+    }
+    *out = &(g_host_pipes[std::make_pair(dev, caller)] = hp);
+    return TG_OK;
+}
+
 }  // namespace
 
 tg_status_t tg_internal_device(int *num_sms, unsigned **error_word,
@@ -653,21 +701,64 @@ tg_status_t tg_gemm_host(const void *A_host, const void *B_host, const void *bia
     char *w = static_cast<char *>(workspace);
     const size_t a_bytes = 2 * static_cast<size_t>(M * K), b_bytes = 2 * static_cast<size_t>(K * N);
     const size_t bias_bytes = has_bias ? 2 * static_cast<size_t>(N) : 0;
-    const size_t c_bytes = 2 * static_cast<size_t>(M * N);
     char *dA = w;
     char *dB = dA + round256(a_bytes);
     char *dbias = dB + round256(b_bytes);
     char *dC = dbias + round256(bias_bytes);
-    if ((a_bytes && cudaMemcpyAsync(dA, A_host, a_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) ||
-        (b_bytes && cudaMemcpyAsync(dB, B_host, b_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) ||
-        (bias_bytes &&
-         cudaMemcpyAsync(dbias, bias_host, bias_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)) {
-        cudaGetLastError();
-        return TG_ERR_CUDA;
-    }
-    st = gemm_impl(dA, dB, has_bias ? dbias : nullptr, dC, M, N, K, epilogue, nullptr, s);
+    HostPipe *hp = nullptr;
+    st = host_pipe(s, &hp);
     if (st != TG_OK) return st;
-    if (cudaMemcpyAsync(C_host, dC, c_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+    const int panels = static_cast<int>(
+        std::min<int64_t>(kMaxHostPanels, std::max<int64_t>(1, ceil_div(M, kHostPanelRows))));
+    const int64_t rows = ceil_div(M, panels);
+    const char *Ah = static_cast<const char *>(A_host);
+    char *Ch = static_cast<char *>(C_host);
+    bool ok = cudaEventRecord(hp->entry, s) == cudaSuccess &&
+              cudaStreamWaitEvent(hp->in, hp->entry, 0) == cudaSuccess &&
+              cudaStreamWaitEvent(hp->out, hp->entry, 0) == cudaSuccess;
+    // Up: bias and B, then the panels of A.
+    ok = ok &&
+         (!bias_bytes || cudaMemcpyAsync(dbias, bias_host, bias_bytes, cudaMemcpyHostToDevice,
+                                         hp->in) == cudaSuccess) &&
+         (!b_bytes ||
+          cudaMemcpyAsync(dB, B_host, b_bytes, cudaMemcpyHostToDevice, hp->in) == cudaSuccess) &&
+         cudaEventRecord(hp->b_ready, hp->in) == cudaSuccess;
+    for (int i = 0; ok && i < panels; ++i) {
+        const int64_t r0 = i * rows, r1 = std::min<int64_t>(M, r0 + rows);
+        const size_t off = 2 * static_cast<size_t>(r0 * K), len = 2 * static_cast<size_t>((r1 - r0) * K);
+        ok = (!len || cudaMemcpyAsync(dA + off, Ah + off, len, cudaMemcpyHostToDevice, hp->in) ==
+                          cudaSuccess) &&
+             cudaEventRecord(hp->a_ready[i], hp->in) == cudaSuccess;
+    }
+    // Compute: each panel once its rows are up.
+    ok = ok && cudaStreamWaitEvent(s, hp->b_ready, 0) == cudaSuccess;
+    for (int i = 0; ok && i < panels; ++i) {
+        const int64_t r0 = i * rows, r1 = std::min<int64_t>(M, r0 + rows);
+        ok = cudaStreamWaitEvent(s, hp->a_ready[i], 0) == cudaSuccess;
+        if (!ok) break;
+        if (r1 > r0) {
+            st = gemm_impl(dA + 2 * static_cast<size_t>(r0 * K), dB, has_bias ? dbias : nullptr,
+                           dC + 2 * static_cast<size_t>(r0 * N), r1 - r0, N, K, epilogue, nullptr,
+                           s);
+            if (st != TG_OK) break;
+        }
+        ok = cudaEventRecord(hp->c_ready[i], s) == cudaSuccess;
+    }
+    // Down: each panel of C once computed.
+    for (int i = 0; ok && st == TG_OK && i < panels; ++i) {
+        const int64_t r0 = i * rows, r1 = std::min<int64_t>(M, r0 + rows);
+        const size_t off = 2 * static_cast<size_t>(r0 * N), len = 2 * static_cast<size_t>((r1 - r0) * N);
+        ok = cudaStreamWaitEvent(hp->out, hp->c_ready[i], 0) == cudaSuccess &&
+             (!len || cudaMemcpyAsync(Ch + off, dC + off, len, cudaMemcpyDeviceToHost, hp->out) ==
+                          cudaSuccess);
+    }
+    // Join both internal streams back into the caller's stream, whatever happened.
+    const bool joined = cudaEventRecord(hp->out_done, hp->out) == cudaSuccess &&
+                        cudaStreamWaitEvent(s, hp->out_done, 0) == cudaSuccess &&
+                        cudaEventRecord(hp->b_ready, hp->in) == cudaSuccess &&
+                        cudaStreamWaitEvent(s, hp->b_ready, 0) == cudaSuccess;
+    if (st != TG_OK) return st;
+    if (!ok || !joined) {
         cudaGetLastError();
         return TG_ERR_CUDA;
     }

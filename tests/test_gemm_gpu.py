@@ -253,6 +253,23 @@ def test_host_entry_matches_device_entry():
     assert torch.equal(c_host, c_dev)
 
 
+@pytest.mark.parametrize("M,N,K", [(5000, 300, 200), (4099, 129, 201), (16384, 64, 64)])
+def test_host_entry_in_row_panels(M, N, K):
+    """Problems of more than 2048 rows go through the host entry in row panels
+    (uploads, panel GEMMs and downloads overlapped on three streams); every
+    panel boundary and an unaligned K (repacked per panel) against the oracle,
+    twice in a row on the same workspace."""
+    A, B, bias = wl.make_inputs(M, N, K, seed=901 + K, dist="uniform", bias=True)
+    ref = run_oracle(A, B, bias, GELU)
+    ws = torch.empty(binding.tg_gemm_host_workspace_size(M, N, K, True), dtype=torch.uint8,
+                     device="cuda:0")
+    for _ in range(2):
+        c_host = binding.gemm_host(A.pin_memory(), B.pin_memory(), bias.pin_memory(),
+                                   epilogue=GELU, workspace=ws)
+        assert binding.tg_gemm_check_error(torch.cuda.current_stream().cuda_stream) == 0
+        assert_close(c_host, ref, f"host entry {M}x{N}x{K}")
+
+
 @pytest.mark.parametrize("config_id", [0, 3, 9])
 def test_bounded_wait_reports_timeout_and_context_survives(config_id):
     """A skipped operand load makes the consumer's bounded wait expire: the

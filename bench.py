@@ -45,19 +45,30 @@ EPI_NAMES = {0: "none", 1: "bias", 2: "bias_gelu", 3: "bias_gelu_tanh", 4: "bias
 
 # ---------------------------------------------------------------------------- helpers
 
-GEMM_SOURCES = ("tg_configs.inc", "tg_gemm.cu", "tg_kernels.cuh", "tg_ptx.cuh")
+GEMM_DEVICE_SOURCES = ("tg_kernels.cuh", "tg_ptx.cuh")
 
 
-def kernel_source_hash() -> str:
-    """Hash of the GEMM kernel's sources (device code, launch code and the
-    configuration table); ncu traffic figures are valid only for it."""
+def kernel_source_hash(kernel_config: dict) -> str:
+    """Hash of the GEMM kernel's device code and of the configuration it is
+    launched with (tile shape, stages, CTA pair, rasterisation panel, work
+    division, loader): ncu traffic figures hold only for that pair."""
     h = hashlib.sha256()
-    files = [os.path.join(ROOT, "tensor_core_gemm_fp16_b200", "csrc", f) for f in GEMM_SOURCES]
+    files = [os.path.join(ROOT, "tensor_core_gemm_fp16_b200", "csrc", f) for f in GEMM_DEVICE_SOURCES]
     for f in files:
         with open(f, "rb") as fh:
             h.update(os.path.basename(f).encode())
             h.update(fh.read())
+    h.update(json.dumps(kernel_config, sort_keys=True).encode())
     return h.hexdigest()[:16]
+
+
+def workload_kernel_hash(name: str, num_sms: int = 148) -> str:
+    """kernel_source_hash of the configuration the library picks for a named
+    GEMM workload (a host-only query: no GPU needed)."""
+    from tensor_core_gemm_fp16_b200 import binding
+    from tensor_core_gemm_fp16_b200 import workloads as wl
+    w = wl.WORKLOADS[name]
+    return kernel_source_hash(binding.tg_gemm_select_config(w.M, w.N, w.K, w.epilogue, num_sms))
 
 
 def load_peaks():
@@ -70,9 +81,10 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, kernel_config: dict):
     """DRAM bytes per launch of the GEMM kernel from the committed ncu summary
-    for this workload, or None when absent or taken on other kernel sources."""
+    for this workload, or None when absent or taken on another kernel (device
+    code or launch configuration)."""
     path = os.path.join(ROOT, "profiles", f"gemm_persistent_kernel_{workload}.md")
     try:
         text = open(path).read()
@@ -80,7 +92,7 @@ def profiled_traffic(workload: str):
         return None
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     h = re.search(r"source_hash:\s*([0-9a-f]+)", text)
-    if not m or not h or h.group(1) != kernel_source_hash():
+    if not m or not h or h.group(1) != kernel_source_hash(kernel_config):
         return None
     return float(m.group(1))
 
@@ -449,7 +461,10 @@ def finish(torch, binding, dist, w, s, args, rank, world, dev, step_ms, value, k
         achieved = w.algorithmic_bytes / (kernel_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peak_src} copy bandwidth"}
-    traffic = profiled_traffic(w.name)
+    kcfg = binding.tg_config_info(args.config) if args.config >= 0 else \
+        binding.tg_gemm_select_config(w.M, w.N, w.K, w.epilogue,
+                                      torch.cuda.get_device_properties(dev).multi_processor_count)
+    traffic = profiled_traffic(w.name, kcfg)
     roof["traffic"] = traffic
     roof["algorithmic_per_launch"] = {"flops": w.flops, "bytes": w.algorithmic_bytes}
     roof["kernel_ms"] = kernel_ms
@@ -466,9 +481,6 @@ def finish(torch, binding, dist, w, s, args, rank, world, dev, step_ms, value, k
         dist.destroy_process_group()
     if rank != 0:
         return 0
-    kcfg = binding.tg_config_info(args.config) if args.config >= 0 else \
-        binding.tg_gemm_select_config(w.M, w.N, w.K, w.epilogue,
-                                      torch.cuda.get_device_properties(dev).multi_processor_count)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,

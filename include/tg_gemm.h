@@ -228,9 +228,10 @@ tg_status_t tg_gemm_ex(const void *A, const void *B, const void *bias, void *C,
  *
  * Enqueues host-to-device copies of the inputs into the workspace, tg_gemm,
  * and the device-to-host copy of C, overlapped: B and the bias go up first,
- * then A in panels of about 2048 rows (at most 8 panels); each panel's GEMM
- * runs on `stream` as soon as its rows are up, and its rows of C go down
- * while later panels are uploaded and computed.  The copies run on two
+ * then A in panels of about 1024 rows (at most 16, the last one split in
+ * two halves so that little is left to do after the last upload); each
+ * panel's GEMM runs on `stream` as soon as its rows are up, and its rows of C
+ * go down while later panels are uploaded and computed.  The copies run on two
  * library streams (created once per device and caller stream) that are
  * joined back into `stream` before the call returns, so the call is ordered
  * on `stream` like any other work.  Returns after enqueueing; synchronise

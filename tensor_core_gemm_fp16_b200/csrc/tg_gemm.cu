@@ -588,8 +588,29 @@ size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 // next panels are uploaded and computed.  Streams and events are created once
 // per (device, caller stream) and reused; everything joins back into the
 // caller's stream before the call returns.
-constexpr int kMaxHostPanels = 8;
-constexpr int64_t kHostPanelRows = 2048;
+// Panels of about kHostPanelRows rows (at most kMaxPanelsEqual), the last one
+// halved: what is left after the final upload (that panel's GEMM and its
+// download) is then a short tail.
+constexpr int kMaxPanelsEqual = 16;
+constexpr int kMaxHostPanels = kMaxPanelsEqual + 1;
+constexpr int64_t kHostPanelRows = 1024;
+
+// Row boundaries of the panels: edge[0] = 0 < edge[1] < ... < edge[n] = M.
+int host_panels(int64_t M, int64_t (&edge)[kMaxHostPanels + 1])
+{
+    const int64_t n = std::min<int64_t>(kMaxPanelsEqual, std::max<int64_t>(1, ceil_div(M, kHostPanelRows)));
+    const int64_t rows = ceil_div(M, n);
+    int k = 0;
+    edge[0] = 0;
+    for (int64_t r = 0; r < M; r += rows) edge[++k] = std::min<int64_t>(M, r + rows);
+    const int64_t last = edge[k] - edge[k - 1];
+    if (k >= 2 && last >= 256) {
+        edge[k + 1] = edge[k];
+        edge[k] = edge[k - 1] + last / 2;
+        ++k;
+    }
+    return k;
+}
 
 struct HostPipe {
     cudaStream_t in = nullptr, out = nullptr;
@@ -708,9 +729,8 @@ tg_status_t tg_gemm_host(const void *A_host, const void *B_host, const void *bia
     HostPipe *hp = nullptr;
     st = host_pipe(s, &hp);
     if (st != TG_OK) return st;
-    const int panels = static_cast<int>(
-        std::min<int64_t>(kMaxHostPanels, std::max<int64_t>(1, ceil_div(M, kHostPanelRows))));
-    const int64_t rows = ceil_div(M, panels);
+    int64_t edge[kMaxHostPanels + 1];
+    const int panels = host_panels(M, edge);
     const char *Ah = static_cast<const char *>(A_host);
     char *Ch = static_cast<char *>(C_host);
     bool ok = cudaEventRecord(hp->entry, s) == cudaSuccess &&
@@ -724,7 +744,7 @@ tg_status_t tg_gemm_host(const void *A_host, const void *B_host, const void *bia
           cudaMemcpyAsync(dB, B_host, b_bytes, cudaMemcpyHostToDevice, hp->in) == cudaSuccess) &&
          cudaEventRecord(hp->b_ready, hp->in) == cudaSuccess;
     for (int i = 0; ok && i < panels; ++i) {
-        const int64_t r0 = i * rows, r1 = std::min<int64_t>(M, r0 + rows);
+        const int64_t r0 = edge[i], r1 = edge[i + 1];
         const size_t off = 2 * static_cast<size_t>(r0 * K), len = 2 * static_cast<size_t>((r1 - r0) * K);
         ok = (!len || cudaMemcpyAsync(dA + off, Ah + off, len, cudaMemcpyHostToDevice, hp->in) ==
                           cudaSuccess) &&
@@ -733,7 +753,7 @@ tg_status_t tg_gemm_host(const void *A_host, const void *B_host, const void *bia
     // Compute: each panel once its rows are up.
     ok = ok && cudaStreamWaitEvent(s, hp->b_ready, 0) == cudaSuccess;
     for (int i = 0; ok && i < panels; ++i) {
-        const int64_t r0 = i * rows, r1 = std::min<int64_t>(M, r0 + rows);
+        const int64_t r0 = edge[i], r1 = edge[i + 1];
         ok = cudaStreamWaitEvent(s, hp->a_ready[i], 0) == cudaSuccess;
         if (!ok) break;
         if (r1 > r0) {
@@ -746,7 +766,7 @@ tg_status_t tg_gemm_host(const void *A_host, const void *B_host, const void *bia
     }
     // Down: each panel of C once computed.
     for (int i = 0; ok && st == TG_OK && i < panels; ++i) {
-        const int64_t r0 = i * rows, r1 = std::min<int64_t>(M, r0 + rows);
+        const int64_t r0 = edge[i], r1 = edge[i + 1];
         const size_t off = 2 * static_cast<size_t>(r0 * N), len = 2 * static_cast<size_t>((r1 - r0) * N);
         ok = cudaStreamWaitEvent(hp->out, hp->c_ready[i], 0) == cudaSuccess &&
              (!len || cudaMemcpyAsync(Ch + off, dC + off, len, cudaMemcpyDeviceToHost, hp->out) ==

@@ -255,7 +255,7 @@ def test_host_entry_matches_device_entry():
 
 @pytest.mark.parametrize("M,N,K", [(5000, 300, 200), (4099, 129, 201), (16384, 64, 64)])
 def test_host_entry_in_row_panels(M, N, K):
-    """Problems of more than 2048 rows go through the host entry in row panels
+    """Problems of more than 1024 rows go through the host entry in row panels
     (uploads, panel GEMMs and downloads overlapped on three streams); every
     panel boundary and an unaligned K (repacked per panel) against the oracle,
     twice in a row on the same workspace."""

@@ -43,9 +43,18 @@ extern "C" {
  *
  * All four are device pointers owned by the caller, 16-byte aligned (else
  * TG_ERR_MISALIGNED); O must not overlap Q, K or V (TG_ERR_INVALID_ARG).
- * The call is asynchronous and keeps no pointer after it returns; it
- * allocates nothing.  batch * heads * seq_q == 0 is a no-op; seq_k == 0
- * writes O = 0.  Bad sizes, head_dim, causal or a non-finite scale return
+ * The call is asynchronous and keeps no pointer after it returns.
+ * batch * heads * seq_q == 0 is a no-op; seq_k == 0 writes O = 0.
+ *
+ * Work division: one CTA per (batch x head, 256 queries).  Non-causal calls
+ * whose last wave of CTAs would occupy at most half of the SMs split each
+ * of that wave's units into two CTAs, one per half of the keys; the half
+ * that finishes second merges the two partial results (the FlashAttention
+ * rescaling by the row maxima).  Such a call uses a library workspace per
+ * (device, stream) of about 266 KB per split unit, allocated in stream
+ * order on first need (cudaMallocAsync; TG_ERR_OOM if that fails) and kept
+ * for the process; calls that share a stream are ordered by it, calls on
+ * different streams use different workspaces.  Bad sizes, head_dim, causal or a non-finite scale return
  * TG_ERR_INVALID_ARG before anything is launched; a device other than
  * compute capability 10.0 returns TG_ERR_UNSUPPORTED_DEVICE (there is no CPU
  * path).  Every device-side wait is bounded (2 s by default); an expiry is
@@ -55,6 +64,13 @@ tg_status_t tg_attention_fwd(const void *Q, const void *K, const void *V, void *
                              int64_t heads, int64_t seq_q, int64_t seq_k, int64_t head_dim,
                              int causal, float scale, void *stream);
 
+/* Key-half split of tg_attention_options_t.kv_split. */
+enum {
+    TG_ATTN_SPLIT_AUTO = 0,   /* split the units of a sparse last wave (non-causal) */
+    TG_ATTN_SPLIT_NEVER = 1,  /* one CTA per unit */
+    TG_ATTN_SPLIT_ALL = 2     /* split every unit (non-causal, at least 2 key tiles) */
+};
+
 /*
  * Options of tg_attention_fwd_ex (NULL: the defaults of tg_attention_fwd).
  *   wait_limit_ns  0: default (2 s); else the limit of every device-side wait
@@ -63,10 +79,13 @@ tg_status_t tg_attention_fwd(const void *Q, const void *K, const void *V, void *
  *                  bounded wait expires (testing the timeout path only); the
  *                  kernel exits cleanly and tg_gemm_check_error returns
  *                  TG_ERR_TIMEOUT.
+ *   kv_split       TG_ATTN_SPLIT_*; other values: TG_ERR_INVALID_ARG.  Causal
+ *                  calls and calls with seq_k <= 128 never split.
  */
 typedef struct {
     uint64_t wait_limit_ns;
     int inject;
+    int kv_split;
 } tg_attention_options_t;
 
 tg_status_t tg_attention_fwd_ex(const void *Q, const void *K, const void *V, void *O,

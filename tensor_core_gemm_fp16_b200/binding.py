@@ -36,6 +36,7 @@ TG_ERR_CUDA = 7
 TG_ERR_SCRATCH_LIMIT = 8
 
 TG_INJECT_SKIP_FIRST_LOAD = 1
+TG_ATTN_SPLIT_AUTO, TG_ATTN_SPLIT_NEVER, TG_ATTN_SPLIT_ALL = 0, 1, 2
 TG_INJECT_SKIP_STREAMK_FLAGS = 2
 TG_SPLIT_AUTO = 0
 TG_SPLIT_TILES = 1
@@ -62,7 +63,8 @@ class tg_config_t(ctypes.Structure):
 
 
 class tg_attention_options_t(ctypes.Structure):
-    _fields_ = [("wait_limit_ns", ctypes.c_uint64), ("inject", ctypes.c_int)]
+    _fields_ = [("wait_limit_ns", ctypes.c_uint64), ("inject", ctypes.c_int),
+                ("kv_split", ctypes.c_int)]
 
 
 class tg_options_t(ctypes.Structure):
@@ -261,18 +263,19 @@ def tg_attention_fwd(Q, K, V, O, batch, heads, seq_q, seq_k, head_dim, causal, s
 
 
 def tg_attention_fwd_ex(Q, K, V, O, batch, heads, seq_q, seq_k, head_dim, causal, scale,
-                        wait_limit_ns=0, inject=0, stream=None) -> int:
-    opts = tg_attention_options_t(wait_limit_ns, inject)
+                        wait_limit_ns=0, inject=0, stream=None, kv_split=0) -> int:
+    opts = tg_attention_options_t(wait_limit_ns, inject, kv_split)
     return load().tg_attention_fwd_ex(Q, K, V, O, batch, heads, seq_q, seq_k, head_dim,
                                       int(causal), float(scale), ctypes.byref(opts), stream)
 
 
-def attention(q, k, v, causal=False, scale=0.0, out=None, *, wait_limit_ns=0, inject=0):
+def attention(q, k, v, causal=False, scale=0.0, out=None, *, wait_limit_ns=0, inject=0,
+              kv_split=0):
     """O = softmax(scale q k^T) v on the GPU through tg_attention_fwd_ex.
 
     q: (B, H, Sq, D), k and v: (B, H, Sk, D), fp16 contiguous CUDA tensors,
-    D in {64, 128}; scale 0 means 1/sqrt(D).  Returns ``out`` (allocated if
-    None).
+    D in {64, 128}; scale 0 means 1/sqrt(D).  kv_split: TG_ATTN_SPLIT_*.
+    Returns ``out`` (allocated if None).
     """
     import torch
     for name, t in (("q", q), ("k", k), ("v", v), ("out", out)):
@@ -297,7 +300,8 @@ def attention(q, k, v, causal=False, scale=0.0, out=None, *, wait_limit_ns=0, in
     with torch.cuda.device(q.device):
         st = tg_attention_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H,
                                  Sq, Sk, D, causal, scale, wait_limit_ns=wait_limit_ns,
-                                 inject=inject, stream=_stream_handle(torch, q.device))
+                                 inject=inject, stream=_stream_handle(torch, q.device),
+                                 kv_split=kv_split)
     if st != TG_OK:
         raise TgError(st, "tg_attention_fwd")
     return out

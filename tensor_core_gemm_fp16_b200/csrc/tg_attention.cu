@@ -53,6 +53,9 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "tg_attention.h"
 #include "tg_internal.h"
@@ -90,6 +93,15 @@ struct AttnParams {
     int inject;
     uint64_t wait_limit_ns;
     unsigned *error_word;
+    // Work division.  A unit is one (batch x head, pair of query tiles); units
+    // [0, num_full) take one CTA each, the next split_units take two CTAs,
+    // one per half of the key tiles, and are combined by whichever half
+    // finishes second (non-causal only).
+    int num_full;
+    int split_units;
+    float *part;         // [split unit][key half][tile][D + 2][128]: O (unnormalised), m, l
+    unsigned *flags;     // [split unit][tile][lane quarter]: epoch of the first half to finish
+    unsigned epoch;
 };
 
 template <int D>
@@ -235,12 +247,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // Unit of this CTA, and its key half (-1: all key tiles).
+    int unit = static_cast<int>(blockIdx.x), half = -1;
+    if (unit >= p.num_full) {
+        const int i = unit - p.num_full;
+        unit = p.num_full + (i >> 1);
+        half = i & 1;
+    }
     // Heavier query pairs first (causal: later queries see more keys).
-    const int qp = p.num_qp - 1 - static_cast<int>(blockIdx.x / p.num_bh);
-    const int bh = static_cast<int>(blockIdx.x % p.num_bh);
+    const int qp = p.num_qp - 1 - unit / p.num_bh;
+    const int bh = unit % p.num_bh;
     const int64_t qbase = static_cast<int64_t>(qp) * kTilesPerCta * kTileQ;
-    const int n0 = tile_key_tiles(p, qbase);
-    const int n1 = tile_key_tiles(p, qbase + kTileQ);
+    const int n0_all = tile_key_tiles(p, qbase);
+    const int n1_all = tile_key_tiles(p, qbase + kTileQ);
+    const int n_units = n0_all > n1_all ? n0_all : n1_all;
+    // Key tiles [kv_lo, kv_lo + n_t) for tile t; j below counts from kv_lo.
+    // A split unit is non-causal, so each tile has all key tiles or none.
+    const int kv_lo = half == 1 ? n_units / 2 : 0;
+    const int kv_n = half < 0 ? n_units : (half == 0 ? n_units / 2 : n_units - n_units / 2);
+    const int n0 = half < 0 ? n0_all : (n0_all > 0 ? kv_n : 0);
+    const int n1 = half < 0 ? n1_all : (n1_all > 0 ? kv_n : 0);
     const int n_all = n0 > n1 ? n0 : n1;
     const uint64_t limit = p.wait_limit_ns;
 
@@ -293,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!(p.inject == 1 && blockIdx.x == 0 && jk == 0))
                         for (int a = 0; a < S::kAtoms; ++a)
                             tma_load_3d(kdst + a * kAtomBytes, &tmK, &k_full[st], a * kAtom,
-                                        jk * kTileK, bh);
+                                        (kv_lo + jk) * kTileK, bh);
                     k_filled[st] = jk / SK + 1;
                     ++jk;
                     progress = true;
@@ -305,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(&v_full[st], S::kTileBytes);
                     for (int a = 0; a < S::kAtoms; ++a)
                         tma_load_3d(vdst + a * kAtomBytes, &tmV, &v_full[st], a * kAtom,
-                                    jv * kTileK, bh);
+                                    (kv_lo + jv) * kTileK, bh);
                     v_filled[st] = jv / SV + 1;
                     ++jv;
                     progress = true;
@@ -466,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // exponent is one fused multiply-add: 2^(s * scale * log2 e - m).
             // Two passes over the row in TMEM, 64 columns at a time (registers
             // for a whole row would spill): the maximum, then the exponentials.
-            const int64_t key0 = static_cast<int64_t>(j) * kTileK;
+            const int64_t key0 = static_cast<int64_t>(kv_lo + j) * kTileK;
             const bool need_mask =
                 key0 + kTileK > p.Sk || (p.causal && key0 + kTileK - 1 > q0);
             int64_t lim = kTileK;   // valid columns: keys [key0, Sk) and, causal, <= qi
@@ -602,26 +628,79 @@ __global__ void __launch_bounds__(kThreads, 1)
             okw = __shfl_sync(0xffffffffu, okw, 0);
             if (okw) {
                 tc_fence_after_sync();
-                const float inv_l = l > 0.f ? rcp(l) : 0.f;
-                __half *orow = p.O + (static_cast<int64_t>(bh) * p.Sq + qi) * D;
+                // Whole unit: O / l.  Split unit: publish this half's O, m and l
+                // (column-major over the tile's rows, so a warp's accesses are
+                // coalesced); the half that finishes second merges both:
+                //   O = (O_a 2^(m_a - m) + O_b 2^(m_b - m)) / (l_a 2^(m_a - m) + l_b 2^(m_b - m)),
+                //   m = max(m_a, m_b).
+                float wa = 1.f, wb = 0.f;   // weights of this half's O and of the other's
+                const float *other = nullptr;
+                bool store = true;
+                if (half >= 0) {
+                    const int us = unit - p.num_full;
+                    float *mine =
+                        p.part + static_cast<size_t>((us * 2 + half) * 2 + t) * (D + 2) * kTileQ;
+                    other =
+                        p.part + static_cast<size_t>((us * 2 + (1 - half)) * 2 + t) * (D + 2) * kTileQ;
 #pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t o[32];
-                    tmem_ld_32x32b_x32(t_lane + S::kOCol + static_cast<uint32_t>(c * 32), o);
-                    tmem_wait_ld_dep(o);
-                    if (qi < p.Sq) {
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld_32x32b_x32(t_lane + S::kOCol + static_cast<uint32_t>(c * 32), o);
+                        tmem_wait_ld_dep(o);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint4 u;
-                            u.x = pack_half2(__uint_as_float(o[q * 8 + 0]) * inv_l,
-                                             __uint_as_float(o[q * 8 + 1]) * inv_l);
-                            u.y = pack_half2(__uint_as_float(o[q * 8 + 2]) * inv_l,
-                                             __uint_as_float(o[q * 8 + 3]) * inv_l);
-                            u.z = pack_half2(__uint_as_float(o[q * 8 + 4]) * inv_l,
-                                             __uint_as_float(o[q * 8 + 5]) * inv_l);
-                            u.w = pack_half2(__uint_as_float(o[q * 8 + 6]) * inv_l,
-                                             __uint_as_float(o[q * 8 + 7]) * inv_l);
-                            *reinterpret_cast<uint4 *>(orow + c * 32 + q * 8) = u;
+                        for (int e = 0; e < 32; ++e)
+                            __stcg(mine + (c * 32 + e) * kTileQ + row, __uint_as_float(o[e]));
+                    }
+                    __stcg(mine + D * kTileQ + row, m);
+                    __stcg(mine + (D + 1) * kTileQ + row, l);
+                    __threadfence();
+                    __syncwarp();
+                    unsigned prev = 0;
+                    if (lane == 0) prev = atomicExch(&p.flags[(us * 2 + t) * 4 + quarter], p.epoch);
+                    prev = __shfl_sync(0xffffffffu, prev, 0);
+                    store = prev == p.epoch;
+                    if (store) {
+                        __threadfence();
+                        const float mo = __ldcg(other + D * kTileQ + row);
+                        const float lo = __ldcg(other + (D + 1) * kTileQ + row);
+                        const float mm = fmaxf(m, mo);
+                        wa = m == -INFINITY ? 0.f : ex2(m - mm);
+                        wb = mo == -INFINITY ? 0.f : ex2(mo - mm);
+                        // Half 0's terms first, whichever half merges: the
+                        // result does not depend on which finished second.
+                        l = half == 0 ? fmaf(lo, wb, l * wa) : fmaf(l, wa, lo * wb);
+                    }
+                }
+                if (store) {
+                    const float inv_l = l > 0.f ? rcp(l) : 0.f;
+                    const float sa = wa * inv_l, sb = wb * inv_l;
+                    __half *orow = p.O + (static_cast<int64_t>(bh) * p.Sq + qi) * D;
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld_32x32b_x32(t_lane + S::kOCol + static_cast<uint32_t>(c * 32), o);
+                        tmem_wait_ld_dep(o);
+                        if (qi < p.Sq) {
+                            float v[32];
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * sa;
+                            if (other) {
+#pragma unroll
+                                for (int e = 0; e < 32; ++e) {
+                                    const float x = __ldcg(other + (c * 32 + e) * kTileQ + row);
+                                    v[e] = half == 0 ? fmaf(x, sb, v[e])
+                                                     : fmaf(__uint_as_float(o[e]), sa, x * sb);
+                                }
+                            }
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                uint4 u;
+                                u.x = pack_half2(v[q * 8 + 0], v[q * 8 + 1]);
+                                u.y = pack_half2(v[q * 8 + 2], v[q * 8 + 3]);
+                                u.z = pack_half2(v[q * 8 + 4], v[q * 8 + 5]);
+                                u.w = pack_half2(v[q * 8 + 6], v[q * 8 + 7]);
+                                *reinterpret_cast<uint4 *>(orow + c * 32 + q * 8) = u;
+                            }
                         }
                     }
                 }
@@ -657,6 +736,70 @@ bool encode_3d(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap *tm, const 
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Workspace of the key-half split, per (device, stream): the halves' partial
+// results and one flag word per (split unit, tile, lane quarter).  It grows
+// in stream order (cudaFreeAsync / cudaMallocAsync on the caller's stream);
+// each launch takes a fresh epoch, so flags need no reset between launches.
+struct SplitWorkspace {
+    void *mem = nullptr;
+    int units = 0;
+    unsigned epoch = 0;
+};
+std::mutex g_ws_mutex;
+std::map<std::pair<int, cudaStream_t>, SplitWorkspace> g_split_ws;
+
+constexpr size_t split_part_floats(int units) { return static_cast<size_t>(units) * 2 * 2 * (128 + 2) * tga::kTileQ; }
+
+tg_status_t split_workspace(int units, cudaStream_t stream, float **part, unsigned **flags,
+                            unsigned *epoch)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lock(g_ws_mutex);
+    SplitWorkspace &w = g_split_ws[std::make_pair(dev, stream)];
+    if (units > w.units) {
+        const size_t part_bytes = split_part_floats(units) * sizeof(float);
+        const size_t flag_bytes = static_cast<size_t>(units) * 2 * 4 * sizeof(unsigned);
+        if (w.mem && cudaFreeAsync(w.mem, stream) != cudaSuccess) {
+            cudaGetLastError();
+            return TG_ERR_CUDA;
+        }
+        w.mem = nullptr;
+        w.units = 0;
+        if (cudaMallocAsync(&w.mem, part_bytes + flag_bytes, stream) != cudaSuccess) {
+            cudaGetLastError();
+            w.mem = nullptr;
+            return TG_ERR_OOM;
+        }
+        if (cudaMemsetAsync(static_cast<char *>(w.mem) + part_bytes, 0, flag_bytes, stream) !=
+            cudaSuccess) {
+            cudaGetLastError();
+            return TG_ERR_CUDA;
+        }
+        w.units = units;
+    }
+    if (++w.epoch == 0) w.epoch = 1;
+    *part = static_cast<float *>(w.mem);
+    *flags = reinterpret_cast<unsigned *>(static_cast<char *>(w.mem) +
+                                          split_part_floats(w.units) * sizeof(float));
+    *epoch = w.epoch;
+    return TG_OK;
+}
+
+// Units split into key halves.  Auto: when the last wave of units would fill
+// at most half of the SMs, its units are split, so that it takes half as
+// long; never for causal attention or a single key tile.
+int split_units(int64_t units, int num_sms, int64_t key_tiles, int causal, int mode)
+{
+    if (causal || key_tiles < 2 || mode == TG_ATTN_SPLIT_NEVER) return 0;
+    if (mode == TG_ATTN_SPLIT_ALL) return static_cast<int>(units);
+    const int64_t rem = units % num_sms;
+    return rem > 0 && 2 * rem <= num_sms ? static_cast<int>(rem) : 0;
+}
 
 bool overlaps(const void *a, size_t na, const void *b, size_t nb)
 {
@@ -699,6 +842,8 @@ tg_status_t attention_impl(const void *Q, const void *K, const void *V, void *O,
         return TG_ERR_INVALID_ARG;
     if (opts && opts->inject != 0 && opts->inject != TG_INJECT_SKIP_FIRST_LOAD)
         return TG_ERR_INVALID_ARG;
+    if (opts && (opts->kv_split < TG_ATTN_SPLIT_AUTO || opts->kv_split > TG_ATTN_SPLIT_ALL))
+        return TG_ERR_INVALID_ARG;
     const int64_t bh = B * H;
     if (B > 0 && H > (int64_t(1) << 31) / B) return TG_ERR_INVALID_ARG;
     if (bh == 0 || Sq == 0) return TG_OK;
@@ -739,7 +884,21 @@ tg_status_t attention_impl(const void *Q, const void *K, const void *V, void *O,
     p.inject = opts ? opts->inject : 0;
     p.wait_limit_ns = (opts && opts->wait_limit_ns) ? opts->wait_limit_ns : kDefaultWaitLimitNs;
     p.error_word = error_word;
-    const int grid = static_cast<int>(bh * num_qp);
+    const int64_t units = bh * num_qp;
+    const int64_t key_tiles = (Sk + tga::kTileK - 1) / tga::kTileK;
+    const int split = split_units(units, num_sms, key_tiles, causal,
+                                  opts ? opts->kv_split : TG_ATTN_SPLIT_AUTO);
+    if (units + split > 0x7fffffff) return TG_ERR_INVALID_ARG;
+    p.num_full = static_cast<int>(units - split);
+    p.split_units = split;
+    p.part = nullptr;
+    p.flags = nullptr;
+    p.epoch = 0;
+    if (split > 0) {
+        st = split_workspace(split, stream, &p.part, &p.flags, &p.epoch);
+        if (st != TG_OK) return st;
+    }
+    const int grid = static_cast<int>(units + split);
     return D == 64 ? launch_attn<64>(tq, tk, tv, p, grid, stream)
                    : launch_attn<128>(tq, tk, tv, p, grid, stream);
 }

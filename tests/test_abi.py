@@ -35,6 +35,8 @@ def test_attention_host_validation_without_a_device():
     assert f(q + 8, k, v, o, 1, 1, 128, 128, 64, 0, 0.0) == binding.TG_ERR_MISALIGNED
     assert f(q, k, v, o, 0, 4, 128, 128, 64, 0, 0.0) == binding.TG_OK   # empty: no-op
     assert binding.tg_attention_fwd_ex(q, k, v, o, 1, 1, 8, 8, 64, 0, 0.0, inject=9) == bad
+    assert binding.tg_attention_fwd_ex(q, k, v, o, 1, 1, 8, 8, 64, 0, 0.0, kv_split=3) == bad
+    assert binding.tg_attention_fwd_ex(q, k, v, o, 1, 1, 8, 8, 64, 0, 0.0, kv_split=-1) == bad
 
 
 def test_status_strings():

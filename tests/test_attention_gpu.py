@@ -166,3 +166,52 @@ def test_workload_sampled_rows(name):
     ref = oracle_attn(Q, K, V, w.causal, rows=rows)
     assert_close(O.reshape(-1, w.D)[rows], ref, f"{name} sampled rows")
     assert torch.isfinite(O.float()).all()
+
+
+# ---------------------------------------------------------------- key-half split
+
+SPLIT_SHAPES = [  # B, H, Sq, Sk, D (non-causal; at least two key tiles)
+    (2, 3, 200, 333, 64),      # three key tiles: halves of one and two
+    (1, 2, 384, 256, 128),     # two key tiles
+    (1, 1, 257, 129, 128),     # the second half holds one valid key
+    (3, 1, 64, 700, 64),       # six key tiles, one partial query tile
+    (1, 4, 1000, 1000, 128),
+]
+
+
+@pytest.mark.parametrize("shape", SPLIT_SHAPES, ids=["x".join(map(str, s)) for s in SPLIT_SHAPES])
+def test_kv_split_modes_match_the_oracle(shape):
+    """Every unit split in two key halves (merged by the half that finishes
+    second), no split, and the automatic choice: each against the oracle."""
+    B, H, Sq, Sk, D = shape
+    Q, K, V = wl.attention_inputs(B, H, Sq, Sk, D, seed=300 + Sq + Sk + D)
+    ref = oracle_attn(Q, K, V, False).reshape(-1, D)
+    for mode in (binding.TG_ATTN_SPLIT_ALL, binding.TG_ATTN_SPLIT_NEVER,
+                 binding.TG_ATTN_SPLIT_AUTO):
+        O = run_attn(Q, K, V, False, kv_split=mode)
+        assert_close(O.reshape(-1, D), ref, f"{shape} kv_split={mode}")
+
+
+def test_kv_split_not_applied_where_it_cannot_be():
+    """Causal calls and a single key tile never split: forcing the split gives
+    the unsplit result bit for bit."""
+    for (B, H, Sq, Sk, D), causal in (((1, 2, 384, 384, 64), True),
+                                      ((2, 2, 300, 128, 128), False)):
+        Q, K, V = wl.attention_inputs(B, H, Sq, Sk, D, seed=400 + Sq)
+        a = run_attn(Q, K, V, causal, kv_split=binding.TG_ATTN_SPLIT_ALL)
+        b = run_attn(Q, K, V, causal, kv_split=binding.TG_ATTN_SPLIT_NEVER)
+        assert torch.equal(a, b)
+
+
+def test_kv_split_workspace_growth_and_reuse():
+    """Split calls of growing and shrinking unit counts on one stream (the
+    workspace grows in stream order, each launch takes a fresh epoch), then
+    the first call again: the same result bit for bit."""
+    small = wl.attention_inputs(1, 1, 256, 512, 64, seed=501)
+    big = wl.attention_inputs(2, 8, 1024, 512, 64, seed=502)
+    first = run_attn(*small, False, kv_split=binding.TG_ATTN_SPLIT_ALL)
+    for Q, K, V in (big, small, big):
+        O = run_attn(Q, K, V, False, kv_split=binding.TG_ATTN_SPLIT_ALL)
+        assert_close(O.reshape(-1, 64), oracle_attn(Q, K, V, False).reshape(-1, 64), "regrow")
+    again = run_attn(*small, False, kv_split=binding.TG_ATTN_SPLIT_ALL)
+    assert torch.equal(first, again)

@@ -205,6 +205,29 @@ def oracle_sample(w, A, B, bias, target_s: float):
     return 2.0 * len(sel) * w.N * w.K / dt / 1e12, dt, len(sel), oracle.num_threads()
 
 
+def oracle_single_core(target_s: float = 1.0):
+    """The oracle on one core for gemm_256 (whole) and gemm_2048 (a row sample
+    of about target_s): GFLOP/s of each, as a per-core reference."""
+    import oracle
+    from tensor_core_gemm_fp16_b200 import workloads as wl
+    prev = oracle.set_num_threads(1)
+    try:
+        out = {}
+        for name in ("gemm_256", "gemm_2048"):
+            w = wl.WORKLOADS[name]
+            A, B, bias = wl.workload_inputs(w)
+            a, b, bb = wl.to_bits(A), wl.to_bits(B), wl.to_bits(bias)
+            sel = evenly_spaced(w.M, oracle_rows_for(w, a, b, bb, target_s))
+            t0 = time.perf_counter()
+            oracle.gemm(a, b, bb, w.epilogue, rows=sel)
+            dt = time.perf_counter() - t0
+            out[name] = {"gflops": 2.0 * len(sel) * w.N * w.K / dt / 1e9,
+                         "rows": f"{len(sel)} of {w.M}", "seconds": dt}
+        return out
+    finally:
+        oracle.set_num_threads(prev)
+
+
 # ---------------------------------------------------------------------------- arms
 
 def run_reference(args, w, rank, world):
@@ -475,7 +498,8 @@ def finish(torch, binding, dist, w, s, args, rank, world, dev, step_ms, value, k
                                                   target_s=args.cpu_seconds)
         cpu = {"value": tflops, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{rows} evenly spaced full rows of the {w.M}x{w.N}x{w.K} output "
-                         f"({rows * w.N} outputs) in {secs:.1f} s, fp64, one call incl. decode"}
+                         f"({rows * w.N} outputs) in {secs:.1f} s, fp64, one call incl. decode",
+               "single_core": oracle_single_core()}
 
     if world > 1:
         dist.destroy_process_group()

@@ -75,6 +75,8 @@ def _load():
         lib.tgo_gelu_n.argtypes = [f64p, i64, f64p]
         lib.tgo_gelu_tanh_n.argtypes = [f64p, i64, f64p]
         lib.tgo_num_threads.restype = ctypes.c_int
+        lib.tgo_set_num_threads.argtypes = [ctypes.c_int]
+        lib.tgo_set_num_threads.restype = ctypes.c_int
         lib.tgo_attention.argtypes = [u16p, u16p, u16p, i64, i64, i64, i64, i64, ctypes.c_int,
                                       ctypes.c_double, i64p, i64, f64p]
         lib.tgo_attention.restype = ctypes.c_int
@@ -218,3 +220,9 @@ def gelu_tanh(x) -> np.ndarray:
 def num_threads() -> int:
     """OpenMP threads the oracle uses (OMP_NUM_THREADS or all cores)."""
     return int(_load().tgo_num_threads())
+
+
+def set_num_threads(n: int) -> int:
+    """Threads for the oracle's later calls from this thread (timing only: the
+    results do not depend on it); returns the previous count."""
+    return int(_load().tgo_set_num_threads(int(n)))

@@ -304,6 +304,21 @@ int tgo_num_threads(void)
 #endif
 }
 
+/* Threads for the calling thread's later parallel regions (n >= 1; other
+ * values change nothing).  Returns the previous count.  Timing only: the
+ * results do not depend on it. */
+int tgo_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    const int prev = omp_get_max_threads();
+    if (n >= 1) omp_set_num_threads(n);
+    return prev;
+#else
+    (void)n;
+    return 1;
+#endif
+}
+
 /* Array versions of the element codecs (for exhaustive tests). */
 void tgo_half_to_double_n(const uint16_t *h, int64_t n, double *out)
 {

@@ -453,3 +453,19 @@ def test_softmax_k0_is_softmax_of_bias():
     e = np.exp(_dec(bias) - 2.0)
     assert np.allclose(_oracle_gemm(A, B, bias, oracle.EPI_BIAS_SOFTMAX),
                        np.tile(e / e.sum(), (3, 1)), rtol=1e-15)
+
+
+def test_thread_count_changes_no_result():
+    """The oracle's threads only split the output rows: one thread gives the
+    same bits as all of them (the bench's single-core timing relies on it)."""
+    A, B, bias = wl.make_inputs(37, 29, 301, seed=77, bias=True)
+    a, b, bb = wl.to_bits(A), wl.to_bits(B), wl.to_bits(bias)
+    many = oracle.gemm(a, b, bb, oracle.EPI_BIAS_GELU)
+    prev = oracle.set_num_threads(1)
+    try:
+        assert oracle.num_threads() == 1
+        one = oracle.gemm(a, b, bb, oracle.EPI_BIAS_GELU)
+    finally:
+        oracle.set_num_threads(prev)
+    assert oracle.num_threads() == prev
+    assert np.array_equal(many, one)

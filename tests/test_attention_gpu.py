@@ -215,3 +215,27 @@ def test_kv_split_workspace_growth_and_reuse():
         assert_close(O.reshape(-1, 64), oracle_attn(Q, K, V, False).reshape(-1, 64), "regrow")
     again = run_attn(*small, False, kv_split=binding.TG_ATTN_SPLIT_ALL)
     assert torch.equal(first, again)
+
+
+def test_kv_split_on_two_streams_at_once():
+    """Split launches on two streams overlap in time; each stream has its own
+    workspace and flags, so both results match the oracle."""
+    dev = torch.device("cuda:0")
+    cases = [wl.attention_inputs(2, 4, 512, 768, 64, seed=601),
+             wl.attention_inputs(2, 4, 512, 768, 64, seed=602)]
+    streams = [torch.cuda.Stream(dev), torch.cuda.Stream(dev)]
+    outs = []
+    torch.cuda.synchronize()
+    dev_in = [tuple(x.to(dev) for x in c) for c in cases]
+    torch.cuda.synchronize()
+    for _ in range(3):
+        outs = []
+        for (q, k, v), s in zip(dev_in, streams):
+            with torch.cuda.stream(s):
+                outs.append(binding.attention(q, k, v, False, kv_split=binding.TG_ATTN_SPLIT_ALL))
+    torch.cuda.synchronize()
+    for s in streams:
+        assert binding.tg_gemm_check_error(s.cuda_stream) == binding.TG_OK
+    for (Q, K, V), o in zip(cases, outs):
+        ref = oracle_attn(Q, K, V, False).reshape(-1, 64)
+        assert_close(o.cpu().reshape(-1, 64), ref, "two streams")

@@ -749,7 +749,12 @@ struct SplitWorkspace {
 std::mutex g_ws_mutex;
 std::map<std::pair<int, cudaStream_t>, SplitWorkspace> g_split_ws;
 
-constexpr size_t split_part_floats(int units) { return static_cast<size_t>(units) * 2 * 2 * (128 + 2) * tga::kTileQ; }
+// Floats of partial results per split unit: 2 key halves x 2 tiles x (O of
+// up to 128 columns, m, l) x 128 rows.
+constexpr size_t split_part_floats(int units)
+{
+    return static_cast<size_t>(units) * 2 * 2 * (128 + 2) * tga::kTileQ;
+}
 
 tg_status_t split_workspace(int units, cudaStream_t stream, float **part, unsigned **flags,
                             unsigned *epoch)

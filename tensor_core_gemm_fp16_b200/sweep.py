@@ -13,8 +13,11 @@ schedule depends on the architecture and the shape.  This tool does the
 same over this library's compiled configurations on B200: every candidate
 is checked against torch's fp32 matmul of the same fp16 inputs (relative
 Frobenius error < 2e-2, as in the tutorial's sweep) before it is timed, and
-it is timed with CUDA events (median of `reps` launches; L2 flushed before
-each launch when the operands fit in L2).
+it is timed with CUDA events (L2 flushed before each launch when the
+operands fit in L2).  The events on B200 tick in steps of about 2 us, so a
+single launch's time is quantised; the mean over many launches, whose start
+falls at random within a tick, resolves finer than a tick, and a median would
+not.
 """
 from __future__ import annotations
 
@@ -73,7 +76,7 @@ def time_config(torch, binding, a, b, bias, c, M, N, K, epi, cfg, reps, warmup, 
     st = binding.tg_gemm_check_error(stream.cuda_stream)
     if st != binding.TG_OK:
         raise binding.TgError(st, f"config {cfg}")
-    return statistics.median(times)
+    return statistics.fmean(times)
 
 
 def time_library(torch, a, b, bias, epi, reps, warmup, flush):
@@ -106,7 +109,7 @@ def time_library(torch, a, b, bias, epi, reps, warmup, flush):
         e1.record()
         e1.synchronize()
         times.append(e0.elapsed_time(e1))
-    return statistics.median(times)
+    return statistics.fmean(times)
 
 
 def sweep_shape(torch, binding, name, M, N, K, epi, reps, warmup, configs, group_ms=(0,),
@@ -154,7 +157,7 @@ def sweep_shape(torch, binding, name, M, N, K, epi, reps, warmup, configs, group
     # Interleaved rounds: every candidate (and the library context) is timed
     # once per round, so slow drifts of the GPU's clock (power, temperature)
     # touch all of them alike; each result is the median over rounds of the
-    # per-round medians.
+    # per-round means.
     per_round = {i: [] for i in range(len(candidates))}
     lib_rounds = []
     per = max(1, reps // rounds)
@@ -203,7 +206,7 @@ def write_table(results, path=TABLE):
         "// which rewrites this file; shapes it does not list fall back to the cost",
         "// rule in tg_gemm.cu.  The last row is a sentinel (M = -1).",
         "//",
-        "// Written by the sweep on a B200; per row: median ms and TFLOP/s of the winner.",
+        "// Written by the sweep on a B200; per row: ms and TFLOP/s of the winner.",
         "static const TableRow kShapeTable[] = {",
     ]
     for r in results:

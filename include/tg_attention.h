@@ -93,6 +93,22 @@ tg_status_t tg_attention_fwd_ex(const void *Q, const void *K, const void *V, voi
                                 int64_t head_dim, int causal, float scale,
                                 const tg_attention_options_t *opts, void *stream);
 
+/*
+ * tg_attention_plan -- host only: the launch tg_attention_fwd_ex would make
+ * for these arguments on a device with num_sms SMs (148 on B200), without
+ * touching a device.
+ *   units  out: work units, (batch x heads) x ceil(seq_q / 256)
+ *   split  out: units split into two key halves (kv_split, causal and
+ *          seq_k decide, as for tg_attention_fwd_ex)
+ *   grid   out: CTAs launched, units + split
+ * All three are 0 when nothing would be launched (an empty call, seq_k == 0).
+ * Returns TG_ERR_INVALID_ARG for a null output, num_sms <= 0, or the sizes,
+ * head_dim, causal or kv_split that tg_attention_fwd_ex rejects as such.
+ */
+tg_status_t tg_attention_plan(int64_t batch, int64_t heads, int64_t seq_q, int64_t seq_k,
+                              int64_t head_dim, int causal, int kv_split, int num_sms,
+                              int64_t *units, int64_t *split, int64_t *grid);
+
 #ifdef __cplusplus
 }
 #endif

@@ -116,6 +116,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.tg_attention_fwd_ex.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int,
                                         ctypes.c_float, ctypes.POINTER(tg_attention_options_t), vp]
     lib.tg_attention_fwd_ex.restype = c_int
+    i64p = ctypes.POINTER(i64)
+    lib.tg_attention_plan.argtypes = [i64, i64, i64, i64, i64, c_int, c_int, c_int, i64p, i64p,
+                                      i64p]
+    lib.tg_attention_plan.restype = c_int
     _lib = lib
     return lib
 
@@ -260,6 +264,19 @@ def tg_attention_fwd(Q, K, V, O, batch, heads, seq_q, seq_k, head_dim, causal, s
                      stream=None) -> int:
     return load().tg_attention_fwd(Q, K, V, O, batch, heads, seq_q, seq_k, head_dim, int(causal),
                                    float(scale), stream)
+
+
+def tg_attention_plan(batch, heads, seq_q, seq_k, head_dim, causal, kv_split=0,
+                      num_sms=148) -> dict:
+    """Host-only: units, split units and grid of the launch tg_attention_fwd_ex
+    would make (no device needed)."""
+    units, split, grid = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    st = load().tg_attention_plan(batch, heads, seq_q, seq_k, head_dim, int(causal), kv_split,
+                                  num_sms, ctypes.byref(units), ctypes.byref(split),
+                                  ctypes.byref(grid))
+    if st != TG_OK:
+        raise TgError(st, "tg_attention_plan")
+    return {"units": units.value, "split": split.value, "grid": grid.value}
 
 
 def tg_attention_fwd_ex(Q, K, V, O, batch, heads, seq_q, seq_k, head_dim, causal, scale,

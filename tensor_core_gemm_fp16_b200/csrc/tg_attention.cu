@@ -920,6 +920,32 @@ tg_status_t tg_attention_fwd(const void *Q, const void *K, const void *V, void *
                           static_cast<cudaStream_t>(stream));
 }
 
+tg_status_t tg_attention_plan(int64_t batch, int64_t heads, int64_t seq_q, int64_t seq_k,
+                              int64_t head_dim, int causal, int kv_split, int num_sms,
+                              int64_t *units, int64_t *split, int64_t *grid)
+{
+    if (!units || !split || !grid || num_sms <= 0 || batch < 0 || heads < 0 || seq_q < 0 ||
+        seq_k < 0 || (head_dim != 64 && head_dim != 128) || (causal != 0 && causal != 1) ||
+        kv_split < TG_ATTN_SPLIT_AUTO || kv_split > TG_ATTN_SPLIT_ALL)
+        return TG_ERR_INVALID_ARG;
+    if (batch > 0 && heads > (int64_t(1) << 31) / batch) return TG_ERR_INVALID_ARG;
+    if (seq_q > (int64_t(1) << 31) - tga::kTileQ || seq_k > (int64_t(1) << 31) - tga::kTileK)
+        return TG_ERR_INVALID_ARG;
+    *units = *split = *grid = 0;
+    const int64_t bh = batch * heads;
+    if (bh == 0 || seq_q == 0 || seq_k == 0) return TG_OK;   // nothing launched
+    const int64_t pair_rows = static_cast<int64_t>(tga::kTilesPerCta) * tga::kTileQ;
+    const int64_t n_units = bh * ((seq_q + pair_rows - 1) / pair_rows);
+    if (n_units > 0x7fffffff) return TG_ERR_INVALID_ARG;
+    const int64_t key_tiles = (seq_k + tga::kTileK - 1) / tga::kTileK;
+    const int s = split_units(n_units, num_sms, key_tiles, causal, kv_split);
+    if (n_units + s > 0x7fffffff) return TG_ERR_INVALID_ARG;
+    *units = n_units;
+    *split = s;
+    *grid = n_units + s;
+    return TG_OK;
+}
+
 tg_status_t tg_attention_fwd_ex(const void *Q, const void *K, const void *V, void *O,
                                 int64_t batch, int64_t heads, int64_t seq_q, int64_t seq_k,
                                 int64_t head_dim, int causal, float scale,

@@ -175,3 +175,32 @@ def test_softmax_limits_are_checked_on_the_host():
     assert c["epi_warps"] == 4 and c["block_n"] >= 200
     assert binding.tg_gemm(0x1000, 0x200000, None, 0x400000, 4, 4, 4, 5, None) == \
         binding.TG_ERR_INVALID_ARG
+
+
+def test_attention_plan_without_a_device():
+    """The work division of the attention launch, as a host-only query: one
+    unit per (batch x head, 256 queries); a non-causal last wave that fills at
+    most half of the SMs is split into key halves; never for causal calls or a
+    single key tile; forced or disabled by kv_split."""
+    plan = binding.tg_attention_plan
+    assert plan(4, 16, 2048, 2048, 128, False) == {"units": 512, "split": 68, "grid": 580}
+    assert plan(4, 16, 2048, 2048, 64, True) == {"units": 512, "split": 0, "grid": 512}
+    assert plan(4, 16, 2048, 2048, 128, False, kv_split=binding.TG_ATTN_SPLIT_NEVER)["split"] == 0
+    assert plan(1, 2, 256, 256, 64, False) == {"units": 2, "split": 2, "grid": 4}
+    assert plan(1, 2, 256, 128, 64, False)["split"] == 0                  # one key tile
+    assert plan(1, 2, 256, 128, 64, False, kv_split=binding.TG_ATTN_SPLIT_ALL)["split"] == 0
+    assert plan(2, 3, 200, 333, 64, False, kv_split=binding.TG_ATTN_SPLIT_ALL) == \
+        {"units": 6, "split": 6, "grid": 12}
+    assert plan(1, 296, 256, 512, 64, False)["split"] == 0                # two full waves
+    assert plan(1, 248, 256, 512, 64, False)["split"] == 0                # last wave 100 > 74
+    assert plan(1, 222, 256, 512, 64, False)["split"] == 74               # last wave 74
+    assert plan(1, 8, 1000, 512, 64, False, num_sms=16) == {"units": 32, "split": 0, "grid": 32}
+    assert plan(1, 9, 1000, 512, 64, False, num_sms=16) == {"units": 36, "split": 4, "grid": 40}
+    assert plan(0, 4, 128, 128, 64, False) == {"units": 0, "split": 0, "grid": 0}
+    assert plan(1, 1, 128, 0, 64, False) == {"units": 0, "split": 0, "grid": 0}
+    for bad in ({"head_dim": 96}, {"kv_split": 3}, {"num_sms": 0}, {"causal": 2}):
+        args = {"batch": 1, "heads": 1, "seq_q": 128, "seq_k": 128, "head_dim": 64,
+                "causal": 0, "kv_split": 0, "num_sms": 148}
+        args.update(bad)
+        with pytest.raises(binding.TgError):
+            plan(**args)

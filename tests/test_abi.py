@@ -204,3 +204,26 @@ def test_attention_plan_without_a_device():
         args.update(bad)
         with pytest.raises(binding.TgError):
             plan(**args)
+
+
+def test_plain_c_client_compiles_links_and_runs(tmp_path):
+    """Both public headers compile as strict C99, and a C program linked
+    against the library runs its host-only entry points (no GPU needed)."""
+    import os
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(binding.LIB_PATH)
+    exe = tmp_path / "abi_client"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(root, "include"),
+                    os.path.join(root, "tests", "c_client", "abi_client.c"),
+                    "-L", libdir, "-ltg_gemm", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                   check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stdout + out.stderr
+    assert "attention plan: units 512 split 68 grid 580" in out.stdout
+    assert out.stdout.strip().endswith("OK")

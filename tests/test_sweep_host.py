@@ -1,0 +1,75 @@
+"""Host logic of the offline sweep and of the compiled configuration table,
+checked without a GPU: the winner rule (stream-K must win by a margin), the
+table writer's output (it compiles as C++ and reads back the same rows), and
+that the library's configuration choice honours every committed table row."""
+import os
+import re
+import shutil
+import subprocess
+
+import pytest
+
+from tensor_core_gemm_fp16_b200 import binding
+from tensor_core_gemm_fp16_b200 import sweep
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+ROW = re.compile(r"^\s*\{(-?\d+), (-?\d+), (-?\d+), (-?\d+), (-?\d+), (-?\d+)\},")
+
+
+def _row(cfg, split, ms, **kw):
+    return {"config": cfg, "split": split, "ms": ms, "tflops": 1.0, **kw}
+
+
+def test_pick_best_handicaps_stream_k():
+    tiles = _row(3, 1, 1.00e-2)
+    assert sweep.pick_best([tiles, _row(4, 2, 0.98e-2)])["config"] == 3     # 2% faster: not enough
+    assert sweep.pick_best([tiles, _row(4, 2, 0.95e-2)])["config"] == 4     # 5% faster: wins
+    assert sweep.pick_best([tiles, _row(5, 1, 0.99e-2)])["config"] == 5     # whole tiles: plain min
+    assert sweep.pick_best([{"config": 1, "split": 1, "error": "x"}, tiles])["config"] == 3
+    assert sweep.pick_best([{"config": 1, "split": 1, "error": "x"}]) is None
+
+
+def _parse(path):
+    rows = []
+    with open(path) as f:
+        for line in f:
+            m = ROW.match(line)
+            if m:
+                rows.append(tuple(int(g) for g in m.groups()))
+    return rows
+
+
+def test_table_writer_round_trip(tmp_path):
+    results = [
+        {"shape": "a", "M": 64, "N": 128, "K": 256, "epilogue": 2, "best": 3, "best_split": 1,
+         "rows": [_row(3, 1, 1e-2), _row(3, 2, 2e-2)]},
+        {"shape": "b", "M": 7, "N": 9, "K": 11, "epilogue": 0, "best": 4, "best_split": 2,
+         "rows": [_row(4, 2, 1e-3)]},
+        {"shape": "none", "M": 1, "N": 1, "K": 1, "epilogue": 0, "best": None,
+         "best_split": None, "rows": []},
+    ]
+    out = tmp_path / "t.inc"
+    sweep.write_table(results, path=str(out))
+    assert _parse(out) == [(64, 128, 256, 2, 3, 1), (7, 9, 11, 0, 4, 2), (-1, -1, -1, -1, -1, -1)]
+    cxx = shutil.which("g++")
+    if cxx is None:
+        pytest.skip("no C++ compiler")
+    src = tmp_path / "t.cc"
+    src.write_text("#include <cstdint>\nstruct TableRow { int64_t M, N, K; int epilogue; "
+                   "int config; int split; };\n#include \"t.inc\"\n"
+                   "int main() { return kShapeTable[2].M == -1 ? 0 : 1; }\n")
+    exe = tmp_path / "t"
+    subprocess.run([cxx, "-std=c++17", "-Wall", "-Werror", "-I", str(tmp_path), str(src), "-o",
+                    str(exe)], check=True)
+    assert subprocess.run([str(exe)]).returncode == 0
+
+
+def test_committed_table_rows_are_what_the_library_picks():
+    path = os.path.join(ROOT, "tensor_core_gemm_fp16_b200", "csrc", "tg_configs.inc")
+    rows = _parse(path)
+    assert rows and rows[-1] == (-1, -1, -1, -1, -1, -1)
+    n_cfg = binding.tg_num_configs()
+    for M, N, K, epi, cfg, split in rows[:-1]:
+        assert 0 <= cfg < n_cfg and split in (1, 2)
+        got = binding.tg_gemm_select_config(M, N, K, max(epi, 0))   # -1: any epilogue
+        assert (got["id"], got["split"]) == (cfg, split), (M, N, K, epi)

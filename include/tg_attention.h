@@ -54,8 +54,9 @@ extern "C" {
  * (device, stream) of about 266 KB per split unit, allocated in stream
  * order on first need (cudaMallocAsync; TG_ERR_OOM if that fails) and kept
  * for the process; calls that share a stream are ordered by it, calls on
- * different streams use different workspaces.  Bad sizes, head_dim, causal or a non-finite scale return
- * TG_ERR_INVALID_ARG before anything is launched; a device other than
+ * different streams use different workspaces.  Bad sizes, head_dim, causal
+ * or a non-finite scale return TG_ERR_INVALID_ARG before anything is
+ * launched; a device other than
  * compute capability 10.0 returns TG_ERR_UNSUPPORTED_DEVICE (there is no CPU
  * path).  Every device-side wait is bounded (2 s by default); an expiry is
  * reported by tg_gemm_check_error as TG_ERR_TIMEOUT.

@@ -220,7 +220,8 @@ __device__ __forceinline__ int tile_key_tiles(const AttnParams &p, int64_t q0)
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ,
+                    const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p)
 {
     using S = AttnShape<D>;
@@ -360,7 +361,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     !mbar_wait_drain(&k_full[st], (k_filled[st] - 1) & 1, limit))
                     atomicOr(p.error_word, kErrAttnDrain);
             for (int st = 0; st < SV; ++st)
-                if (v_filled[st] > 0 && !mbar_wait_drain(&v_full[st], (v_filled[st] - 1) & 1, limit))
+                if (v_filled[st] > 0 &&
+                    !mbar_wait_drain(&v_full[st], (v_filled[st] - 1) & 1, limit))
                     atomicOr(p.error_word, kErrAttnDrain);
         }
         __syncwarp();
@@ -640,8 +642,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int us = unit - p.num_full;
                     float *mine =
                         p.part + static_cast<size_t>((us * 2 + half) * 2 + t) * (D + 2) * kTileQ;
-                    other =
-                        p.part + static_cast<size_t>((us * 2 + (1 - half)) * 2 + t) * (D + 2) * kTileQ;
+                    other = p.part +
+                            static_cast<size_t>((us * 2 + (1 - half)) * 2 + t) * (D + 2) * kTileQ;
 #pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t o[32];
@@ -827,7 +829,8 @@ tg_status_t launch_attn(const CUtensorMap &tq, const CUtensorMap &tk, const CUte
     const uint64_t bit = uint64_t(1) << dev;
     if (!(attr_set.load() & bit)) {
         if (cudaFuncSetAttribute(tga::attn_fwd_kernel<D>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem) != cudaSuccess) {
             cudaGetLastError();
             return TG_ERR_LAUNCH;
         }
@@ -842,7 +845,8 @@ tg_status_t attention_impl(const void *Q, const void *K, const void *V, void *O,
                            int64_t H, int64_t Sq, int64_t Sk, int64_t D, int causal, float scale,
                            const tg_attention_options_t *opts, cudaStream_t stream)
 {
-    if (B < 0 || H < 0 || Sq < 0 || Sk < 0 || (D != 64 && D != 128) || (causal != 0 && causal != 1) ||
+    if (B < 0 || H < 0 || Sq < 0 || Sk < 0 || (D != 64 && D != 128) ||
+        (causal != 0 && causal != 1) ||
         !std::isfinite(scale) || (scale != 0.f && std::fabs(scale) < 1e-30f))
         return TG_ERR_INVALID_ARG;
     if (opts && opts->inject != 0 && opts->inject != TG_INJECT_SKIP_FIRST_LOAD)

@@ -56,10 +56,10 @@ extern "C" {
  * for the process; calls that share a stream are ordered by it, calls on
  * different streams use different workspaces.  Bad sizes, head_dim, causal
  * or a non-finite scale return TG_ERR_INVALID_ARG before anything is
- * launched; a device other than
- * compute capability 10.0 returns TG_ERR_UNSUPPORTED_DEVICE (there is no CPU
- * path).  Every device-side wait is bounded (2 s by default); an expiry is
- * reported by tg_gemm_check_error as TG_ERR_TIMEOUT.
+ * launched; a device other than compute capability 10.0 returns
+ * TG_ERR_UNSUPPORTED_DEVICE (there is no CPU path).  Every device-side wait
+ * is bounded (2 s by default); an expiry is reported by tg_gemm_check_error
+ * as TG_ERR_TIMEOUT.
  */
 tg_status_t tg_attention_fwd(const void *Q, const void *K, const void *V, void *O, int64_t batch,
                              int64_t heads, int64_t seq_q, int64_t seq_k, int64_t head_dim,

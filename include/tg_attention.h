@@ -54,7 +54,9 @@ extern "C" {
  * (device, stream) of about 266 KB per split unit, allocated in stream
  * order on first need (cudaMallocAsync; TG_ERR_OOM if that fails) and kept
  * for the process; calls that share a stream are ordered by it, calls on
- * different streams use different workspaces.  Bad sizes, head_dim, causal
+ * different streams use different workspaces.  While `stream` is capturing a
+ * CUDA graph nothing is split (the merge flags carry a per-call epoch, which
+ * every replay would repeat).  Bad sizes, head_dim, causal
  * or a non-finite scale return TG_ERR_INVALID_ARG before anything is
  * launched; a device other than compute capability 10.0 returns
  * TG_ERR_UNSUPPORTED_DEVICE (there is no CPU path).  Every device-side wait
@@ -81,7 +83,9 @@ enum {
  *                  kernel exits cleanly and tg_gemm_check_error returns
  *                  TG_ERR_TIMEOUT.
  *   kv_split       TG_ATTN_SPLIT_*; other values: TG_ERR_INVALID_ARG.  Causal
- *                  calls and calls with seq_k <= 128 never split.
+ *                  calls and calls with seq_k <= 128 never split, nor calls
+ *                  on a capturing stream (TG_ATTN_SPLIT_ALL there returns
+ *                  TG_ERR_INVALID_ARG).
  */
 typedef struct {
     uint64_t wait_limit_ns;
@@ -103,6 +107,7 @@ tg_status_t tg_attention_fwd_ex(const void *Q, const void *K, const void *V, voi
  *          seq_k decide, as for tg_attention_fwd_ex)
  *   grid   out: CTAs launched, units + split
  * All three are 0 when nothing would be launched (an empty call, seq_k == 0).
+ * The plan is that of a stream that is not capturing a graph.
  * Returns TG_ERR_INVALID_ARG for a null output, num_sms <= 0, or the sizes,
  * head_dim, causal or kv_split that tg_attention_fwd_ex rejects as such.
  */

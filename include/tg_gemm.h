@@ -118,7 +118,10 @@ typedef enum {
  * epilogue.  The partials live in a workspace owned by the library, created
  * once per (device, stream) on first use (a cudaMalloc of about
  * 148 x 128 KiB plus flags), so stream-K calls on one stream are ordered by
- * that stream; a first call inside a stream capture cannot create it.
+ * that stream; a first call inside a stream capture cannot create it.  While
+ * `stream` is capturing a CUDA graph, stream-K is never used: its flags carry
+ * a per-call epoch, which every replay of the graph would repeat.  Such calls
+ * run whole tiles (an explicit TG_SPLIT_STREAM_K returns TG_ERR_INVALID_ARG).
  */
 tg_status_t tg_gemm(const void *A, const void *B, const void *bias, void *C,
                     int64_t M, int64_t N, int64_t K, int epilogue, void *stream);
@@ -197,7 +200,8 @@ tg_status_t tg_gemm_select_config(int64_t M, int64_t N, int64_t K, int epilogue,
  *   split          TG_SPLIT_AUTO: the table's split for a listed shape, else
  *                  the cost rule of tg_gemm_select_config (for a forced
  *                  config_id too); TG_SPLIT_TILES: always whole tiles;
- *                  TG_SPLIT_STREAM_K: always stream-K (see tg_gemm).
+ *                  TG_SPLIT_STREAM_K: always stream-K (see tg_gemm; not
+ *                  while the stream is capturing a graph).
  */
 #define TG_INJECT_SKIP_FIRST_LOAD 1
 #define TG_INJECT_SKIP_STREAMK_FLAGS 2

@@ -895,8 +895,12 @@ tg_status_t attention_impl(const void *Q, const void *K, const void *V, void *O,
     p.error_word = error_word;
     const int64_t units = bh * num_qp;
     const int64_t key_tiles = (Sk + tga::kTileK - 1) / tga::kTileK;
-    const int split = split_units(units, num_sms, key_tiles, causal,
-                                  opts ? opts->kv_split : TG_ATTN_SPLIT_AUTO);
+    // The merge flags hold a per-call epoch, which a replayed graph would
+    // repeat: no split while the stream is capturing.
+    const int mode = opts ? opts->kv_split : TG_ATTN_SPLIT_AUTO;
+    const bool capturing = tg_internal_capturing(stream);
+    if (capturing && mode == TG_ATTN_SPLIT_ALL) return TG_ERR_INVALID_ARG;
+    const int split = capturing ? 0 : split_units(units, num_sms, key_tiles, causal, mode);
     if (units + split > 0x7fffffff) return TG_ERR_INVALID_ARG;
     p.num_full = static_cast<int>(units - split);
     p.split_units = split;

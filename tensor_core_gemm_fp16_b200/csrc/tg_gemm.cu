@@ -477,6 +477,12 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
         choice = {opts->config_id, rule_split(opts->config_id, M, N, K, epilogue, dev->num_sms)};
     else
         choice = choose_config(M, N, K, epilogue, dev->num_sms);
+    // Stream-K flags hold a per-call epoch, which a replayed graph would
+    // repeat: whole tiles while the stream is capturing.
+    if (tg_internal_capturing(stream)) {
+        if (opts && opts->split == TG_SPLIT_STREAM_K) return TG_ERR_INVALID_ARG;
+        choice.split = TG_SPLIT_TILES;
+    }
     const int cfg_id = choice.config;
     const KernelConfig &cfg = kConfigs[cfg_id];
     const int bn = cfg.info.block_n;

@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cuda_runtime.h>
 
 #include "tg_gemm.h"
 
@@ -13,3 +14,17 @@
 // reads and clears it) and the driver's tensor-map encoder.
 __attribute__((visibility("hidden"))) tg_status_t tg_internal_device(
     int *num_sms, unsigned **error_word, PFN_cuTensorMapEncodeTiled_v12000 *encode);
+
+// True while `stream` is capturing a CUDA graph.  A graph replays a kernel
+// with the parameters it was captured with, so the launches whose cross-CTA
+// flags carry a per-call epoch (stream-K GEMM, key-half split attention)
+// would meet their own epoch on every replay; callers avoid them then.
+static inline bool tg_internal_capturing(cudaStream_t stream)
+{
+    cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &st) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return st != cudaStreamCaptureStatusNone;
+}

@@ -25,6 +25,7 @@ import argparse
 import json
 import math
 import os
+import re
 import statistics
 import sys
 
@@ -196,7 +197,25 @@ def pick_best(rows):
     return min(ok, key=lambda r: r["ms"] * (STREAM_K_MARGIN if r.get("split") == 2 else 1.0))
 
 
-def write_table(results, path=TABLE):
+_TABLE_ROW = re.compile(r"^\s*\{(-?\d+), (-?\d+), (-?\d+), (-?\d+), (-?\d+), (-?\d+)\},"
+                        r"\s*(//.*)?$")
+
+
+def read_table(path=TABLE):
+    """The rows of a configuration table file, each (M, N, K, epilogue, config,
+    split, comment), sentinel excluded."""
+    rows = []
+    with open(path) as f:
+        for line in f:
+            m = _TABLE_ROW.match(line)
+            if m and int(m.group(1)) >= 0:
+                rows.append(tuple(int(g) for g in m.groups()[:6]) + ((m.group(7) or "").strip(),))
+    return rows
+
+
+def write_table(results, path=TABLE, keep=()):
+    """Write the table: one row per swept shape with a winner, then the rows
+    of `keep` (from read_table) whose shape this sweep did not cover."""
     lines = [
         "// tg_configs.inc -- per-shape configuration table.",
         "//",
@@ -217,6 +236,11 @@ def write_table(results, path=TABLE):
         lines.append(f"    {{{r['M']}, {r['N']}, {r['K']}, {r['epilogue']}, {r['best']}, "
                      f"{r['best_split']}}},"
                      f"  // {r['shape']}: {w['ms'] * 1e3:.1f} us, {w['tflops']:.0f} TFLOP/s")
+    swept = {(r["M"], r["N"], r["K"], r["epilogue"]) for r in results}
+    for M, N, K, epi, cfg, split, comment in keep:
+        if (M, N, K, epi) not in swept:
+            lines.append(f"    {{{M}, {N}, {K}, {epi}, {cfg}, {split}}},"
+                         + (f"  {comment}" if comment else ""))
     lines += ["    {-1, -1, -1, -1, -1, -1},", "};", ""]
     with open(path, "w") as f:
         f.write("\n".join(lines))
@@ -238,6 +262,9 @@ def main(argv=None):
     ap.add_argument("--context", action="store_true",
                     help="also time torch.matmul (+ eager bias/GELU) on each shape")
     ap.add_argument("--write", action="store_true", help="rewrite csrc/tg_configs.inc")
+    ap.add_argument("--keep-others", action="store_true",
+                    help="with --write or --from-json: keep the table's rows for shapes this "
+                         "sweep did not cover")
     ap.add_argument("--json", default=None)
     ap.add_argument("--from-json", default=None,
                     help="rewrite the table from a saved sweep (no GPU needed)")
@@ -249,7 +276,7 @@ def main(argv=None):
             best = pick_best(r["rows"])
             r["best"] = best["config"] if best else None
             r["best_split"] = best["split"] if best else None
-        write_table(results)
+        write_table(results, keep=read_table() if args.keep_others else ())
         return 0
     sys.path.insert(0, os.path.dirname(HERE))
     import torch
@@ -282,7 +309,7 @@ def main(argv=None):
         with open(args.json, "w") as f:
             json.dump(results, f, indent=1)
     if args.write:
-        write_table(results)
+        write_table(results, keep=read_table() if args.keep_others else ())
     return 0
 
 

@@ -73,3 +73,21 @@ def test_committed_table_rows_are_what_the_library_picks():
         assert 0 <= cfg < n_cfg and split in (1, 2)
         got = binding.tg_gemm_select_config(M, N, K, max(epi, 0))   # -1: any epilogue
         assert (got["id"], got["split"]) == (cfg, split), (M, N, K, epi)
+
+
+def test_partial_sweep_keeps_the_other_rows(tmp_path):
+    """A sweep of some shapes rewrites their rows and, with keep, leaves the
+    table's other rows (and their comments) as they were."""
+    committed = sweep.read_table()
+    assert len(committed) >= 2 and all(len(r) == 7 for r in committed)
+    first = committed[0]
+    results = [{"shape": "new", "M": first[0], "N": first[1], "K": first[2],
+                "epilogue": first[3], "best": 1, "best_split": 2,
+                "rows": [_row(1, 2, 1e-2)]}]
+    out = tmp_path / "t.inc"
+    sweep.write_table(results, path=str(out), keep=committed)
+    merged = sweep.read_table(str(out))
+    assert merged[0][:6] == first[:4] + (1, 2)
+    assert merged[1:] == committed[1:]
+    sweep.write_table(results, path=str(out))
+    assert len(sweep.read_table(str(out))) == 1

@@ -87,7 +87,8 @@ def profiled_traffic(workload: str, kernel_config: dict):
     code or launch configuration)."""
     path = os.path.join(ROOT, "profiles", f"gemm_persistent_kernel_{workload}.md")
     try:
-        text = open(path).read()
+        with open(path) as f:
+            text = f.read()
     except OSError:
         return None
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)

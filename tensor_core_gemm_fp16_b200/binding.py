@@ -128,7 +128,8 @@ def header_symbols(headers=None):
     """Function names declared in the library's headers (include/*.h)."""
     names = set()
     for header in ([headers] if isinstance(headers, str) else (headers or HEADERS)):
-        text = open(header).read()
+        with open(header) as f:
+            text = f.read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
         names.update(re.findall(r"\b(tg_[a-z0-9_]+)\s*\(", text))
     return sorted(names)

@@ -41,6 +41,13 @@
 // in TMEM only on those tiles; O / l uses the same m, so the result is the
 // same softmax.
 //
+// Key-half split (non-causal): when the last wave of units would fill at
+// most half of the SMs, each of its units runs as two CTAs over the first and
+// the second half of the key tiles.  Each half publishes its unnormalised O,
+// m and l; the warp that finds its partner's publication (an epoch swapped
+// into a flag word) merges the two with the same rescaling, half 0's terms
+// first.  Nothing waits on the other half.
+//
 // Every mbarrier wait is bounded by a global-timer limit; on expiry a CTA
 // abort flag is set, a site bit is OR-ed into the library error word, and
 // the CTA tears down after letting its own copies and MMAs land.

@@ -470,3 +470,36 @@ def test_thread_count_changes_no_result():
         oracle.set_num_threads(prev)
     assert oracle.num_threads() == prev
     assert np.array_equal(many, one)
+
+
+def test_brute_force_every_tiny_shape_exact():
+    """Every (M, N, K) in {1..9}^3, plus 17 x 31 x 17 and 31 x 17 x 31, random
+    fp16 operands and bias: the oracle against the exact sum, computed in
+    integers (each fp16 value times 2^24 is an integer, so every product is
+    an exact integer multiple of 2^-48).  NONE and BIAS within the fp64 bound
+    of a K-term sum; BIAS_GELU within that bound carried through v Phi(v)."""
+    import itertools
+    shapes = list(itertools.product(range(1, 10), repeat=3)) + [(17, 31, 17), (31, 17, 31)]
+    scale = 1 << 24
+    for idx, (M, N, K) in enumerate(shapes):
+        A, B, bias = wl.make_inputs(M, N, K, seed=10_000 + idx, bias=True)
+        a, b, bb = _dec(A), _dec(B), _dec(bias)
+        ai = [[int(a[i, k] * scale) for k in range(K)] for i in range(M)]
+        bi = [[int(b[k, j] * scale) for j in range(N)] for k in range(K)]
+        epis = (oracle.EPI_NONE, oracle.EPI_BIAS) if idx % 7 else \
+            (oracle.EPI_NONE, oracle.EPI_BIAS, oracle.EPI_BIAS_GELU)
+        got = {epi: _oracle_gemm(A, B, bias, epi) for epi in epis}
+        for i in range(M):
+            for j in range(N):
+                exact = Fraction(sum(ai[i][k] * bi[k][j] for k in range(K)), scale * scale)
+                mag = float(sum(abs(ai[i][k] * bi[k][j]) for k in range(K))) / scale ** 2
+                for epi in epis:
+                    s = exact + (Fraction(bb[j]) if epi != oracle.EPI_NONE else 0)
+                    v = float(s)
+                    bound = (K + 1) * 2.0 ** -52 * (mag + abs(bb[j]))
+                    if epi == oracle.EPI_BIAS_GELU:
+                        want = v * ndtr(v)
+                        bound = 2 * bound + 1e-13 * abs(want) + 1e-300
+                    else:
+                        want = v
+                    assert abs(got[epi][i, j] - want) <= bound, (M, N, K, epi, i, j)

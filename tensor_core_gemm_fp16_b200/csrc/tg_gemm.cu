@@ -449,6 +449,80 @@ tg_status_t launch_pack(const void *src, int64_t rows, int64_t cols, void *dst, 
     return cudaGetLastError() == cudaSuccess ? TG_OK : TG_ERR_LAUNCH;
 }
 
+// Tensor maps, kernel parameters, work division and launch of the GEMM on
+// operands already in a form the configuration can read (TMA: 16-byte
+// aligned bases and pitches lda, ldb; the plain loader: any 2-byte aligned
+// pitch).  Shared by tg_gemm and tg_gemm_noalloc, which differ only in where
+// repacked operands live.  `split` is TG_SPLIT_TILES or TG_SPLIT_STREAM_K;
+// stream-K takes the (device, stream) workspace.
+tg_status_t launch_staged(const KernelConfig &cfg, const void *Aeff, int64_t lda, const void *Beff,
+                          int64_t ldb, const void *bias, void *C, int64_t M, int64_t N, int64_t K,
+                          int epilogue, int split, const tg_options_t *opts, int num_sms,
+                          unsigned *error_word, cudaStream_t stream)
+{
+    const bool plain = cfg.info.loader == tg::kLoadPlain;
+    const bool c_rows16 = aligned(C, 16) && (N % 8 == 0);
+    const int store = c_rows16 ? cfg.store_pref : tg::kStoreScalar;
+    CUtensorMap ta, tb, tc;
+    std::memset(&ta, 0, sizeof(ta));
+    std::memset(&tb, 0, sizeof(tb));
+    std::memset(&tc, 0, sizeof(tc));
+    if ((!plain && (!encode_2d(&ta, Aeff, K, M, 2 * lda, tg::kAtomK, tg::kBlockM,
+                               CU_TENSOR_MAP_SWIZZLE_128B) ||
+                    !encode_2d(&tb, Beff, N, K, 2 * ldb, tg::kBChunkN, cfg.info.block_k,
+                               CU_TENSOR_MAP_SWIZZLE_128B))) ||
+        (store == tg::kStoreTma &&
+         !encode_2d(&tc, C, N, M, 2 * N, tg::kStoreCols, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
+        return TG_ERR_CUDA;
+
+    tg::GemmParams p;
+    p.A = static_cast<const __half *>(Aeff);
+    p.B = static_cast<const __half *>(Beff);
+    p.lda = lda;
+    p.ldb = ldb;
+    p.bias = static_cast<const __half *>(bias);
+    p.C = static_cast<__half *>(C);
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.ldc = N;
+    p.num_m_tiles = static_cast<int>(ceil_div(M, cfg.info.block_m));
+    p.num_n_tiles = static_cast<int>(ceil_div(N, cfg.info.block_n));
+    p.num_k_blocks = static_cast<int>(ceil_div(K, cfg.info.block_k));
+    p.num_tiles = p.num_m_tiles * p.num_n_tiles;
+    p.group_m = (opts && opts->group_m > 0) ? opts->group_m : cfg.info.group_m;
+    p.inject = opts ? opts->inject : 0;
+    p.bias_vec = (bias && aligned(bias, 16)) ? 1 : 0;
+    p.wait_limit_ns = (opts && opts->wait_limit_ns) ? opts->wait_limit_ns : kDefaultWaitLimitNs;
+    p.error_word = error_word;
+    // Persistent grid: one CTA (or CTA pair) per SM (pair of SMs).  Whole
+    // tiles: never more units than tiles.
+    const int units = cfg.info.cta_pair ? num_sms / 2 : num_sms;
+    const int64_t iters = static_cast<int64_t>(p.num_tiles) * p.num_k_blocks;
+    const bool stream_k = split == TG_SPLIT_STREAM_K;
+    p.stream_k = stream_k ? 1 : 0;
+    p.sk_partials = nullptr;
+    p.sk_flags = nullptr;
+    p.sk_epoch = 0;
+    if (stream_k) {
+        const tg_status_t st =
+            streamk_workspace(num_sms, stream, &p.sk_partials, &p.sk_flags, &p.sk_epoch);
+        if (st != TG_OK) return st;
+    }
+    // Stream-K: at most one unit per iteration, so that no unit's range is empty.
+    const int grid = static_cast<int>(stream_k ? std::min<int64_t>(iters, units)
+                                               : std::min<int64_t>(p.num_tiles, units)) *
+                     (cfg.info.cta_pair ? 2 : 1);
+
+    const cudaError_t e =
+        cfg.fn[epilogue][store == tg::kStoreScalar ? 0 : 1](ta, tb, tc, p, grid, stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_LAUNCH;
+    }
+    return TG_OK;
+}
+
 tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, int64_t M,
                       int64_t N, int64_t K, int epilogue, const tg_options_t *opts,
                       cudaStream_t stream)
@@ -485,7 +559,6 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
     }
     const int cfg_id = choice.config;
     const KernelConfig &cfg = kConfigs[cfg_id];
-    const int bn = cfg.info.block_n;
     if (epilogue == TG_EPILOGUE_BIAS_SOFTMAX && !softmax_capable(cfg.info, N))
         return TG_ERR_INVALID_ARG;
     const bool plain = cfg.info.loader == tg::kLoadPlain;
@@ -518,71 +591,11 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
         }
     }
 
-    const bool c_rows16 = aligned(C, 16) && (N % 8 == 0);
-    const int store = c_rows16 ? cfg.store_pref : tg::kStoreScalar;
-    CUtensorMap ta, tb, tc;
-    std::memset(&ta, 0, sizeof(ta));
-    std::memset(&tb, 0, sizeof(tb));
-    std::memset(&tc, 0, sizeof(tc));
-    if ((!plain && (!encode_2d(&ta, Aeff, K, M, 2 * lda, tg::kAtomK, tg::kBlockM,
-                               CU_TENSOR_MAP_SWIZZLE_128B) ||
-                    !encode_2d(&tb, Beff, N, K, 2 * ldb, tg::kBChunkN, cfg.info.block_k,
-                               CU_TENSOR_MAP_SWIZZLE_128B))) ||
-        (store == tg::kStoreTma &&
-         !encode_2d(&tc, C, N, M, 2 * N, tg::kStoreCols, 32, CU_TENSOR_MAP_SWIZZLE_64B))) {
-        if (tmp) cudaFreeAsync(tmp, stream);
-        return TG_ERR_CUDA;
-    }
-
-    tg::GemmParams p;
-    p.A = static_cast<const __half *>(Aeff);
-    p.B = static_cast<const __half *>(Beff);
-    p.lda = lda;
-    p.ldb = ldb;
-    p.bias = static_cast<const __half *>(bias);
-    p.C = static_cast<__half *>(C);
-    p.M = M;
-    p.N = N;
-    p.K = K;
-    p.ldc = N;
-    p.num_m_tiles = static_cast<int>(ceil_div(M, cfg.info.block_m));
-    p.num_n_tiles = static_cast<int>(ceil_div(N, bn));
-    p.num_k_blocks = static_cast<int>(ceil_div(K, cfg.info.block_k));
-    p.num_tiles = p.num_m_tiles * p.num_n_tiles;
-    p.group_m = (opts && opts->group_m > 0) ? opts->group_m : cfg.info.group_m;
-    p.inject = opts ? opts->inject : 0;
-    p.bias_vec = (bias && aligned(bias, 16)) ? 1 : 0;
-    p.wait_limit_ns = (opts && opts->wait_limit_ns) ? opts->wait_limit_ns : kDefaultWaitLimitNs;
-    p.error_word = dev->error_word;
-    // Persistent grid: one CTA (or CTA pair) per SM (pair of SMs).  Whole
-    // tiles: never more units than tiles.
-    const int units = cfg.info.cta_pair ? dev->num_sms / 2 : dev->num_sms;
-    const int split = (opts && opts->split != TG_SPLIT_AUTO) ? opts->split : choice.split;
-    const int64_t iters = static_cast<int64_t>(p.num_tiles) * p.num_k_blocks;
-    const bool stream_k = split == TG_SPLIT_STREAM_K;
-    p.stream_k = stream_k ? 1 : 0;
-    p.sk_partials = nullptr;
-    p.sk_flags = nullptr;
-    p.sk_epoch = 0;
-    if (stream_k) {
-        st = streamk_workspace(dev->num_sms, stream, &p.sk_partials, &p.sk_flags, &p.sk_epoch);
-        if (st != TG_OK) {
-            if (tmp) cudaFreeAsync(tmp, stream);
-            return st;
-        }
-    }
-    // Stream-K: at most one unit per iteration, so that no unit's range is empty.
-    const int grid = static_cast<int>(stream_k ? std::min<int64_t>(iters, units)
-                                               : std::min<int64_t>(p.num_tiles, units)) *
-                     (cfg.info.cta_pair ? 2 : 1);
-
-    cudaError_t e = cfg.fn[epilogue][store == tg::kStoreScalar ? 0 : 1](ta, tb, tc, p, grid, stream);
+    st = launch_staged(cfg, Aeff, lda, Beff, ldb, bias, C, M, N, K, epilogue,
+                       (opts && opts->split != TG_SPLIT_AUTO) ? opts->split : choice.split, opts,
+                       dev->num_sms, dev->error_word, stream);
     if (tmp) cudaFreeAsync(tmp, stream);
-    if (e != cudaSuccess) {
-        cudaGetLastError();
-        return TG_ERR_LAUNCH;
-    }
-    return TG_OK;
+    return st;
 }
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
@@ -947,51 +960,9 @@ tg_status_t gemm_noalloc_impl(const void *A, const void *B, const void *bias, vo
         Beff = bdst;
     }
 
-    const bool c_rows16 = aligned(C, 16) && (N % 8 == 0);
-    const int store = c_rows16 ? cfg.store_pref : tg::kStoreScalar;
-    CUtensorMap ta, tb, tc;
-    std::memset(&tc, 0, sizeof(tc));
-    if (!encode_2d(&ta, Aeff, K, M, 2 * lda, tg::kAtomK, tg::kBlockM,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&tb, Beff, N, K, 2 * ldb, tg::kBChunkN, cfg.info.block_k,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        (store == tg::kStoreTma &&
-         !encode_2d(&tc, C, N, M, 2 * N, tg::kStoreCols, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
-        return TG_ERR_CUDA;
-
-    tg::GemmParams p;
-    p.A = static_cast<const __half *>(Aeff);
-    p.B = static_cast<const __half *>(Beff);
-    p.lda = lda;
-    p.ldb = ldb;
-    p.bias = static_cast<const __half *>(bias);
-    p.C = static_cast<__half *>(C);
-    p.M = M;
-    p.N = N;
-    p.K = K;
-    p.ldc = N;
-    p.num_m_tiles = static_cast<int>(ceil_div(M, cfg.info.block_m));
-    p.num_n_tiles = static_cast<int>(ceil_div(N, cfg.info.block_n));
-    p.num_k_blocks = static_cast<int>(ceil_div(K, cfg.info.block_k));
-    p.num_tiles = p.num_m_tiles * p.num_n_tiles;
-    p.group_m = cfg.info.group_m;
-    p.inject = 0;
-    p.bias_vec = (bias && aligned(bias, 16)) ? 1 : 0;
-    p.wait_limit_ns = kDefaultWaitLimitNs;
-    p.error_word = dev->error_word;
-    p.stream_k = 0;   // stream-K needs a workspace; this entry point allocates nothing
-    p.sk_partials = nullptr;
-    p.sk_flags = nullptr;
-    p.sk_epoch = 0;
-    const int units = cfg.info.cta_pair ? dev->num_sms / 2 : dev->num_sms;
-    const int grid = static_cast<int>(std::min<int64_t>(p.num_tiles, units)) *
-                     (cfg.info.cta_pair ? 2 : 1);
-    if (cfg.fn[epilogue][store == tg::kStoreScalar ? 0 : 1](ta, tb, tc, p, grid, stream) !=
-        cudaSuccess) {
-        cudaGetLastError();
-        return TG_ERR_LAUNCH;
-    }
-    return TG_OK;
+    // stream-K needs a workspace; this entry point allocates nothing
+    return launch_staged(cfg, Aeff, lda, Beff, ldb, bias, C, M, N, K, epilogue, TG_SPLIT_TILES,
+                         nullptr, dev->num_sms, dev->error_word, stream);
 }
 
 }  // namespace

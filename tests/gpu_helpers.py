@@ -53,6 +53,34 @@ def assert_close(C, ref, what=""):
     return rel
 
 
+def assert_close_blocked(C, ref, what="", block_rows=512):
+    """assert_close over the whole output, taken in row blocks so that a
+    full 8192 x 8192 comparison needs no (M, N) temporaries beyond the two
+    operands: the per-element rule and the finiteness check per block, the
+    relative Frobenius error from sums accumulated over every block."""
+    c_all = C if isinstance(C, torch.Tensor) else torch.from_numpy(np.asarray(C))
+    assert tuple(c_all.shape) == ref.shape, (tuple(c_all.shape), ref.shape)
+    err2 = 0.0
+    ref2 = 0.0
+    for r0 in range(0, ref.shape[0], block_rows):
+        r1 = min(ref.shape[0], r0 + block_rows)
+        c = c_all[r0:r1].to(torch.float64).numpy()
+        rb = ref[r0:r1]
+        assert np.all(np.isfinite(c)), f"{what}: non-finite output in rows {r0}..{r1}"
+        err = np.abs(c - rb)
+        bad = err > ELEM_TOL * np.maximum(1.0, np.abs(rb))
+        if bad.any():
+            i, j = np.argwhere(bad)[0]
+            raise AssertionError(f"{what}: {bad.sum()} elements over tolerance in rows "
+                                 f"{r0}..{r1}; first at ({r0 + i},{j}): got {c[i, j]!r} "
+                                 f"want {rb[i, j]!r}")
+        err2 += float(np.sum(err * err))
+        ref2 += float(np.sum(rb * rb))
+    rel = np.sqrt(err2 / ref2) if ref2 > 0 else np.sqrt(err2)
+    assert rel <= REL_FROB_TOL, f"{what}: relative Frobenius error {rel:.3e} > {REL_FROB_TOL}"
+    return rel
+
+
 def assert_bits_equal(C, expected_bits, what=""):
     got = wl.to_bits(C.contiguous())
     exp = np.asarray(expected_bits, dtype=np.uint16)

@@ -12,6 +12,13 @@ from tensor_core_gemm_fp16_b200 import binding
 NONE, BIAS, GELU = 0, 1, 2
 
 
+# Tests marked no_device_only pass made-up device addresses that host validation must reject
+# before any device call.  They run only where no CUDA device exists, so a
+# regression in the validation can never reach a GPU with those addresses.
+no_device_only = pytest.mark.skipif(torch.cuda.is_available(),
+                                    reason="made-up addresses: host-only check")
+
+
 def test_library_exports_every_header_symbol():
     lib = binding.load()
     names = binding.header_symbols()
@@ -21,6 +28,7 @@ def test_library_exports_every_header_symbol():
         assert hasattr(lib, name), f"{name} declared in include/*.h but not exported"
 
 
+@no_device_only
 def test_attention_host_validation_without_a_device():
     """Every call here is rejected on the host before any device query."""
     f = binding.tg_attention_fwd
@@ -103,6 +111,7 @@ def test_select_config_rejects_bad_args():
         binding.tg_gemm_select_config(4, 4, 4, 0, 0)
 
 
+@no_device_only
 def test_host_validation_rejects_bad_calls_without_a_device():
     g = binding.tg_gemm
     # bad epilogue
@@ -137,6 +146,7 @@ def test_empty_problems_are_ok_without_a_device():
     assert binding.tg_gemm(None, None, None, None, 4, 0, 4, 2, None) == binding.TG_OK
 
 
+@no_device_only
 def test_host_entry_validation():
     lib = binding
     need = lib.tg_gemm_host_workspace_size(10, 20, 30, True)
@@ -149,7 +159,26 @@ def test_host_entry_validation():
         binding.TG_ERR_INVALID_ARG
 
 
-@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device answer")
+@no_device_only
+def test_noalloc_scratch_limit_is_checked_on_the_host():
+    # K = 127 repacks A into 128-element rows (256 bytes each): 131072 rows
+    # need exactly TG_NOALLOC_SCRATCH_BYTES and pass the size check (then
+    # find no device); one row more needs 256 bytes more and is rejected.
+    limit = binding.noalloc_scratch_bytes()
+    M = limit // 256
+    f = binding.tg_gemm_noalloc
+    assert f(0x1000000, 0x100000000, None, 0x200000000, M, 8, 127, 0, None) == \
+        binding.TG_ERR_UNSUPPORTED_DEVICE
+    st = f(0x1000000, 0x100000000, None, 0x200000000, M + 1, 8, 127, 0, None)
+    assert st == binding.TG_ERR_SCRATCH_LIMIT
+    # B repacked alone: K * N8 * 2 bytes (N = 1023 -> 1024-element rows)
+    assert f(0x1000000, 0x100000000, None, 0x200000000, 8, 1023, limit // 2048, 0, None) == \
+        binding.TG_ERR_UNSUPPORTED_DEVICE
+    assert f(0x1000000, 0x100000000, None, 0x200000000, 8, 1023, limit // 2048 + 1, 0, None) == \
+        binding.TG_ERR_SCRATCH_LIMIT
+
+
+@no_device_only
 def test_valid_call_without_a_device_reports_unsupported_device():
     # Passes host validation, then finds no sm_100 device: nothing runs.
     st = binding.tg_gemm(0x100000, 0x200000, None, 0x300000, 4, 4, 4, 0, None)
@@ -166,6 +195,7 @@ def test_binding_checks_tensor_arguments():
         binding.gemm(h, h)          # not CUDA tensors
 
 
+@no_device_only
 def test_softmax_limits_are_checked_on_the_host():
     assert binding.tg_gemm(0x1000, 0x200000, None, 0x400000, 4, 257, 4, 4, None) == \
         binding.TG_ERR_INVALID_ARG

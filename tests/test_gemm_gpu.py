@@ -8,7 +8,8 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import assert_bits_equal, assert_close, run_gpu, run_oracle
+from gpu_helpers import (assert_bits_equal, assert_close, assert_close_blocked, run_gpu,
+                         run_oracle)
 from tensor_core_gemm_fp16_b200 import binding
 from tensor_core_gemm_fp16_b200 import workloads as wl
 
@@ -217,24 +218,17 @@ def test_workload_full_parity(name):
     assert_close(C, run_oracle(A, B, bias, w.epilogue), name)
 
 
-def _sample_rows(M, n, seed):
-    rng = np.random.default_rng(seed)
-    fixed = [0, 1, 127, 128, 255, M // 2, M - 129, M - 128, M - 2, M - 1]
-    rnd = rng.choice(M, size=n, replace=False)
-    return sorted(set(int(r) for r in fixed + list(rnd) if 0 <= r < M))
-
-
 @pytest.mark.parametrize("name", ["fused_8192", "fused_8192_literal"])
-def test_large_workload_sampled_rows(name):
-    """Full-size 8192^3 launch (the benchmark's configuration); every column
-    of ~40 sampled rows against the oracle, plus whole-output sanity."""
+def test_large_workload_full_parity(name):
+    """Full-size 8192^3 launch in the benchmark's configuration, every one of
+    the 67,108,864 outputs against the whole fp64 oracle result (about 40 s
+    of oracle time on 16 host cores per workload)."""
     w = wl.WORKLOADS[name]
     A, B, bias = wl.workload_inputs(w)
     C = run_gpu(A, B, bias, w.epilogue)
-    rows = _sample_rows(w.M, 30, seed=w.seed)
-    ref = run_oracle(A, B, bias, w.epilogue, rows=rows)
-    assert_close(C[rows], ref, f"{name} sampled rows")
-    assert torch.isfinite(C.float()).all()
+    ref = run_oracle(A, B, bias, w.epilogue)
+    assert ref.shape == (w.M, w.N)
+    assert_close_blocked(C, ref, name)
 
 
 def test_deterministic():

@@ -6,10 +6,11 @@ driver's allocator) use tg_gemm_noalloc: repacking scratch for unaligned
 operands comes from a fixed device array inside the library instead of a
 memory pool.  These tests call it through the C ABI and compare its output
 with tg_gemm's, under the same acceptance rule as the parity tests, on calls
-in a row that reuse the shared scratch array.  The file is named so that
+in a row that reuse the shared scratch array.  Every buffer handed to the
+library is a real device allocation of the size the call implies, including
+in the calls that are expected to be rejected.  The file is named so that
 pytest collects it last.
 """
-import numpy as np
 import pytest
 import torch
 
@@ -37,6 +38,16 @@ def _run(entry, a, b, bias, M, N, K, epilogue):
     return c.cpu()
 
 
+def _scratch_needed(M, N, K):
+    """Bytes of repacking scratch a call with 16-byte aligned bases needs, as
+    the header states it: 2*M*K8 rounded up to 256 when K % 8 != 0, plus
+    2*K*N8 when N % 8 != 0."""
+    k8, n8 = -(-K // 8) * 8, -(-N // 8) * 8
+    a = 0 if K % 8 == 0 else -(-(2 * M * k8) // 256) * 256
+    b = 0 if N % 8 == 0 else 2 * K * n8
+    return a + b
+
+
 @pytest.fixture(scope="module", autouse=True)
 def _device():
     if not torch.cuda.is_available():
@@ -56,22 +67,41 @@ def test_noalloc_matches_tg_gemm_on_two_calls_in_a_row():
         assert_close(got, ref, f"tg_gemm_noalloc call {call + 1}")
 
 
-def test_noalloc_after_a_larger_call_and_with_aligned_operands():
-    # A smaller unaligned problem after a larger one (the scratch keeps the
-    # larger call's bytes), then an aligned problem that needs no scratch.
-    for (M, N, K, seed) in [(1000, 777, 1030, 11), (512, 1024, 768, 12)]:
-        a, b, bias = _device_inputs(M, N, K, seed=seed, dist="normal")
-        ref = _run(binding.tg_gemm, a, b, bias, M, N, K, binding.TG_EPILOGUE_BIAS).double().numpy()
-        got = _run(binding.tg_gemm_noalloc, a, b, bias, M, N, K, binding.TG_EPILOGUE_BIAS)
-        assert_close(got, ref, f"tg_gemm_noalloc {M}x{N}x{K}")
+@pytest.mark.parametrize("M,N,K,seed", [
+    (1000, 777, 1030, 11),   # A and B repacked, after a larger call
+    (700, 333, 512, 13),     # B alone repacked: it starts at the array's first byte
+    (640, 256, 390, 14),     # A alone repacked
+    (512, 1024, 768, 12),    # aligned: no scratch
+])
+def test_noalloc_repacking_cases(M, N, K, seed):
+    # The scratch keeps the bytes of whatever call ran before.
+    a, b, bias = _device_inputs(M, N, K, seed=seed, dist="normal")
+    ref = _run(binding.tg_gemm, a, b, bias, M, N, K, binding.TG_EPILOGUE_BIAS).double().numpy()
+    got = _run(binding.tg_gemm_noalloc, a, b, bias, M, N, K, binding.TG_EPILOGUE_BIAS)
+    assert_close(got, ref, f"tg_gemm_noalloc {M}x{N}x{K}")
 
 
-def test_noalloc_rejects_problems_beyond_its_scratch():
-    # A needs repacking (K not a multiple of 8): 2 * M * K8 bytes > the limit.
+def test_noalloc_accepts_exactly_its_scratch_and_rejects_one_block_more():
+    # K = 127 repacks A into 128-element rows: 256 bytes of scratch per row.
+    # 131072 rows need exactly TG_NOALLOC_SCRATCH_BYTES (accepted); 131073
+    # rows need 256 bytes more (rejected before anything is launched).
     limit = binding.noalloc_scratch_bytes()
-    K = 4001
-    M = limit // (2 * 4008) + 1
-    st = binding.tg_gemm_noalloc(0x100000, 0x40000000000, None, 0x80000000000, M, 8, K,
-                                 binding.TG_EPILOGUE_NONE, None)
-    assert st == binding.TG_ERR_SCRATCH_LIMIT
+    K, N = 127, 8
+    M_fit = limit // 256
+    assert _scratch_needed(M_fit, N, K) == limit
+    assert _scratch_needed(M_fit + 1, N, K) == limit + 256
+    epi = binding.TG_EPILOGUE_NONE
+    a, b, bias = _device_inputs(M_fit + 1, N, K, seed=15, dist="normal")
+    a_fit = a[:M_fit]
+    ref = _run(binding.tg_gemm, a_fit, b, bias, M_fit, N, K, epi).double().numpy()
+    got = _run(binding.tg_gemm_noalloc, a_fit, b, bias, M_fit, N, K, epi)
+    assert_close(got, ref, "tg_gemm_noalloc at exactly its scratch size")
+
+    c = torch.full((M_fit + 1, N), 7.0, dtype=torch.float16, device=a.device)
+    stream = torch.cuda.current_stream().cuda_stream
+    st = binding.tg_gemm_noalloc(a.data_ptr(), b.data_ptr(), None, c.data_ptr(), M_fit + 1, N, K,
+                                 epi, stream)
+    assert st == binding.TG_ERR_SCRATCH_LIMIT, binding.tg_status_string(st)
     assert "TG_NOALLOC_SCRATCH_BYTES" in binding.tg_status_string(st)
+    torch.cuda.synchronize()
+    assert bool((c == 7.0).all()), "a rejected call must launch nothing"

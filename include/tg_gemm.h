@@ -252,10 +252,11 @@ tg_status_t tg_gemm_host(const void *A_host, const void *B_host, const void *bia
  * tg_gemm_launch_count -- number of kernels tg_gemm would launch for these
  * arguments (host only, no device call; the configuration choice assumes
  * 148 SMs): 0 for an empty problem, 1 for the GEMM kernel (or the K == 0
- * kernel), plus one repacking kernel for each of A and B whose base address
- * or row pitch is not a multiple of 16 bytes when the chosen configuration
- * loads with TMA (a table row choosing a plain-loader configuration repacks
- * nothing).  Returns -1 if the arguments would be rejected.
+ * kernel), plus one repacking kernel (it repacks both operands) when the
+ * base address or row pitch of A or B is not a multiple of 16 bytes and the
+ * chosen configuration loads with TMA (a table row choosing a plain-loader
+ * configuration repacks nothing).  Returns -1 if the arguments would be
+ * rejected.
  */
 int tg_gemm_launch_count(const void *A, const void *B, const void *bias, const void *C,
                          int64_t M, int64_t N, int64_t K, int epilogue);

@@ -438,14 +438,32 @@ tg_status_t launch_k0(const void *bias, void *C, int64_t M, int64_t N, int epilo
     return cudaGetLastError() == cudaSuccess ? TG_OK : TG_ERR_LAUNCH;
 }
 
-tg_status_t launch_pack(const void *src, int64_t rows, int64_t cols, void *dst, int64_t ld_dst,
-                        cudaStream_t stream, int num_sms)
+// A repacking job for an operand of rows x cols at src into dst with pitch
+// ld_dst, or an empty job when src is null.
+tg::PackJob pack_job(const void *src, int64_t rows, int64_t cols, void *dst, int64_t ld_dst)
 {
-    const int64_t groups = rows * (ld_dst / 8);
-    if (groups == 0) return TG_OK;
-    const int grid = static_cast<int>(std::min<int64_t>(ceil_div(groups, 256), 16ll * num_sms));
-    tg::pack_pad_kernel<<<grid, 256, 0, stream>>>(static_cast<const __half *>(src), rows, cols,
-                                                  static_cast<__half *>(dst), ld_dst);
+    tg::PackJob j;
+    j.src = static_cast<const __half *>(src);
+    j.dst = static_cast<__half *>(dst);
+    j.cols = cols;
+    j.ld_dst = ld_dst;
+    j.groups_per_row = static_cast<uint32_t>(ld_dst / 8);
+    j.groups = src ? static_cast<uint64_t>(rows) * static_cast<uint64_t>(ld_dst / 8) : 0;
+    return j;
+}
+
+// One launch repacks both operands (either job may be empty).  At most four
+// 256-thread blocks per SM, so that the GEMM's CTA (launched with
+// programmatic serialisation) fits beside them and runs its prologue while
+// they finish.
+tg_status_t launch_pack2(const tg::PackJob &a, const tg::PackJob &b, cudaStream_t stream,
+                         int num_sms)
+{
+    const uint64_t total = a.groups + b.groups;
+    if (total == 0) return TG_OK;
+    const int grid = static_cast<int>(
+        std::min<uint64_t>((total + 255) / 256, 4ull * static_cast<uint64_t>(num_sms)));
+    tg::pack_pad2_kernel<<<grid, 256, 0, stream>>>(a, b);
     return cudaGetLastError() == cudaSuccess ? TG_OK : TG_ERR_LAUNCH;
 }
 
@@ -576,15 +594,11 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
             cudaGetLastError();
             return TG_ERR_OOM;
         }
-        if (!a_direct) {
-            st = launch_pack(A, M, K, tmp, lda, stream, dev->num_sms);
-            Aeff = tmp;
-        }
-        if (st == TG_OK && !b_direct) {
-            void *bdst = static_cast<char *>(tmp) + a_pad;
-            st = launch_pack(B, K, N, bdst, ldb, stream, dev->num_sms);
-            Beff = bdst;
-        }
+        void *bdst = static_cast<char *>(tmp) + a_pad;
+        if (!a_direct) Aeff = tmp;
+        if (!b_direct) Beff = bdst;
+        st = launch_pack2(pack_job(a_direct ? nullptr : A, M, K, tmp, lda),
+                          pack_job(b_direct ? nullptr : B, K, N, bdst, ldb), stream, dev->num_sms);
         if (st != TG_OK) {
             cudaFreeAsync(tmp, stream);
             return st;
@@ -814,7 +828,7 @@ int tg_gemm_launch_count(const void *A, const void *B, const void *bias, const v
     const bool b_direct = aligned(B, 16) && (N % 8 == 0);
     const Choice c = choose_config(M, N, K, epilogue, 148);
     if (kConfigs[c.config].info.loader == tg::kLoadPlain) return 1;
-    return 1 + (a_direct ? 0 : 1) + (b_direct ? 0 : 1);
+    return 1 + ((a_direct && b_direct) ? 0 : 1);
 }
 
 tg_status_t tg_gemm_check_error(void *stream)
@@ -947,18 +961,12 @@ tg_status_t gemm_noalloc_impl(const void *A, const void *B, const void *bias, vo
     const int cfg_id =
         choose_config(M, N, K, epilogue, dev->num_sms, false).config;
     const KernelConfig &cfg = kConfigs[cfg_id];
-    const void *Aeff = A, *Beff = B;
-    if (!a_direct) {
-        st = launch_pack(A, M, K, dev->scratch, lda, stream, dev->num_sms);
-        if (st != TG_OK) return st;
-        Aeff = dev->scratch;
-    }
-    if (!b_direct) {
-        unsigned char *bdst = dev->scratch + a_pad;
-        st = launch_pack(B, K, N, bdst, ldb, stream, dev->num_sms);
-        if (st != TG_OK) return st;
-        Beff = bdst;
-    }
+    const void *Aeff = a_direct ? A : dev->scratch;
+    const void *Beff = b_direct ? B : dev->scratch + a_pad;
+    st = launch_pack2(pack_job(a_direct ? nullptr : A, M, K, dev->scratch, lda),
+                      pack_job(b_direct ? nullptr : B, K, N, dev->scratch + a_pad, ldb), stream,
+                      dev->num_sms);
+    if (st != TG_OK) return st;
 
     // stream-K needs a workspace; this entry point allocates nothing
     return launch_staged(cfg, Aeff, lda, Beff, ldb, bias, C, M, N, K, epilogue, TG_SPLIT_TILES,

@@ -3,9 +3,10 @@
 //   gemm_persistent_kernel  C = g(A.B + beta) with tcgen05 MMA into TMEM,
 //                           TMA-fed swizzled shared-memory ring, one CTA per
 //                           SM walking an L2-grouped tile order.
-//   pack_pad_kernel         copies a row-major fp16 matrix into a copy whose
-//                           row pitch is a multiple of 8 elements (16 bytes),
-//                           zero-padded, so TMA can address it.
+//   pack_pad2_kernel        copies up to two row-major fp16 matrices into
+//                           copies whose row pitch is a multiple of 8
+//                           elements (16 bytes), zero-padded, so TMA can
+//                           address them.
 //   k0_epilogue_kernel      the K == 0 case: C = g(beta).
 //
 // Operation: "Designing High-Performance GPU Kernels with TileLang"
@@ -195,7 +196,7 @@ struct KernelShape {
     static constexpr int kStageBytes = kABytes + kBChunks * kBChunkBytes;
     static constexpr uint32_t kTxBytes = kCG * kStageBytes;      // both CTAs land on the leader
     static constexpr int kRingBytes = STAGES * kStageBytes;
-    static constexpr int kStagingBytes = STORE != kStoreVec ? EPI_WARPS * 2 * kStoreBoxBytes : 0;
+    static constexpr int kStagingBytes = STORE == kStoreTma ? EPI_WARPS * 2 * kStoreBoxBytes : 0;
     // Stream-K fold: once a head segment's MMAs are done the operand ring is
     // idle, and each epilogue warp streams the contributors' partials into its
     // own kFoldSlots slots of kFoldSlotBytes (one warp's 32 rows x 32 columns
@@ -292,31 +293,94 @@ __device__ __forceinline__ float exp2_approx(float x)
     return r;
 }
 
+// Two fp32 values in one 64-bit register, for the packed f32x2 arithmetic of
+// sm_100 (two lanes' worth of FMA per instruction).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void f2_unpack(uint64_t r, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 // GELU(v) = v * Phi(v), Phi the standard normal CDF.  With a = |v| and the
-// tail T = Phi(-a) = erfc(a / sqrt 2) / 2, GELU(v) = max(v, 0) - a * T for
-// either sign of v.  T uses the Chebyshev-type form of erfc of Numerical
-// Recipes (2nd ed., section 6.2), erfc(z) = t exp(-z^2 + P(t)), t = 1/(1+z/2),
-// written with a base-2 exponent and the 1/2 folded into the polynomial:
-//   T = t * 2^(-a^2 log2(e)/2 + Q(t)),  t = 1 / (1 + a / (2 sqrt 2)),
-// Q of degree 6 fitted by csrc/fit_erfc.py (our coefficients; max error of Q
-// 8.2e-6 in log2 units on z in [0, 9]).  In fp32 with the approximate
-// reciprocal and exponential the relative error of GELU stays near 1e-5 for
-// |v| <= 8.5 (fp16's half-ulp is 2.4e-4) and the tail keeps full relative
-// accuracy.  14 instructions per element, two of them MUFU.
+// lower tail T = Phi(-a), GELU(v) = max(v, 0) - a * T for either sign of v.
+// log2 T(a) is the Gaussian exponent -a^2 log2(e) / 2 plus a smooth
+// remainder (the logarithm of the Mills ratio, falling like -log2(a) for
+// large a), which a degree-7 polynomial Q in x = min(a, 6) / 3 - 1 fits to
+// 5e-6 in log2 units (csrc/fit_gelu.py; our coefficients):
+//   T = 2^( -a^2 log2(e) / 2 + Q(x) ).
+// Past a = 6 the Gaussian term alone puts a * T below half the smallest fp16
+// subnormal, so the clamp of x changes no fp16 result.  One exponential, no
+// division; in fp32 the result is within one fp16 ulp of the correctly
+// rounded GELU for every fp16 input (0.4% of them off by one).
+constexpr float kGeluQ0 = -3.040808201e+00f, kGeluQ1 = -1.225311518e+00f,
+                kGeluQ2 = 4.581521749e-01f, kGeluQ3 = -2.038841099e-01f,
+                kGeluQ4 = 9.168275446e-02f, kGeluQ5 = -4.095217586e-02f,
+                kGeluQ6 = 1.681641303e-02f, kGeluQ7 = -4.013689235e-03f;
+constexpr float kGeluAMax = 6.0f;
+constexpr float kHalfLog2e = 0.721347520444481703f;   // log2(e) / 2
+
 __device__ __forceinline__ float gelu_erf(float v)
 {
     const float a = fabsf(v);
-    const float t = rcp_approx(fmaf(a, 0.353553390593273762f, 1.0f));
-    float p = -3.214579429e-02f;
-    p = fmaf(p, t, 4.489113895e-01f);
-    p = fmaf(p, t, -1.198654278e+00f);
-    p = fmaf(p, t, 8.162180034e-01f);
-    p = fmaf(p, t, 3.145696625e-01f);
-    p = fmaf(p, t, 1.479150420e+00f);
-    p = fmaf(p, t, -2.828041197e+00f);
-    const float x = fmaf(-a * 0.721347520444481703f, a, p);   // log2(e)/2 = 0.7213...
-    const float tail = t * exp2_approx(x);
-    return fmaf(-a, tail, fmaxf(v, 0.0f));
+    const float x = fmaf(fminf(a, kGeluAMax), 2.0f / kGeluAMax, -1.0f);
+    float p = fmaf(kGeluQ7, x, kGeluQ6);
+    p = fmaf(p, x, kGeluQ5);
+    p = fmaf(p, x, kGeluQ4);
+    p = fmaf(p, x, kGeluQ3);
+    p = fmaf(p, x, kGeluQ2);
+    p = fmaf(p, x, kGeluQ1);
+    p = fmaf(p, x, kGeluQ0);
+    const float t = exp2_approx(fmaf(-a * kHalfLog2e, a, p));
+    return fmaf(-a, t, fmaxf(v, 0.0f));
+}
+
+// gelu_erf of two values at once: the polynomial and the exponent run as
+// packed f32x2 operations (the same roundings as the scalar form).
+__device__ __forceinline__ void gelu_erf2(float &v0, float &v1)
+{
+    const float a0 = fabsf(v0), a1 = fabsf(v1);
+    const uint64_t a = f2_pack(a0, a1);
+    const uint64_t x = f2_fma(f2_pack(fminf(a0, kGeluAMax), fminf(a1, kGeluAMax)),
+                              f2_pack(2.0f / kGeluAMax, 2.0f / kGeluAMax), f2_pack(-1.0f, -1.0f));
+    uint64_t p = f2_fma(f2_pack(kGeluQ7, kGeluQ7), x, f2_pack(kGeluQ6, kGeluQ6));
+    p = f2_fma(p, x, f2_pack(kGeluQ5, kGeluQ5));
+    p = f2_fma(p, x, f2_pack(kGeluQ4, kGeluQ4));
+    p = f2_fma(p, x, f2_pack(kGeluQ3, kGeluQ3));
+    p = f2_fma(p, x, f2_pack(kGeluQ2, kGeluQ2));
+    p = f2_fma(p, x, f2_pack(kGeluQ1, kGeluQ1));
+    p = f2_fma(p, x, f2_pack(kGeluQ0, kGeluQ0));
+    const uint64_t e = f2_fma(f2_mul(a, f2_pack(-kHalfLog2e, -kHalfLog2e)), a, p);
+    float e0, e1;
+    f2_unpack(e, e0, e1);
+    v0 = fmaf(-a0, exp2_approx(e0), fmaxf(v0, 0.0f));
+    v1 = fmaf(-a1, exp2_approx(e1), fmaxf(v1, 0.0f));
 }
 
 // tanh approximation of GELU (Hendrycks & Gimpel, "Gaussian Error Linear
@@ -396,7 +460,12 @@ __device__ __forceinline__ uint4 epilogue8(const uint32_t *r, const float (&b)[8
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
         float lo, hi;
-        if constexpr (EPI == kEpiBiasSoftmax) {
+        if constexpr (EPI == kEpiBiasGelu) {
+            const uint64_t v = f2_add(f2_pack(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])),
+                                      f2_pack(b[2 * e], b[2 * e + 1]));
+            f2_unpack(v, lo, hi);
+            gelu_erf2(lo, hi);
+        } else if constexpr (EPI == kEpiBiasSoftmax) {
             lo = exp2_approx((__uint_as_float(r[2 * e]) + b[2 * e] - sm_max) * kLog2e) * sm_scale;
             hi = exp2_approx((__uint_as_float(r[2 * e + 1]) + b[2 * e + 1] - sm_max) * kLog2e) *
                  sm_scale;
@@ -408,6 +477,84 @@ __device__ __forceinline__ uint4 epilogue8(const uint32_t *r, const float (&b)[8
     }
     return u;
 }
+
+// The low (hi == 0) or high half of a packed pair of fp16 values.
+__device__ __forceinline__ __half half_of(uint32_t w, int hi)
+{
+    return __ushort_as_half(static_cast<unsigned short>(hi ? w >> 16 : w & 0xFFFFu));
+}
+
+// Stores of one thread's row of C when C's rows are not 16-byte aligned.
+// The thread holds 32 consecutive columns of its row at a time (a chunk) and
+// walks a run of chunks from `run` on.  The run starts h elements past a
+// 16-byte boundary (h in 1..8; 8 means aligned).  Each chunk's 16 packed
+// words, after the previous chunk's last four (the carry), are shifted by
+// h elements in registers, so that the chunk's data leaves as four aligned
+// 16-byte vectors: the first one ends the previous chunk (columns
+// [-h, 8 - h) of this chunk), the next three hold [8j - h, 8j - h + 8).  Only
+// the run's first 8 - h and last h columns go out as 2-byte stores.  The
+// shift is the same code for every lane: h differs from row to row, so it
+// selects its source words with selects and byte permutes, not branches.
+struct RowShifter {
+    int h;              // 1..8
+    uint32_t qsel;      // (8 - h) / 2: whole words to skip
+    uint32_t perm;      // byte-permute selector: no shift, or 2 bytes (h odd)
+    uint32_t carry[4];  // columns 24..31 of the previous chunk
+    int64_t last_col0;  // first column of the last full chunk stored (-1: none)
+
+    __device__ __forceinline__ explicit RowShifter(const __half *run)
+    {
+        const int r = static_cast<int>((reinterpret_cast<uintptr_t>(run) >> 1) & 7u);
+        h = r == 0 ? 8 : r;
+        qsel = static_cast<uint32_t>(8 - h) >> 1;
+        perm = (h & 1) ? 0x5432u : 0x3210u;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) carry[i] = 0u;
+        last_col0 = -1;
+    }
+
+    // o[k] = bytes [2 (8 - h) + 4k, + 4) of x (x holds at least NW + 4 words).
+    template <int NW>
+    __device__ __forceinline__ void shift(const uint32_t *x, uint32_t (&o)[NW]) const
+    {
+        uint32_t y[NW + 1];
+#pragma unroll
+        for (int k = 0; k <= NW; ++k) {
+            const uint32_t a = (qsel & 1u) ? x[k + 1] : x[k];
+            const uint32_t b = (qsel & 1u) ? x[k + 3] : x[k + 2];
+            y[k] = (qsel & 2u) ? b : a;
+        }
+#pragma unroll
+        for (int k = 0; k < NW; ++k) o[k] = __byte_perm(y[k], y[k + 1], perm);
+    }
+
+    // The run's first chunk: of its first shifted vector (columns [-h, 8 - h)),
+    // only columns [0, 8 - h) are this run's.  c0 points at the chunk's column 0.
+    __device__ __forceinline__ void store_head(__half *c0, const uint32_t (&o)[16]) const
+    {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (i >= h) c0[i - h] = half_of(o[i >> 1], i & 1);
+    }
+
+    // Columns [32 - h, 32) of the last full chunk stored, if any.
+    __device__ __forceinline__ void flush_tail(__half *crow)
+    {
+        if (last_col0 < 0) return;
+        uint32_t x[8] = {carry[0], carry[1], carry[2], carry[3], 0u, 0u, 0u, 0u};
+        uint32_t o[4];
+        shift<4>(x, o);
+        __half *dst = crow + last_col0 + kStoreCols - h;
+        if (h == 8) {
+            *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 7; ++i)
+                if (i < h) dst[i] = half_of(o[i >> 1], i & 1);
+        }
+        last_col0 = -1;
+    }
+};
 
 // ---------------------------------------------------------------------------
 // Persistent warp-specialised GEMM.
@@ -647,6 +794,12 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
             // (leading), 8-k-row groups 1024 B apart (stride).
             const uint64_t b_desc0 =
                 smem_desc_sw128(smem_base + S::kABytes, S::kBChunkBytes, 1024);
+            // The last k-block may hold fewer than BK valid K columns (the rest
+            // of its stage is TMA zero fill): only its first ceil(rem / 16)
+            // MMAs contribute, so the rest are not issued.
+            const int last_kb = p.num_k_blocks - 1;
+            const int last_kk = static_cast<int>(
+                (p.K - static_cast<int64_t>(last_kb) * BK + kUmmaK - 1) / kUmmaK);
             WorkIter work(p, unit, num_units);
             int tile, k0, k1, role;
             while (work.next(tile, k0, k1, role)) {
@@ -668,8 +821,10 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                     ready = mbar_test_wait(&full_bar[next_stage], next_phase);
                     const uint64_t stage_off =
                         static_cast<uint64_t>((stage * S::kStageBytes) >> 4);
+                    const int kk_end = kb == last_kb ? last_kk : BK / kUmmaK;
 #pragma unroll
                     for (int kk = 0; kk < BK / kUmmaK; ++kk) {
+                        if (kk >= kk_end) break;
                         // K step: for A, the next 32 B inside a 128-B swizzle row,
                         // moving to the next 128 x 64 box every 4 steps; for B,
                         // the next 16 k-rows (2 KiB).
@@ -979,30 +1134,17 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                 sm_max = run_max;
                 sm_scale = rcp_approx(run_sum);
             }
-#pragma unroll 1
-            for (int c = chunk0; c < chunk0 + S::kChunksPerWarp; ++c) {
+            RowShifter rs(crow + static_cast<int64_t>(nt) * BN + chunk0 * kStoreCols);
+            // One chunk: epilogue on its 32 accumulator columns r, then its
+            // store (into staging box `buf` for the TMA store mode).
+            auto emit = [&](int c, const uint32_t (&r)[32], const uint4 (&bq)[4], uint32_t buf) {
                 const int64_t col0 = static_cast<int64_t>(nt) * BN + c * kStoreCols;
-                // warp-uniform: the chunk lies entirely past N, or all 32 rows past M
-                if (col0 >= p.N || row0 >= p.M) break;
-                uint4 bias_cur[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) bias_cur[q] = bias_next[q];
-                if (c + 1 < chunk0 + S::kChunksPerWarp)
-                    fetch_bias32<EPI>(p.bias, col0 + kStoreCols, p.N, bias_vec, bias_next);
-                uint32_t r[32];
-                load_acc_chunk(c, r);
                 if constexpr (STORE == kStoreTma) {
-                    // Stage a 32 x 32 fp16 box (64-B rows, 64-B swizzle) and let
-                    // one lane store it with TMA; two boxes alternate.
-                    const uint32_t buf = staging + (store_count & 1u) * kStoreBoxBytes;
-                    if (store_count >= 2) {
-                        if (lane == 0) bulk_wait_group_read<1>();
-                        __syncwarp();
-                    }
+                    // a 32 x 32 fp16 box: 64-B rows, 64-B swizzle
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         float b[8];
-                        unpack_bias8(bias_cur[q], b);
+                        unpack_bias8(bq[q], b);
                         const uint4 u = epilogue8<EPI>(r + q * 8, b, sm_max, sm_scale);
                         const uint32_t phys = static_cast<uint32_t>(q) ^ ((lane >> 1) & 3u);
                         const uint32_t addr = buf + lane * 64u + phys * 16u;
@@ -1010,66 +1152,119 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                                      "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w)
                                      : "memory");
                     }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&tmC, buf, static_cast<int32_t>(col0),
-                                     static_cast<int32_t>(row0));
-                        bulk_commit_group();
-                    }
-                    ++store_count;
                 } else if constexpr (STORE == kStoreVec) {
                     if (row_ok) {
                         const bool full = col0 + kStoreCols <= p.N;
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             float b[8];
-                            unpack_bias8(bias_cur[q], b);
+                            unpack_bias8(bq[q], b);
                             const uint4 u = epilogue8<EPI>(r + q * 8, b, sm_max, sm_scale);
                             if (full) {
                                 *reinterpret_cast<uint4 *>(crow + col0 + q * 8) = u;
                             } else {
-                                const __half *h = reinterpret_cast<const __half *>(&u);
+                                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
                                 for (int e = 0; e < 8; ++e)
-                                    if (col0 + q * 8 + e < p.N) crow[col0 + q * 8 + e] = h[e];
+                                    if (col0 + q * 8 + e < p.N)
+                                        crow[col0 + q * 8 + e] = half_of(w[e >> 1], e & 1);
                             }
                         }
                     }
                 } else {
-                    // Any pitch: stage the 32 x 32 box (same swizzled layout as
-                    // the TMA path), then write it back one row per
-                    // instruction, lane l storing column l (64 contiguous bytes).
-                    const uint32_t buf = staging + (store_count & 1u) * kStoreBoxBytes;
+                    // Any pitch: each lane writes its own row (see RowShifter).
+                    uint32_t x[20];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) x[i] = rs.carry[i];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         float b[8];
-                        unpack_bias8(bias_cur[q], b);
+                        unpack_bias8(bq[q], b);
                         const uint4 u = epilogue8<EPI>(r + q * 8, b, sm_max, sm_scale);
-                        const uint32_t phys = static_cast<uint32_t>(q) ^ ((lane >> 1) & 3u);
-                        const uint32_t addr = buf + lane * 64u + phys * 16u;
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                                     "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w)
-                                     : "memory");
+                        x[4 + 4 * q] = u.x;
+                        x[5 + 4 * q] = u.y;
+                        x[6 + 4 * q] = u.z;
+                        x[7 + 4 * q] = u.w;
                     }
-                    __syncwarp();
-                    const bool col_ok = col0 + lane < p.N;
-                    const uint32_t q = static_cast<uint32_t>(lane) >> 3;
-                    const uint32_t within = (static_cast<uint32_t>(lane) & 7u) * 2u;
-#pragma unroll 4
-                    for (int rr = 0; rr < 32; ++rr) {
-                        const uint32_t phys = q ^ ((static_cast<uint32_t>(rr) >> 1) & 3u);
-                        unsigned short h;
-                        asm volatile("ld.shared.u16 %0, [%1];"
-                                     : "=h"(h)
-                                     : "r"(buf + static_cast<uint32_t>(rr) * 64u + phys * 16u +
-                                           within));
-                        if (col_ok && row0 + rr < p.M)
-                            p.C[(row0 + rr) * p.ldc + col0 + lane] = __ushort_as_half(h);
+                    if (row_ok) {
+                        if (col0 + kStoreCols <= p.N) {
+                            uint32_t o[16];
+                            rs.shift<16>(x, o);
+                            if (c == chunk0)
+                                rs.store_head(crow + col0, o);
+                            else
+                                *reinterpret_cast<uint4 *>(crow + col0 - rs.h) =
+                                    make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+                            for (int j = 1; j < 4; ++j)
+                                *reinterpret_cast<uint4 *>(crow + col0 + 8 * j - rs.h) =
+                                    make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+                            rs.last_col0 = col0;
+                        } else {
+                            // the chunk that crosses N: the previous chunk's
+                            // tail, then element stores up to N
+                            rs.flush_tail(crow);
+#pragma unroll
+                            for (int e = 0; e < kStoreCols; ++e)
+                                if (col0 + e < p.N) crow[col0 + e] = half_of(x[4 + (e >> 1)], e & 1);
+                        }
                     }
-                    __syncwarp();
-                    ++store_count;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) rs.carry[i] = x[16 + i];
                 }
+            };
+            // Chunks go two at a time: both TMEM loads are in flight behind one
+            // wait, and the two chunks' arithmetic interleaves.
+#pragma unroll 1
+            for (int c = chunk0; c < chunk_end; c += 2) {
+                const bool two = c + 1 < chunk_end;
+                const int64_t col0 = static_cast<int64_t>(nt) * BN + c * kStoreCols;
+                uint32_t ra[32], rb[32];
+                if (folding) {
+                    load_acc_chunk(c, ra);
+                    if (two) load_acc_chunk(c + 1, rb);
+                } else {
+                    tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * kStoreCols), ra);
+                    if (two)
+                        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((c + 1) * kStoreCols), rb);
+                }
+                uint4 ba[4], bb[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) ba[q] = bias_next[q];
+                if (two) fetch_bias32<EPI>(p.bias, col0 + kStoreCols, p.N, bias_vec, bb);
+                if (c + 2 < chunk_end)
+                    fetch_bias32<EPI>(p.bias, col0 + 2 * kStoreCols, p.N, bias_vec, bias_next);
+                if (!folding) {
+                    tmem_wait_ld_dep(ra);
+                    if (two) tmem_wait_ld_dep(rb);
+                }
+                if constexpr (STORE == kStoreTma) {
+                    // the previous pair's boxes must have been read out
+                    if (store_count > 0) {
+                        if (lane == 0) bulk_wait_group_read<0>();
+                        __syncwarp();
+                    }
+                    emit(c, ra, ba, staging);
+                    if (two) emit(c + 1, rb, bb, staging + kStoreBoxBytes);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmC, staging, static_cast<int32_t>(col0),
+                                     static_cast<int32_t>(row0));
+                        if (two)
+                            tma_store_2d(&tmC, staging + kStoreBoxBytes,
+                                         static_cast<int32_t>(col0 + kStoreCols),
+                                         static_cast<int32_t>(row0));
+                        bulk_commit_group();
+                    }
+                    ++store_count;
+                } else {
+                    emit(c, ra, ba, 0u);
+                    if (two) emit(c + 1, rb, bb, 0u);
+                }
+            }
+            if constexpr (STORE == kStoreScalar) {
+                if (row_ok) rs.flush_tail(crow);
             }
             fold_drain();
             // All TMEM reads of this accumulator are complete (wait::ld above).
@@ -1086,7 +1281,7 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                 acc_phase ^= 1u;
             }
         }
-        if (STORE == kStoreTma && lane == 0) bulk_wait_group_all();
+        if (STORE == kStoreTma && lane == 0) bulk_wait_group_read<0>();
         __syncwarp();
     }
 
@@ -1104,24 +1299,110 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
 }
 
 // ---------------------------------------------------------------------------
-// dst[r, c] = src[r, c] for c < cols, 0 for cols <= c < ld_dst.  Each thread
-// writes one 16-byte group of 8 destination elements; ld_dst % 8 == 0.
-__global__ void pack_pad_kernel(const __half *__restrict__ src, int64_t rows, int64_t cols,
-                                __half *__restrict__ dst, int64_t ld_dst)
+// Repacking of operands whose base or row pitch is not a multiple of 16 bytes:
+// dst[r, c] = src[r, c] for c < cols, 0 for cols <= c < ld_dst (ld_dst % 8 == 0,
+// dst 16-byte aligned).  Both operands of a call are repacked by one launch.
+struct PackJob {
+    const __half *src;
+    __half *dst;
+    int64_t cols, ld_dst;
+    uint32_t groups_per_row;   // ld_dst / 8: 16-byte groups of one dst row
+    uint64_t groups;           // rows * groups_per_row (0: nothing to do)
+};
+
+// The eight fp16 values src[0 .. 8), of which the first `valid` (1..8) are
+// in bounds and the rest read as zero, from any 2-byte aligned address: the
+// aligned 16-byte vector holding src[0], the next one only when valid
+// elements reach into it, and a byte permutation that shifts the 16 bytes
+// into place.  A 16-byte aligned vector that holds a valid element never
+// crosses a page, so reading its other bytes is always safe; they are
+// discarded.
+__device__ __forceinline__ uint4 load8_any16(const __half *src, int valid)
 {
-    const int64_t groups_per_row = ld_dst / 8;
-    const int64_t total = rows * groups_per_row;
-    for (int64_t g = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; g < total;
-         g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t r = g / groups_per_row;
-        const int64_t c0 = (g - r * groups_per_row) * 8;
-        const __half *s = src + r * cols;
-        uint4 u;
-        __half *h = reinterpret_cast<__half *>(&u);
+    const uintptr_t addr = reinterpret_cast<uintptr_t>(src);
+    const uint32_t b = static_cast<uint32_t>(addr & 15u);   // even
+    const uint4 *v = reinterpret_cast<const uint4 *>(addr - b);
+    const uint4 lo = __ldg(v);
+    const uint4 hi = (b != 0 && b + 2u * static_cast<uint32_t>(valid) > 16u)
+                         ? __ldg(v + 1)
+                         : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t W[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    // output word j = bytes [b + 4j, b + 4j + 4) of lo:hi
+    const uint32_t sel = (b & 2u) ? 0x5432u : 0x3210u;
+    uint32_t w[4];
+    switch (b >> 2) {
+    case 0:
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-            h[e] = (c0 + e < cols) ? s[c0 + e] : __ushort_as_half(static_cast<unsigned short>(0));
-        *reinterpret_cast<uint4 *>(dst + r * ld_dst + c0) = u;
+        for (int j = 0; j < 4; ++j) w[j] = __byte_perm(W[j], W[j + 1], sel);
+        break;
+    case 1:
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[j] = __byte_perm(W[j + 1], W[j + 2], sel);
+        break;
+    case 2:
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[j] = __byte_perm(W[j + 2], W[j + 3], sel);
+        break;
+    default:
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[j] = __byte_perm(W[j + 3], W[j + 4], sel);
+        break;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (2 * i >= valid)
+            w[i] = 0u;
+        else if (2 * i + 1 >= valid)
+            w[i] &= 0xFFFFu;
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Destination group g of a job: its source elements (nullptr when the group
+// lies wholly in the zero padding), how many of its 8 are valid, and where
+// it goes.
+__device__ __forceinline__ void pack_group(const PackJob &j, uint64_t g, const __half *&src,
+                                           int &valid, uint4 *&dst)
+{
+    uint64_t r;
+    uint32_t cg;
+    if (g < (1ull << 32)) {
+        const uint32_t g32 = static_cast<uint32_t>(g);
+        r = g32 / j.groups_per_row;
+        cg = g32 - static_cast<uint32_t>(r) * j.groups_per_row;
+    } else {
+        r = g / j.groups_per_row;
+        cg = static_cast<uint32_t>(g - r * j.groups_per_row);
+    }
+    const int64_t c0 = static_cast<int64_t>(cg) * 8;
+    const int64_t left = j.cols - c0;
+    valid = left <= 0 ? 0 : (left < 8 ? static_cast<int>(left) : 8);
+    src = valid > 0 ? j.src + static_cast<int64_t>(r) * j.cols + c0 : nullptr;
+    dst = reinterpret_cast<uint4 *>(j.dst + static_cast<int64_t>(r) * j.ld_dst + c0);
+}
+
+// Grid-stride over the 16-byte destination groups of job a, then of job b,
+// two groups per thread and step (their loads in flight together).
+// Consecutive threads take consecutive groups of a row: coalesced reads and
+// writes.  The launch lets the dependent GEMM start its prologue at once (it
+// still waits for this grid's completion before reading the copies).
+__global__ void __launch_bounds__(256) pack_pad2_kernel(const PackJob a, const PackJob b)
+{
+    grid_launch_dependents();
+    const uint64_t total = a.groups + b.groups;
+    const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+    for (uint64_t g = blockIdx.x * static_cast<uint64_t>(blockDim.x) + threadIdx.x; g < total;
+         g += 2 * stride) {
+        const uint64_t g2 = g + stride;
+        const __half *s0, *s1 = nullptr;
+        int v0, v1 = 0;
+        uint4 *d0, *d1 = nullptr;
+        pack_group(g < a.groups ? a : b, g < a.groups ? g : g - a.groups, s0, v0, d0);
+        if (g2 < total) pack_group(g2 < a.groups ? a : b, g2 < a.groups ? g2 : g2 - a.groups, s1, v1, d1);
+        const uint4 u0 = s0 ? load8_any16(s0, v0) : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 u1 = s1 ? load8_any16(s1, v1) : make_uint4(0u, 0u, 0u, 0u);
+        *d0 = u0;
+        if (d1) *d1 = u1;
     }
 }
 

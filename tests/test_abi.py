@@ -186,6 +186,20 @@ def test_valid_call_without_a_device_reports_unsupported_device():
     assert binding.tg_gemm_check_error(None) == binding.TG_ERR_UNSUPPORTED_DEVICE
 
 
+def test_launch_count_is_host_only():
+    """One GEMM kernel, plus one repacking kernel for both operands when
+    either row pitch or base is not a multiple of 16 bytes."""
+    f = binding.tg_gemm_launch_count
+    assert f(0x1000, 0x100000, None, 0x1000000, 256, 256, 256, NONE) == 1
+    assert f(0x1000, 0x100000, None, 0x1000000, 256, 256, 250, NONE) == 2   # K % 8
+    assert f(0x1000, 0x100000, None, 0x1000000, 256, 250, 256, NONE) == 2   # N % 8
+    assert f(0x1000, 0x100000, None, 0x1000000, 300, 1537, 2050, GELU) == 2  # both
+    assert f(0x1002, 0x100000, None, 0x1000000, 256, 256, 256, NONE) == 2   # A's base
+    assert f(0x1000, 0x100000, None, 0x1000000, 256, 256, 0, GELU) == 1     # K == 0
+    assert f(0x1000, 0x100000, None, 0x1000000, 0, 256, 256, NONE) == 0
+    assert f(0x1001, 0x100000, None, 0x1000000, 256, 256, 256, NONE) == -1  # misaligned
+
+
 def test_binding_checks_tensor_arguments():
     a = torch.zeros(4, 4, dtype=torch.float32)
     with pytest.raises(TypeError):

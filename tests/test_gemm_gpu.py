@@ -206,6 +206,58 @@ def test_misaligned_operands(config_id):
     assert_close(c.cpu(), run_oracle(A, B, bias, GELU), f"misaligned views, config {config_id}")
 
 
+REPACK_CASES = [((200, 131, 133), 1, 0), ((200, 131, 133), 0, 1), ((64, 70, 262), 2, 3),
+                ((257, 1537, 2050), 3, 5), ((130, 9, 17), 7, 6), ((96, 250, 90), 4, 4),
+                ((33, 1, 7), 5, 2)]
+
+
+@pytest.mark.parametrize("shape,off_a,off_b", REPACK_CASES,
+                         ids=[f"{'x'.join(map(str, c[0]))}-a{c[1]}-b{c[2]}" for c in REPACK_CASES])
+def test_repacked_operands_bit_exact(shape, off_a, off_b):
+    """Operands whose base sits off_* elements past a 16-byte boundary and
+    whose pitches are not multiples of 8 elements go through the repacking
+    kernel (every load alignment and every count of valid elements in a
+    row's last 16-byte group); integer-valued inputs make the exact result
+    an fp16 value, so C must match it bit for bit."""
+    M, N, K = shape
+    dev = torch.device("cuda:0")
+    A, B, _ = wl.integer_inputs(M, N, K, seed=450 + M + off_a, lo=-1, hi=1)
+    a_buf = torch.zeros(M * K + 8, dtype=torch.float16, device=dev)
+    b_buf = torch.zeros(K * N + 8, dtype=torch.float16, device=dev)
+    a = a_buf[off_a:off_a + M * K].view(M, K)
+    b = b_buf[off_b:off_b + K * N].view(K, N)
+    a.copy_(A.to(dev))
+    b.copy_(B.to(dev))
+    c = binding.gemm(a, b, None, epilogue=NONE)
+    torch.cuda.synchronize()
+    assert binding.tg_gemm_check_error(torch.cuda.current_stream().cuda_stream) == binding.TG_OK
+    assert_bits_equal(c.cpu(), oracle.gemm_int_exact(wl.to_bits(A), wl.to_bits(B)),
+                      f"repacked {M}x{N}x{K} offsets {off_a},{off_b}")
+
+
+@pytest.mark.parametrize("config_id", [c for c in CONFIG_IDS if binding.tg_config_info(c)["loader"] == 0])
+@pytest.mark.parametrize("off_c", [1, 2, 3, 4, 5, 6, 7])
+def test_unaligned_c_rows_bit_exact(config_id, off_c):
+    """C whose base sits off_c elements past a 16-byte boundary, with an odd
+    N (every row starts at a different alignment): each row leaves through
+    aligned 16-byte vector stores plus element stores at the ends of each
+    warp's run of columns.  Integer-valued inputs make the exact result an
+    fp16 value, so every element must match bit for bit, and nothing before
+    or after C may be written."""
+    M, N, K = 130, 333, 72
+    dev = torch.device("cuda:0")
+    A, B, _ = wl.integer_inputs(M, N, K, seed=470 + off_c, lo=-2, hi=2)
+    c_buf = torch.full((M * N + 16,), -7.0, dtype=torch.float16, device=dev)
+    c = c_buf[off_c:off_c + M * N].view(M, N)
+    binding.gemm(A.to(dev), B.to(dev), None, epilogue=NONE, out=c, config_id=config_id)
+    torch.cuda.synchronize()
+    assert binding.tg_gemm_check_error(torch.cuda.current_stream().cuda_stream) == binding.TG_OK
+    assert_bits_equal(c.cpu(), oracle.gemm_int_exact(wl.to_bits(A), wl.to_bits(B)),
+                      f"unaligned C offset {off_c} config {config_id}")
+    guard = torch.cat([c_buf[:off_c], c_buf[off_c + M * N:]]).cpu()
+    assert bool((guard == -7.0).all()), "wrote outside C"
+
+
 # ---------------------------------------------------------------- the workloads
 
 @pytest.mark.parametrize("name", ["gemm_256", "gemm_2048", "fused_2048", "ragged_fused",

@@ -196,7 +196,7 @@ struct KernelShape {
     static constexpr int kStageBytes = kABytes + kBChunks * kBChunkBytes;
     static constexpr uint32_t kTxBytes = kCG * kStageBytes;      // both CTAs land on the leader
     static constexpr int kRingBytes = STAGES * kStageBytes;
-    static constexpr int kStagingBytes = STORE == kStoreTma ? EPI_WARPS * 2 * kStoreBoxBytes : 0;
+    static constexpr int kStagingBytes = STORE != kStoreVec ? EPI_WARPS * 2 * kStoreBoxBytes : 0;
     // Stream-K fold: once a head segment's MMAs are done the operand ring is
     // idle, and each epilogue warp streams the contributors' partials into its
     // own kFoldSlots slots of kFoldSlotBytes (one warp's 32 rows x 32 columns
@@ -483,78 +483,6 @@ __device__ __forceinline__ __half half_of(uint32_t w, int hi)
 {
     return __ushort_as_half(static_cast<unsigned short>(hi ? w >> 16 : w & 0xFFFFu));
 }
-
-// Stores of one thread's row of C when C's rows are not 16-byte aligned.
-// The thread holds 32 consecutive columns of its row at a time (a chunk) and
-// walks a run of chunks from `run` on.  The run starts h elements past a
-// 16-byte boundary (h in 1..8; 8 means aligned).  Each chunk's 16 packed
-// words, after the previous chunk's last four (the carry), are shifted by
-// h elements in registers, so that the chunk's data leaves as four aligned
-// 16-byte vectors: the first one ends the previous chunk (columns
-// [-h, 8 - h) of this chunk), the next three hold [8j - h, 8j - h + 8).  Only
-// the run's first 8 - h and last h columns go out as 2-byte stores.  The
-// shift is the same code for every lane: h differs from row to row, so it
-// selects its source words with selects and byte permutes, not branches.
-struct RowShifter {
-    int h;              // 1..8
-    uint32_t qsel;      // (8 - h) / 2: whole words to skip
-    uint32_t perm;      // byte-permute selector: no shift, or 2 bytes (h odd)
-    uint32_t carry[4];  // columns 24..31 of the previous chunk
-    int64_t last_col0;  // first column of the last full chunk stored (-1: none)
-
-    __device__ __forceinline__ explicit RowShifter(const __half *run)
-    {
-        const int r = static_cast<int>((reinterpret_cast<uintptr_t>(run) >> 1) & 7u);
-        h = r == 0 ? 8 : r;
-        qsel = static_cast<uint32_t>(8 - h) >> 1;
-        perm = (h & 1) ? 0x5432u : 0x3210u;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) carry[i] = 0u;
-        last_col0 = -1;
-    }
-
-    // o[k] = bytes [2 (8 - h) + 4k, + 4) of x (x holds at least NW + 4 words).
-    template <int NW>
-    __device__ __forceinline__ void shift(const uint32_t *x, uint32_t (&o)[NW]) const
-    {
-        uint32_t y[NW + 1];
-#pragma unroll
-        for (int k = 0; k <= NW; ++k) {
-            const uint32_t a = (qsel & 1u) ? x[k + 1] : x[k];
-            const uint32_t b = (qsel & 1u) ? x[k + 3] : x[k + 2];
-            y[k] = (qsel & 2u) ? b : a;
-        }
-#pragma unroll
-        for (int k = 0; k < NW; ++k) o[k] = __byte_perm(y[k], y[k + 1], perm);
-    }
-
-    // The run's first chunk: of its first shifted vector (columns [-h, 8 - h)),
-    // only columns [0, 8 - h) are this run's.  c0 points at the chunk's column 0.
-    __device__ __forceinline__ void store_head(__half *c0, const uint32_t (&o)[16]) const
-    {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (i >= h) c0[i - h] = half_of(o[i >> 1], i & 1);
-    }
-
-    // Columns [32 - h, 32) of the last full chunk stored, if any.
-    __device__ __forceinline__ void flush_tail(__half *crow)
-    {
-        if (last_col0 < 0) return;
-        uint32_t x[8] = {carry[0], carry[1], carry[2], carry[3], 0u, 0u, 0u, 0u};
-        uint32_t o[4];
-        shift<4>(x, o);
-        __half *dst = crow + last_col0 + kStoreCols - h;
-        if (h == 8) {
-            *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 7; ++i)
-                if (i < h) dst[i] = half_of(o[i >> 1], i & 1);
-        }
-        last_col0 = -1;
-    }
-};
 
 // ---------------------------------------------------------------------------
 // Persistent warp-specialised GEMM.
@@ -1134,31 +1062,23 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                 sm_max = run_max;
                 sm_scale = rcp_approx(run_sum);
             }
-            RowShifter rs(crow + static_cast<int64_t>(nt) * BN + chunk0 * kStoreCols);
-            // One chunk: epilogue on its 32 accumulator columns r, then its
-            // store (into staging box `buf` for the TMA store mode).
-            auto emit = [&](int c, const uint32_t (&r)[32], const uint4 (&bq)[4], uint32_t buf) {
+            // One chunk: epilogue on its 32 accumulator columns r, then its store.
+            // The bias of chunk c is in bias_next on entry; the next chunk's is
+            // fetched here.
+            auto emit = [&](int c, const uint32_t (&r)[32]) {
                 const int64_t col0 = static_cast<int64_t>(nt) * BN + c * kStoreCols;
-                if constexpr (STORE == kStoreTma) {
-                    // a 32 x 32 fp16 box: 64-B rows, 64-B swizzle
+                uint4 bias_cur[4];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        float b[8];
-                        unpack_bias8(bq[q], b);
-                        const uint4 u = epilogue8<EPI>(r + q * 8, b, sm_max, sm_scale);
-                        const uint32_t phys = static_cast<uint32_t>(q) ^ ((lane >> 1) & 3u);
-                        const uint32_t addr = buf + lane * 64u + phys * 16u;
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                                     "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w)
-                                     : "memory");
-                    }
-                } else if constexpr (STORE == kStoreVec) {
+                for (int q = 0; q < 4; ++q) bias_cur[q] = bias_next[q];
+                if (c + 1 < chunk_end)
+                    fetch_bias32<EPI>(p.bias, col0 + kStoreCols, p.N, bias_vec, bias_next);
+                if constexpr (STORE == kStoreVec) {
                     if (row_ok) {
                         const bool full = col0 + kStoreCols <= p.N;
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             float b[8];
-                            unpack_bias8(bq[q], b);
+                            unpack_bias8(bias_cur[q], b);
                             const uint4 u = epilogue8<EPI>(r + q * 8, b, sm_max, sm_scale);
                             if (full) {
                                 *reinterpret_cast<uint4 *>(crow + col0 + q * 8) = u;
@@ -1171,100 +1091,81 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                             }
                         }
                     }
-                } else {
-                    // Any pitch: each lane writes its own row (see RowShifter).
-                    uint32_t x[20];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) x[i] = rs.carry[i];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        float b[8];
-                        unpack_bias8(bq[q], b);
-                        const uint4 u = epilogue8<EPI>(r + q * 8, b, sm_max, sm_scale);
-                        x[4 + 4 * q] = u.x;
-                        x[5 + 4 * q] = u.y;
-                        x[6 + 4 * q] = u.z;
-                        x[7 + 4 * q] = u.w;
-                    }
-                    if (row_ok) {
-                        if (col0 + kStoreCols <= p.N) {
-                            uint32_t o[16];
-                            rs.shift<16>(x, o);
-                            if (c == chunk0)
-                                rs.store_head(crow + col0, o);
-                            else
-                                *reinterpret_cast<uint4 *>(crow + col0 - rs.h) =
-                                    make_uint4(o[0], o[1], o[2], o[3]);
-#pragma unroll
-                            for (int j = 1; j < 4; ++j)
-                                *reinterpret_cast<uint4 *>(crow + col0 + 8 * j - rs.h) =
-                                    make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-                            rs.last_col0 = col0;
-                        } else {
-                            // the chunk that crosses N: the previous chunk's
-                            // tail, then element stores up to N
-                            rs.flush_tail(crow);
-#pragma unroll
-                            for (int e = 0; e < kStoreCols; ++e)
-                                if (col0 + e < p.N) crow[col0 + e] = half_of(x[4 + (e >> 1)], e & 1);
-                        }
-                    }
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) rs.carry[i] = x[16 + i];
+                    return;
                 }
-            };
-            // Chunks go two at a time: both TMEM loads are in flight behind one
-            // wait, and the two chunks' arithmetic interleaves.
-#pragma unroll 1
-            for (int c = chunk0; c < chunk_end; c += 2) {
-                const bool two = c + 1 < chunk_end;
-                const int64_t col0 = static_cast<int64_t>(nt) * BN + c * kStoreCols;
-                uint32_t ra[32], rb[32];
-                if (folding) {
-                    load_acc_chunk(c, ra);
-                    if (two) load_acc_chunk(c + 1, rb);
-                } else {
-                    tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * kStoreCols), ra);
-                    if (two)
-                        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((c + 1) * kStoreCols), rb);
+                // TMA stores and element stores both stage a 32 x 32 fp16 box
+                // (64-B rows, 64-B swizzle) first; two boxes alternate.
+                const uint32_t slot = store_count & 1u;
+                const uint32_t buf = staging + slot * kStoreBoxBytes;
+                if (STORE == kStoreTma && store_count >= 2) {
+                    if (lane == 0) bulk_wait_group_read<1>();
+                    __syncwarp();
                 }
-                uint4 ba[4], bb[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) ba[q] = bias_next[q];
-                if (two) fetch_bias32<EPI>(p.bias, col0 + kStoreCols, p.N, bias_vec, bb);
-                if (c + 2 < chunk_end)
-                    fetch_bias32<EPI>(p.bias, col0 + 2 * kStoreCols, p.N, bias_vec, bias_next);
-                if (!folding) {
-                    tmem_wait_ld_dep(ra);
-                    if (two) tmem_wait_ld_dep(rb);
+                for (int q = 0; q < 4; ++q) {
+                    float b[8];
+                    unpack_bias8(bias_cur[q], b);
+                    const uint4 u = epilogue8<EPI>(r + q * 8, b, sm_max, sm_scale);
+                    const uint32_t phys = static_cast<uint32_t>(q) ^ ((lane >> 1) & 3u);
+                    const uint32_t addr = buf + lane * 64u + phys * 16u;
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                                 "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w)
+                                 : "memory");
                 }
                 if constexpr (STORE == kStoreTma) {
-                    // the previous pair's boxes must have been read out
-                    if (store_count > 0) {
-                        if (lane == 0) bulk_wait_group_read<0>();
-                        __syncwarp();
-                    }
-                    emit(c, ra, ba, staging);
-                    if (two) emit(c + 1, rb, bb, staging + kStoreBoxBytes);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_2d(&tmC, staging, static_cast<int32_t>(col0),
+                        tma_store_2d(&tmC, buf, static_cast<int32_t>(col0),
                                      static_cast<int32_t>(row0));
-                        if (two)
-                            tma_store_2d(&tmC, staging + kStoreBoxBytes,
-                                         static_cast<int32_t>(col0 + kStoreCols),
-                                         static_cast<int32_t>(row0));
                         bulk_commit_group();
                     }
-                    ++store_count;
                 } else {
-                    emit(c, ra, ba, 0u);
-                    if (two) emit(c + 1, rb, bb, 0u);
+                    // Any pitch: the box goes back out one row per instruction,
+                    // lane l storing column l (64 contiguous bytes of a row per
+                    // store: on rows that are not 16-byte aligned this beats
+                    // per-row vector stores, which touch 32 rows per store).
+                    __syncwarp();
+                    const bool col_ok = col0 + lane < p.N;
+                    const unsigned short *box = reinterpret_cast<const unsigned short *>(
+                        smem + S::kStagingOffset + (warp * 2 + slot) * kStoreBoxBytes);
+                    const uint32_t q = static_cast<uint32_t>(lane) >> 3;
+                    const uint32_t within = static_cast<uint32_t>(lane) & 7u;
+                    __half *dst = p.C + row0 * p.ldc + col0 + lane;
+                    const int rows = p.M - row0 < 32 ? static_cast<int>(p.M - row0) : 32;
+#pragma unroll 8
+                    for (int rr = 0; rr < 32; ++rr) {
+                        const uint32_t phys = q ^ ((static_cast<uint32_t>(rr) >> 1) & 3u);
+                        const unsigned short h = box[rr * 32 + phys * 8 + within];
+                        if (col_ok && rr < rows) dst[rr * p.ldc] = __ushort_as_half(h);
+                    }
+                    __syncwarp();
                 }
-            }
-            if constexpr (STORE == kStoreScalar) {
-                if (row_ok) rs.flush_tail(crow);
+                ++store_count;
+            };
+            // Each chunk's TMEM load is issued one chunk ahead, so that it is in
+            // flight while the previous chunk is converted and stored.  (Heads
+            // of a stream-K split load through the fold, one chunk at a time.)
+            uint32_t ra[32], rb[32];
+            if (!folding && chunk_end > chunk0)
+                tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(chunk0 * kStoreCols), ra);
+#pragma unroll 1
+            for (int c = chunk0; c < chunk_end; c += 2) {
+                if (folding)
+                    load_acc_chunk(c, ra);
+                else
+                    tmem_wait_ld_dep(ra);
+                if (!folding && c + 1 < chunk_end)
+                    tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((c + 1) * kStoreCols), rb);
+                emit(c, ra);
+                if (c + 1 >= chunk_end) break;
+                if (folding)
+                    load_acc_chunk(c + 1, rb);
+                else
+                    tmem_wait_ld_dep(rb);
+                if (!folding && c + 2 < chunk_end)
+                    tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((c + 2) * kStoreCols), ra);
+                emit(c + 1, rb);
             }
             fold_drain();
             // All TMEM reads of this accumulator are complete (wait::ld above).

@@ -487,11 +487,12 @@ def run_e2e(torch, binding, w, s, args, dev, stream, barrier, max_over_ranks, wo
             "path": "tg_gemm_host: pinned host -> device copies, GEMM in row panels, copy back, overlapped on three streams"}
 
 
-def finish(torch, binding, dist, w, s, args, rank, world, dev, step_ms, value, kernel_ms,
-           region_ms, launches_per_step, clocks, also, e2e):
-    peaks, peak_src = load_peaks()
-    peak_kind = "burst" if region_ms < 1000.0 else "sustained"
-    if s["big"] or w.flops / max(w.algorithmic_bytes, 1) > 100:
+def roofline(w, kernel_ms, peaks, peak_src, peak_kind, kcfg, big):
+    """Roofline entry of one GEMM workload: TFLOP/s against the tensor peak for
+    shapes above about 100 flop per byte (or larger than L2), else GB/s of
+    algorithmic bytes against the copy bandwidth; DRAM traffic per launch from
+    the committed ncu summary of the same kernel and configuration, if any."""
+    if big or w.flops / max(w.algorithmic_bytes, 1) > 100:
         tens = peaks["bf16_tflops"] if peak_kind == "burst" else peaks["bf16_tflops_sustained"]
         achieved = w.flops / (kernel_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": tens, "unit": "TFLOP/s",
@@ -501,13 +502,28 @@ def finish(torch, binding, dist, w, s, args, rank, world, dev, step_ms, value, k
         achieved = w.algorithmic_bytes / (kernel_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peak_src} copy bandwidth"}
-    kcfg = binding.tg_config_info(args.config) if args.config >= 0 else \
-        binding.tg_gemm_select_config(w.M, w.N, w.K, w.epilogue,
-                                      torch.cuda.get_device_properties(dev).multi_processor_count)
-    traffic = profiled_traffic(w.name, kcfg)
-    roof["traffic"] = traffic
+    roof["traffic"] = profiled_traffic(w.name, kcfg)
     roof["algorithmic_per_launch"] = {"flops": w.flops, "bytes": w.algorithmic_bytes}
     roof["kernel_ms"] = kernel_ms
+    return roof
+
+
+def finish(torch, binding, dist, w, s, args, rank, world, dev, step_ms, value, kernel_ms,
+           region_ms, launches_per_step, clocks, also, e2e):
+    from tensor_core_gemm_fp16_b200 import workloads as wl
+    peaks, peak_src = load_peaks()
+    peak_kind = "burst" if region_ms < 1000.0 else "sustained"
+    num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    kcfg = binding.tg_config_info(args.config) if args.config >= 0 else \
+        binding.tg_gemm_select_config(w.M, w.N, w.K, w.epilogue, num_sms)
+    roof = roofline(w, kernel_ms, peaks, peak_src, peak_kind, kcfg, s["big"])
+    for entry in also:
+        if entry["kind"] != "gemm":
+            continue
+        w2 = wl.WORKLOADS[entry["workload"]]
+        entry["roofline"] = roofline(
+            w2, entry["ms_per_step"], peaks, peak_src, "burst",
+            binding.tg_gemm_select_config(w2.M, w2.N, w2.K, w2.epilogue, num_sms), False)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -452,17 +452,16 @@ tg::PackJob pack_job(const void *src, int64_t rows, int64_t cols, void *dst, int
     return j;
 }
 
-// One launch repacks both operands (either job may be empty).  At most four
-// 256-thread blocks per SM, so that the GEMM's CTA (launched with
-// programmatic serialisation) fits beside them and runs its prologue while
-// they finish.
+// One launch repacks both operands (either job may be empty): up to eight
+// 256-thread blocks per SM, each thread kPackGroups 16-byte groups per step.
 tg_status_t launch_pack2(const tg::PackJob &a, const tg::PackJob &b, cudaStream_t stream,
                          int num_sms)
 {
     const uint64_t total = a.groups + b.groups;
     if (total == 0) return TG_OK;
-    const int grid = static_cast<int>(
-        std::min<uint64_t>((total + 255) / 256, 4ull * static_cast<uint64_t>(num_sms)));
+    const uint64_t per_block = 256ull * tg::kPackGroups;
+    const int grid = static_cast<int>(std::min<uint64_t>((total + per_block - 1) / per_block,
+                                                         8ull * static_cast<uint64_t>(num_sms)));
     tg::pack_pad2_kernel<<<grid, 256, 0, stream>>>(a, b);
     return cudaGetLastError() == cudaSuccess ? TG_OK : TG_ERR_LAUNCH;
 }

@@ -205,6 +205,8 @@ struct KernelShape {
         kRingBytes / (EPI_WARPS * kFoldSlotBytes) < 8 ? kRingBytes / (EPI_WARPS * kFoldSlotBytes)
                                                       : 8;
     static_assert(kFoldSlots >= 2, "the operand ring must hold two fold slots per epilogue warp");
+    static_assert(kRingBytes >= EPI_WARPS * (BN / kStoreCols / (EPI_WARPS / 4)) * kStoreBoxBytes,
+                  "the operand ring must hold a staging box per chunk of the last tile");
     // barriers: full[STAGES], empty[STAGES], tmem_full[2], tmem_empty[2], drain,
     // fold[EPI_WARPS][kFoldSlots]
     static constexpr int kFoldBar = 2 * STAGES + 5;
@@ -722,12 +724,6 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
             // (leading), 8-k-row groups 1024 B apart (stride).
             const uint64_t b_desc0 =
                 smem_desc_sw128(smem_base + S::kABytes, S::kBChunkBytes, 1024);
-            // The last k-block may hold fewer than BK valid K columns (the rest
-            // of its stage is TMA zero fill): only its first ceil(rem / 16)
-            // MMAs contribute, so the rest are not issued.
-            const int last_kb = p.num_k_blocks - 1;
-            const int last_kk = static_cast<int>(
-                (p.K - static_cast<int64_t>(last_kb) * BK + kUmmaK - 1) / kUmmaK);
             WorkIter work(p, unit, num_units);
             int tile, k0, k1, role;
             while (work.next(tile, k0, k1, role)) {
@@ -749,10 +745,8 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                     ready = mbar_test_wait(&full_bar[next_stage], next_phase);
                     const uint64_t stage_off =
                         static_cast<uint64_t>((stage * S::kStageBytes) >> 4);
-                    const int kk_end = kb == last_kb ? last_kk : BK / kUmmaK;
 #pragma unroll
                     for (int kk = 0; kk < BK / kUmmaK; ++kk) {
-                        if (kk >= kk_end) break;
                         // K step: for A, the next 32 B inside a 128-B swizzle row,
                         // moving to the next 128 x 64 box every 4 steps; for B,
                         // the next 16 k-rows (2 KiB).
@@ -1062,6 +1056,10 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                 sm_max = run_max;
                 sm_scale = rcp_approx(run_sum);
             }
+            // The CTA's last tile (no segment follows): every MMA of the CTA (of
+            // both CTAs of a pair) is complete once its accumulator is, so the
+            // operand ring is idle -- unless a stream-K fold copies into it.
+            const bool ring_staging = work.cur >= work.end && !folding;
             // One chunk: epilogue on its 32 accumulator columns r, then its store.
             // The bias of chunk c is in bias_next on entry; the next chunk's is
             // fetched here.
@@ -1094,10 +1092,18 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                     return;
                 }
                 // TMA stores and element stores both stage a 32 x 32 fp16 box
-                // (64-B rows, 64-B swizzle) first; two boxes alternate.
+                // (64-B rows, 64-B swizzle) first; two boxes alternate.  On the
+                // CTA's last tile the TMA path gives every chunk a box of its own
+                // in the idle operand ring, so no store waits for an earlier one
+                // to be read out.
                 const uint32_t slot = store_count & 1u;
-                const uint32_t buf = staging + slot * kStoreBoxBytes;
-                if (STORE == kStoreTma && store_count >= 2) {
+                const bool own_box = STORE == kStoreTma && ring_staging;
+                const uint32_t buf =
+                    own_box ? smem_base + static_cast<uint32_t>(
+                                              (warp * S::kChunksPerWarp + (c - chunk0)) *
+                                              kStoreBoxBytes)
+                            : staging + slot * kStoreBoxBytes;
+                if (STORE == kStoreTma && !own_box && store_count >= 2) {
                     if (lane == 0) bulk_wait_group_read<1>();
                     __syncwarp();
                 }
@@ -1283,27 +1289,40 @@ __device__ __forceinline__ void pack_group(const PackJob &j, uint64_t g, const _
 }
 
 // Grid-stride over the 16-byte destination groups of job a, then of job b,
-// two groups per thread and step (their loads in flight together).
-// Consecutive threads take consecutive groups of a row: coalesced reads and
-// writes.  The launch lets the dependent GEMM start its prologue at once (it
-// still waits for this grid's completion before reading the copies).
+// kPackGroups groups per thread and step with all their loads in flight
+// together (the copy is bound by DRAM latency otherwise).  Consecutive threads
+// take consecutive groups of a row: coalesced reads and writes.  The launch
+// lets the dependent GEMM start as soon as SMs free up (it still waits for
+// this grid's completion before reading the copies).
+constexpr int kPackGroups = 4;
+
 __global__ void __launch_bounds__(256) pack_pad2_kernel(const PackJob a, const PackJob b)
 {
     grid_launch_dependents();
     const uint64_t total = a.groups + b.groups;
     const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
-    for (uint64_t g = blockIdx.x * static_cast<uint64_t>(blockDim.x) + threadIdx.x; g < total;
-         g += 2 * stride) {
-        const uint64_t g2 = g + stride;
-        const __half *s0, *s1 = nullptr;
-        int v0, v1 = 0;
-        uint4 *d0, *d1 = nullptr;
-        pack_group(g < a.groups ? a : b, g < a.groups ? g : g - a.groups, s0, v0, d0);
-        if (g2 < total) pack_group(g2 < a.groups ? a : b, g2 < a.groups ? g2 : g2 - a.groups, s1, v1, d1);
-        const uint4 u0 = s0 ? load8_any16(s0, v0) : make_uint4(0u, 0u, 0u, 0u);
-        const uint4 u1 = s1 ? load8_any16(s1, v1) : make_uint4(0u, 0u, 0u, 0u);
-        *d0 = u0;
-        if (d1) *d1 = u1;
+    for (uint64_t g0 = blockIdx.x * static_cast<uint64_t>(blockDim.x) + threadIdx.x; g0 < total;
+         g0 += kPackGroups * stride) {
+        const __half *src[kPackGroups];
+        int valid[kPackGroups];
+        uint4 *dst[kPackGroups];
+#pragma unroll
+        for (int i = 0; i < kPackGroups; ++i) {
+            const uint64_t g = g0 + i * stride;
+            src[i] = nullptr;
+            dst[i] = nullptr;
+            valid[i] = 0;
+            if (g < total)
+                pack_group(g < a.groups ? a : b, g < a.groups ? g : g - a.groups, src[i], valid[i],
+                           dst[i]);
+        }
+        uint4 u[kPackGroups];
+#pragma unroll
+        for (int i = 0; i < kPackGroups; ++i)
+            u[i] = src[i] ? load8_any16(src[i], valid[i]) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int i = 0; i < kPackGroups; ++i)
+            if (dst[i]) *dst[i] = u[i];
     }
 }
 

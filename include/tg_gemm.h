@@ -122,6 +122,13 @@ typedef enum {
  * `stream` is capturing a CUDA graph, stream-K is never used: its flags carry
  * a per-call epoch, which every replay of the graph would repeat.  Such calls
  * run whole tiles (an explicit TG_SPLIT_STREAM_K returns TG_ERR_INVALID_ARG).
+ *
+ * Thin N remainder: when N = q * BN + r with 0 < r <= 16 (BN the tile width
+ * of the chosen configuration) and the last, nearly empty column of tiles
+ * would add a whole wave to a whole-tile launch, the tensor-core kernel
+ * covers the first q * BN columns and a second kernel computes the last r
+ * columns on the CUDA cores (fp32 sums of the same fp16 products, the same
+ * epilogue), launched before it on `stream`.  Not for the row softmax.
  */
 tg_status_t tg_gemm(const void *A, const void *B, const void *bias, void *C,
                     int64_t M, int64_t N, int64_t K, int epilogue, void *stream);
@@ -255,8 +262,10 @@ tg_status_t tg_gemm_host(const void *A_host, const void *B_host, const void *bia
  * kernel), plus one repacking kernel (it repacks both operands) when the
  * base address or row pitch of A or B is not a multiple of 16 bytes and the
  * chosen configuration loads with TMA (a table row choosing a plain-loader
- * configuration repacks nothing).  Returns -1 if the arguments would be
- * rejected.
+ * configuration repacks nothing), plus one kernel for the last N mod 256 (at
+ * most 16) columns when that thin remainder would otherwise cost the
+ * tensor-core kernel a whole extra wave of tiles (see tg_gemm).  Returns -1
+ * if the arguments would be rejected.
  */
 int tg_gemm_launch_count(const void *A, const void *B, const void *bias, const void *C,
                          int64_t M, int64_t N, int64_t K, int epilogue);

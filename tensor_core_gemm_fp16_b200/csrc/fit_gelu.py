@@ -2,19 +2,21 @@
 
 GELU(v) = v * Phi(v) = max(v, 0) - a * T(a) for a = |v|, where
 T(a) = Phi(-a) is the standard normal lower tail.  Its logarithm is the
-Gaussian exponent plus a slowly varying remainder,
+Gaussian exponent plus a slowly varying remainder (the logarithm of the
+Mills ratio, which falls like -log2(a sqrt(2 pi)) for large a):
 
-    log2 T(a) = -a^2 * log2(e) / 2 + R(a),   R(a) = log2(Phi(-a)) + a^2 log2(e) / 2,
+    log2 T(a) = -a^2 * log2(e) / 2 + R(a),   R(0) = -1,
 
-and R is smooth on [0, A_MAX] (R(0) = -1; for large a it falls like
--log2(a sqrt(2 pi)), the Mills-ratio asymptote).  The kernel evaluates
+a smooth function on [0, A_MAX] that a polynomial fits closely.  The kernel
+evaluates
 
-    T(a) = 2^( -a^2 * log2(e)/2 + Q(x) ),   x = min(a, A_MAX) / (A_MAX/2) - 1,
+    T(a) = 2^( Q(x) ),   x = min(a, A_MAX) / (A_MAX/2) - 1,   and T = 0 for a > A_MAX,
 
-with Q a polynomial of degree DEGREE in x in [-1, 1] (Horner form), so one
-GELU costs one base-2 exponential and no division.  Past A_MAX the Gaussian
-term alone drives T below 1e-9: a * T then rounds to zero in fp16 whatever
-Q is, so clamping x there loses nothing.
+with Q a polynomial of degree DEGREE in x in [-1, 1] (Horner form) fitted to
+the whole log2 T, Gaussian term included, so one GELU costs one base-2
+exponential, no division and DEGREE + 2 fused multiply-adds.  Past A_MAX,
+a * T is below half the smallest fp16 subnormal for every fp16 input, so
+setting T to zero there changes no fp16 result (at most the sign of a zero).
 
 Q is fitted here by iteratively reweighted least squares (towards minimax) on
 a in [0, A_MAX] against scipy's log_ndtr; the coefficients are our own.  The
@@ -36,7 +38,7 @@ LOG2E = 1.0 / np.log(2.0)
 
 
 def target(a):
-    return log_ndtr(-a) * LOG2E + a * a * LOG2E / 2.0
+    return log_ndtr(-a) * LOG2E
 
 
 def fit(degree=DEGREE, iters=40):
@@ -75,9 +77,8 @@ def gelu_kernel_model(v, q):
     p = np.full_like(x, q[-1])
     for c in q[-2::-1]:
         p = fma32(p, x, c)
-    nac = (-a * f32(LOG2E / 2.0)).astype(np.float32)
-    e = fma32(nac, a, p)
-    t = np.exp2(e.astype(np.float64)).astype(np.float32)
+    t = np.exp2(p.astype(np.float64)).astype(np.float32)
+    t = np.where(a > f32(A_MAX), f32(0.0), t)
     return fma32(-a, t, np.maximum(v, f32(0.0)))
 
 
@@ -102,7 +103,7 @@ if __name__ == "__main__":
     q, max_err = fit(deg)
     for i, c in enumerate(q):
         print(f"q{i} = {c:.9e}f")
-    print(f"max |Q_fit - R| on [0, {A_MAX}] = {max_err:.3e} (log2 units)")
+    print(f"max |Q_fit - log2 T| on [0, {A_MAX}] = {max_err:.3e} (log2 units)")
     worst, frac = ulp_check(q)
     print(f"fp32 model vs correctly rounded GELU on fp16 [-16, 16]: max {worst} ulp, "
           f"{100 * frac:.3f}% of inputs off by one")

@@ -438,6 +438,115 @@ tg_status_t launch_k0(const void *bias, void *C, int64_t M, int64_t N, int epilo
     return cudaGetLastError() == cudaSuccess ? TG_OK : TG_ERR_LAUNCH;
 }
 
+// Thin N remainder: when N = q * BN + r with 0 < r <= kTailMaxCols and the
+// last, nearly empty column of tiles would cost the persistent GEMM a whole
+// extra wave, the GEMM covers the first q * BN columns and tail_cols_kernel
+// the last r on the CUDA cores (one pass over A, read from L2 right after the
+// repack or the GEMM's own loads).  Whole-tile TMA configurations only (the
+// tail kernel reads A with 16-byte loads), not the row softmax (it needs whole
+// rows), and only while B's r columns fit the tail kernel's shared memory.
+constexpr int kTailMaxCols = 16;
+constexpr int64_t kTailSmemBytes = 64 * 1024;
+
+int tail_round(int r) { return r <= 1 ? 1 : r <= 2 ? 2 : r <= 4 ? 4 : r <= 8 ? 8 : 16; }
+
+int tail_cols(const tg_config_t &ci, int64_t M, int64_t N, int64_t K, int epilogue, int split,
+              int num_sms)
+{
+    if (split == TG_SPLIT_STREAM_K || epilogue == TG_EPILOGUE_BIAS_SOFTMAX ||
+        ci.loader != tg::kLoadTma)
+        return 0;
+    const int64_t r = N % ci.block_n;
+    if (r == 0 || r > kTailMaxCols || N < ci.block_n) return 0;
+    if (K * tail_round(static_cast<int>(r)) * 2 > kTailSmemBytes) return 0;
+    const int64_t units = ci.cta_pair ? num_sms / 2 : num_sms;
+    const int64_t m_tiles = ceil_div(M, ci.block_m);
+    const int64_t waves_all = ceil_div(m_tiles * ceil_div(N, ci.block_n), units);
+    const int64_t waves_main = ceil_div(m_tiles * (N / ci.block_n), units);
+    return waves_main < waves_all ? static_cast<int>(r) : 0;
+}
+
+template <int EPI>
+cudaError_t launch_tail_epi(const __half *A, int64_t lda, const __half *B, int64_t ldb,
+                            const __half *bias, __half *C, int64_t ldc, int64_t M, int64_t K,
+                            int64_t n0, int r, int grid, cudaStream_t stream)
+{
+    const int rt = tail_round(r);
+    const size_t smem = static_cast<size_t>(K) * rt * 2;
+    switch (rt) {
+    case 1: tg::tail_cols_kernel<EPI, 1><<<grid, 256, smem, stream>>>(A, lda, B, ldb, bias, C, ldc, M, K, n0, r); break;
+    case 2: tg::tail_cols_kernel<EPI, 2><<<grid, 256, smem, stream>>>(A, lda, B, ldb, bias, C, ldc, M, K, n0, r); break;
+    case 4: tg::tail_cols_kernel<EPI, 4><<<grid, 256, smem, stream>>>(A, lda, B, ldb, bias, C, ldc, M, K, n0, r); break;
+    case 8: tg::tail_cols_kernel<EPI, 8><<<grid, 256, smem, stream>>>(A, lda, B, ldb, bias, C, ldc, M, K, n0, r); break;
+    default: tg::tail_cols_kernel<EPI, 16><<<grid, 256, smem, stream>>>(A, lda, B, ldb, bias, C, ldc, M, K, n0, r); break;
+    }
+    return cudaGetLastError();
+}
+
+// Opt every tail kernel into up to kTailSmemBytes of dynamic shared memory
+// (once per device).
+template <int EPI>
+cudaError_t tail_smem_attrs()
+{
+    cudaError_t e = cudaSuccess;
+    auto set = [&](auto kern) {
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(kTailSmemBytes));
+    };
+    set(tg::tail_cols_kernel<EPI, 1>);
+    set(tg::tail_cols_kernel<EPI, 2>);
+    set(tg::tail_cols_kernel<EPI, 4>);
+    set(tg::tail_cols_kernel<EPI, 8>);
+    set(tg::tail_cols_kernel<EPI, 16>);
+    return e;
+}
+
+tg_status_t launch_tail(const void *A, int64_t lda, const void *B, int64_t ldb, const void *bias,
+                        void *C, int64_t ldc, int64_t M, int64_t K, int64_t n0, int r,
+                        int epilogue, int num_sms, cudaStream_t stream)
+{
+    static std::atomic<uint64_t> attr_set{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_CUDA;
+    }
+    const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+    if (!bit || !(attr_set.load() & bit)) {
+        const cudaError_t e = tail_smem_attrs<0>() == cudaSuccess && tail_smem_attrs<1>() == cudaSuccess &&
+                                      tail_smem_attrs<2>() == cudaSuccess && tail_smem_attrs<3>() == cudaSuccess
+                                  ? cudaSuccess
+                                  : cudaErrorInvalidValue;
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return TG_ERR_CUDA;
+        }
+        attr_set.fetch_or(bit);
+    }
+    // one row per warp at a time, and enough warps that every row's loads go
+    // out at once on moderate M
+    const int grid = static_cast<int>(std::min<int64_t>(ceil_div(M, 8), 32ll * num_sms));
+    const __half *a = static_cast<const __half *>(A);
+    const __half *b = static_cast<const __half *>(B);
+    const __half *bb = static_cast<const __half *>(bias);
+    __half *c = static_cast<__half *>(C);
+    cudaError_t e;
+    if (epilogue == TG_EPILOGUE_NONE)
+        e = launch_tail_epi<0>(a, lda, b, ldb, bb, c, ldc, M, K, n0, r, grid, stream);
+    else if (epilogue == TG_EPILOGUE_BIAS)
+        e = launch_tail_epi<1>(a, lda, b, ldb, bb, c, ldc, M, K, n0, r, grid, stream);
+    else if (epilogue == TG_EPILOGUE_BIAS_GELU)
+        e = launch_tail_epi<2>(a, lda, b, ldb, bb, c, ldc, M, K, n0, r, grid, stream);
+    else
+        e = launch_tail_epi<3>(a, lda, b, ldb, bb, c, ldc, M, K, n0, r, grid, stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_LAUNCH;
+    }
+    return TG_OK;
+}
+
 // A repacking job for an operand of rows x cols at src into dst with pitch
 // ld_dst, or an empty job when src is null.
 tg::PackJob pack_job(const void *src, int64_t rows, int64_t cols, void *dst, int64_t ld_dst)
@@ -480,16 +589,24 @@ tg_status_t launch_staged(const KernelConfig &cfg, const void *Aeff, int64_t lda
     const bool plain = cfg.info.loader == tg::kLoadPlain;
     const bool c_rows16 = aligned(C, 16) && (N % 8 == 0);
     const int store = c_rows16 ? cfg.store_pref : tg::kStoreScalar;
+    // The GEMM covers columns [0, n_main); a thin remainder goes to the tail kernel.
+    const int tail = tail_cols(cfg.info, M, N, K, epilogue, split, num_sms);
+    const int64_t n_main = N - tail;
+    if (tail > 0) {
+        const tg_status_t st = launch_tail(Aeff, lda, Beff, ldb, bias, C, N, M, K, n_main, tail,
+                                           epilogue, num_sms, stream);
+        if (st != TG_OK) return st;
+    }
     CUtensorMap ta, tb, tc;
     std::memset(&ta, 0, sizeof(ta));
     std::memset(&tb, 0, sizeof(tb));
     std::memset(&tc, 0, sizeof(tc));
     if ((!plain && (!encode_2d(&ta, Aeff, K, M, 2 * lda, tg::kAtomK, tg::kBlockM,
                                CU_TENSOR_MAP_SWIZZLE_128B) ||
-                    !encode_2d(&tb, Beff, N, K, 2 * ldb, tg::kBChunkN, cfg.info.block_k,
+                    !encode_2d(&tb, Beff, n_main, K, 2 * ldb, tg::kBChunkN, cfg.info.block_k,
                                CU_TENSOR_MAP_SWIZZLE_128B))) ||
         (store == tg::kStoreTma &&
-         !encode_2d(&tc, C, N, M, 2 * N, tg::kStoreCols, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
+         !encode_2d(&tc, C, n_main, M, 2 * N, tg::kStoreCols, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
         return TG_ERR_CUDA;
 
     tg::GemmParams p;
@@ -500,11 +617,11 @@ tg_status_t launch_staged(const KernelConfig &cfg, const void *Aeff, int64_t lda
     p.bias = static_cast<const __half *>(bias);
     p.C = static_cast<__half *>(C);
     p.M = M;
-    p.N = N;
+    p.N = n_main;
     p.K = K;
     p.ldc = N;
     p.num_m_tiles = static_cast<int>(ceil_div(M, cfg.info.block_m));
-    p.num_n_tiles = static_cast<int>(ceil_div(N, cfg.info.block_n));
+    p.num_n_tiles = static_cast<int>(ceil_div(n_main, cfg.info.block_n));
     p.num_k_blocks = static_cast<int>(ceil_div(K, cfg.info.block_k));
     p.num_tiles = p.num_m_tiles * p.num_n_tiles;
     p.group_m = (opts && opts->group_m > 0) ? opts->group_m : cfg.info.group_m;
@@ -826,8 +943,10 @@ int tg_gemm_launch_count(const void *A, const void *B, const void *bias, const v
     const bool a_direct = aligned(A, 16) && (K % 8 == 0);
     const bool b_direct = aligned(B, 16) && (N % 8 == 0);
     const Choice c = choose_config(M, N, K, epilogue, 148);
-    if (kConfigs[c.config].info.loader == tg::kLoadPlain) return 1;
-    return 1 + ((a_direct && b_direct) ? 0 : 1);
+    const tg_config_t &ci = kConfigs[c.config].info;
+    if (ci.loader == tg::kLoadPlain) return 1;
+    return 1 + ((a_direct && b_direct) ? 0 : 1) +
+           (tail_cols(ci, M, N, K, epilogue, c.split, 148) > 0 ? 1 : 0);
 }
 
 tg_status_t tg_gemm_check_error(void *stream)

@@ -334,19 +334,20 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b)
 // lower tail T = Phi(-a), GELU(v) = max(v, 0) - a * T for either sign of v.
 // log2 T(a) is the Gaussian exponent -a^2 log2(e) / 2 plus a smooth
 // remainder (the logarithm of the Mills ratio, falling like -log2(a) for
-// large a), which a degree-7 polynomial Q in x = min(a, 6) / 3 - 1 fits to
-// 5e-6 in log2 units (csrc/fit_gelu.py; our coefficients):
-//   T = 2^( -a^2 log2(e) / 2 + Q(x) ).
-// Past a = 6 the Gaussian term alone puts a * T below half the smallest fp16
-// subnormal, so the clamp of x changes no fp16 result.  One exponential, no
-// division; in fp32 the result is within one fp16 ulp of the correctly
-// rounded GELU for every fp16 input (0.4% of them off by one).
-constexpr float kGeluQ0 = -3.040808201e+00f, kGeluQ1 = -1.225311518e+00f,
-                kGeluQ2 = 4.581521749e-01f, kGeluQ3 = -2.038841099e-01f,
+// large a); on a in [0, 6] the whole of it is fitted by a degree-7
+// polynomial Q in x = a / 3 - 1 to 5e-6 in log2 units (csrc/fit_gelu.py; our
+// coefficients), so
+//   T = 2^Q(x)   (a <= 6),   T = 0   (a > 6).
+// Past a = 6, a * T is below half the smallest fp16 subnormal for every fp16
+// input, so the cut changes no fp16 result but the sign of a zero.  One
+// exponential, no division, 9 multiply-adds; in fp32 the result is within
+// one fp16 ulp of the correctly rounded GELU for every fp16 input (0.4% of
+// them off by one).
+constexpr float kGeluQ0 = -9.532936096e+00f, kGeluQ1 = -1.420956707e+01f,
+                kGeluQ2 = -6.033975601e+00f, kGeluQ3 = -2.038841099e-01f,
                 kGeluQ4 = 9.168275446e-02f, kGeluQ5 = -4.095217586e-02f,
                 kGeluQ6 = 1.681641303e-02f, kGeluQ7 = -4.013689235e-03f;
 constexpr float kGeluAMax = 6.0f;
-constexpr float kHalfLog2e = 0.721347520444481703f;   // log2(e) / 2
 
 __device__ __forceinline__ float gelu_erf(float v)
 {
@@ -359,16 +360,15 @@ __device__ __forceinline__ float gelu_erf(float v)
     p = fmaf(p, x, kGeluQ2);
     p = fmaf(p, x, kGeluQ1);
     p = fmaf(p, x, kGeluQ0);
-    const float t = exp2_approx(fmaf(-a * kHalfLog2e, a, p));
+    const float t = a > kGeluAMax ? 0.0f : exp2_approx(p);
     return fmaf(-a, t, fmaxf(v, 0.0f));
 }
 
-// gelu_erf of two values at once: the polynomial and the exponent run as
-// packed f32x2 operations (the same roundings as the scalar form).
+// gelu_erf of two values at once: the polynomial runs as packed f32x2
+// operations (the same roundings as the scalar form).
 __device__ __forceinline__ void gelu_erf2(float &v0, float &v1)
 {
     const float a0 = fabsf(v0), a1 = fabsf(v1);
-    const uint64_t a = f2_pack(a0, a1);
     const uint64_t x = f2_fma(f2_pack(fminf(a0, kGeluAMax), fminf(a1, kGeluAMax)),
                               f2_pack(2.0f / kGeluAMax, 2.0f / kGeluAMax), f2_pack(-1.0f, -1.0f));
     uint64_t p = f2_fma(f2_pack(kGeluQ7, kGeluQ7), x, f2_pack(kGeluQ6, kGeluQ6));
@@ -378,11 +378,12 @@ __device__ __forceinline__ void gelu_erf2(float &v0, float &v1)
     p = f2_fma(p, x, f2_pack(kGeluQ2, kGeluQ2));
     p = f2_fma(p, x, f2_pack(kGeluQ1, kGeluQ1));
     p = f2_fma(p, x, f2_pack(kGeluQ0, kGeluQ0));
-    const uint64_t e = f2_fma(f2_mul(a, f2_pack(-kHalfLog2e, -kHalfLog2e)), a, p);
     float e0, e1;
-    f2_unpack(e, e0, e1);
-    v0 = fmaf(-a0, exp2_approx(e0), fmaxf(v0, 0.0f));
-    v1 = fmaf(-a1, exp2_approx(e1), fmaxf(v1, 0.0f));
+    f2_unpack(p, e0, e1);
+    const float t0 = a0 > kGeluAMax ? 0.0f : exp2_approx(e0);
+    const float t1 = a1 > kGeluAMax ? 0.0f : exp2_approx(e1);
+    v0 = fmaf(-a0, t0, fmaxf(v0, 0.0f));
+    v1 = fmaf(-a1, t1, fmaxf(v1, 0.0f));
 }
 
 // tanh approximation of GELU (Hendrycks & Gimpel, "Gaussian Error Linear
@@ -1323,6 +1324,88 @@ __global__ void __launch_bounds__(256) pack_pad2_kernel(const PackJob a, const P
 #pragma unroll
         for (int i = 0; i < kPackGroups; ++i)
             if (dst[i]) *dst[i] = u[i];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// The last r columns of C, when a thin remainder past a multiple of the tile
+// width would cost the tensor-core kernel a whole extra wave of tiles:
+//   C[i][n0 + j] = g( sum_k A[i][k] B[k][n0 + j] + beta[n0 + j] ),  j < r <= RT,
+// on the CUDA cores.  A and B are the operands as the GEMM reads them (row
+// pitches lda, ldb; A's rows 16-byte aligned with zero padding up to lda).
+// B's r columns are staged in shared memory (K x RT fp16, zeros past r);
+// each warp takes one row of A at a time, each lane 8 consecutive k per step,
+// products summed in fp32, then a warp reduction per column.
+constexpr int kTailLoads = 12;  // 16-byte loads of A in flight per lane: K <= 3072 in one step
+
+template <int EPI, int RT>
+__global__ void __launch_bounds__(256) tail_cols_kernel(const __half *A, int64_t lda,
+                                                        const __half *B, int64_t ldb,
+                                                        const __half *bias, __half *C,
+                                                        int64_t ldc, int64_t M, int64_t K,
+                                                        int64_t n0, int r)
+{
+    extern __shared__ __align__(16) __half bs[];   // [K][RT]
+    grid_launch_dependents();
+    // B's r columns into shared memory, eight loads in flight per thread.
+    for (int64_t i0 = threadIdx.x; i0 < K * RT; i0 += 8 * static_cast<int64_t>(blockDim.x)) {
+        __half v[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            const int64_t i = i0 + t * static_cast<int64_t>(blockDim.x);
+            const int64_t k = i / RT;
+            const int j = static_cast<int>(i - k * RT);
+            v[t] = (i < K * RT && j < r) ? B[k * ldb + n0 + j]
+                                         : __ushort_as_half(static_cast<unsigned short>(0));
+        }
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            const int64_t i = i0 + t * static_cast<int64_t>(blockDim.x);
+            if (i < K * RT) bs[i] = v[t];
+        }
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t k8 = (K + 7) / 8;
+    for (int64_t m = static_cast<int64_t>(blockIdx.x) * 8 + warp; m < M;
+         m += static_cast<int64_t>(gridDim.x) * 8) {
+        float acc[RT];
+#pragma unroll
+        for (int j = 0; j < RT; ++j) acc[j] = 0.f;
+        const uint4 *arow = reinterpret_cast<const uint4 *>(A + m * lda);
+        for (int64_t g0 = lane; g0 < k8; g0 += 32 * kTailLoads) {
+            uint4 u[kTailLoads];
+#pragma unroll
+            for (int t = 0; t < kTailLoads; ++t) {
+                const int64_t g = g0 + 32 * t;
+                u[t] = g < k8 ? __ldg(arow + g) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int t = 0; t < kTailLoads; ++t) {
+                const int64_t g = g0 + 32 * t;
+                const uint32_t w[4] = {u[t].x, u[t].y, u[t].z, u[t].w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int64_t k = g * 8 + e;
+                    if (k >= K) break;
+                    const float a = __half2float(half_of(w[e >> 1], e & 1));
+#pragma unroll
+                    for (int j = 0; j < RT; ++j)
+                        acc[j] = fmaf(a, __half2float(bs[k * RT + j]), acc[j]);
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < RT; ++j)
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+#pragma unroll
+        for (int j = 0; j < RT; ++j)
+            if (lane == j && j < r) {
+                const float beta =
+                    (EPI != kEpiNone && bias != nullptr) ? __half2float(bias[n0 + j]) : 0.f;
+                C[m * ldc + n0 + j] = __float2half_rn(apply_epilogue<EPI>(acc[j], beta));
+            }
     }
 }
 

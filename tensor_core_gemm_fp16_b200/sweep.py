@@ -2,7 +2,7 @@
 whole tiles and with stream-K, on each shape and (optionally) rewrite
 csrc/tg_configs.inc with the winners.
 
-    python -m tensor_core_gemm_fp16_b200.sweep [--shapes all|NAME ...]
+    python -m tensor_core_gemm_fp16_b200.sweep [--shapes all|offtable|NAME ...]
         [--reps 30] [--splits 1 2] [--context] [--write] [--json out.json]
 
 The tutorial sweeps tile sizes, pipeline stages, thread counts and an L2
@@ -45,6 +45,22 @@ DEFAULT_SHAPES = {
     "softmax_8192x256x4096": (8192, 256, 4096, 4),
     "deepk_fused_1024x1024x8192": (1024, 1024, 8192, 2),
     "deepk_512x512x16384": (512, 512, 16384, 0),
+}
+
+
+# Shapes that are not in the table, swept to check the cost rule that
+# chooses for them (tests/test_sweep_host.py reads the committed results in
+# offtable_sweep.json): squares between the table's sizes, wide and tall
+# panels, a deep-K shape and unaligned pitches.
+OFF_TABLE_SHAPES = {
+    "fused_1024": (1024, 1024, 1024, 2),
+    "fused_4096": (4096, 4096, 4096, 2),
+    "gemm_1536x3072x2048": (1536, 3072, 2048, 0),
+    "bias_512x4096x1024": (512, 4096, 1024, 1),
+    "fused_6144x2048x512": (6144, 2048, 512, 2),
+    "gemm_768x768x4096": (768, 768, 4096, 0),
+    "fused_2500x999x2998": (2500, 999, 2998, 2),
+    "gemm_4096x512x8192": (4096, 512, 8192, 0),
 }
 
 
@@ -282,11 +298,17 @@ def main(argv=None):
     import torch
     from tensor_core_gemm_fp16_b200 import binding
 
-    names = list(DEFAULT_SHAPES) if args.shapes == ["all"] else args.shapes
+    shapes = dict(DEFAULT_SHAPES, **OFF_TABLE_SHAPES)
+    if args.shapes == ["all"]:
+        names = list(DEFAULT_SHAPES)
+    elif args.shapes == ["offtable"]:
+        names = list(OFF_TABLE_SHAPES)
+    else:
+        names = args.shapes
     configs = args.configs if args.configs is not None else list(range(binding.tg_num_configs()))
     results = []
     for name in names:
-        M, N, K, epi = DEFAULT_SHAPES[name]
+        M, N, K, epi = shapes[name]
         r = sweep_shape(torch, binding, name, M, N, K, epi, args.reps, args.warmup, configs,
                         tuple(args.group_m), args.context, args.rounds, tuple(args.splits))
         results.append(r)

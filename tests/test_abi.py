@@ -188,12 +188,16 @@ def test_valid_call_without_a_device_reports_unsupported_device():
 
 def test_launch_count_is_host_only():
     """One GEMM kernel, plus one repacking kernel for both operands when
-    either row pitch or base is not a multiple of 16 bytes."""
+    either row pitch or base is not a multiple of 16 bytes, plus the thin
+    N-remainder kernel when it saves the GEMM a wave."""
     f = binding.tg_gemm_launch_count
     assert f(0x1000, 0x100000, None, 0x1000000, 256, 256, 256, NONE) == 1
     assert f(0x1000, 0x100000, None, 0x1000000, 256, 256, 250, NONE) == 2   # K % 8
     assert f(0x1000, 0x100000, None, 0x1000000, 256, 250, 256, NONE) == 2   # N % 8
     assert f(0x1000, 0x100000, None, 0x1000000, 300, 1537, 2050, GELU) == 2  # both
+    # 3000 x 1537: the last column of 256-wide tiles (one valid column) would
+    # add a second wave; the tail kernel computes that column instead
+    assert f(0x1000, 0x100000, None, 0x1000000, 3000, 1537, 2050, GELU) == 3
     assert f(0x1002, 0x100000, None, 0x1000000, 256, 256, 256, NONE) == 2   # A's base
     assert f(0x1000, 0x100000, None, 0x1000000, 256, 256, 0, GELU) == 1     # K == 0
     assert f(0x1000, 0x100000, None, 0x1000000, 0, 256, 256, NONE) == 0

@@ -1,8 +1,8 @@
 """The erf-GELU epilogue's fitted constants, checked on the host.
 
 The kernel evaluates GELU(v) = max(v, 0) - a * T(a), a = |v|, with the lower
-normal tail T = 2^(-a^2 log2(e)/2 + Q(x)), x = min(a, 6)/3 - 1, and Q a
-degree-7 polynomial whose coefficients csrc/fit_gelu.py fitted.  This test
+normal tail T = 2^Q(x), x = min(a, 6)/3 - 1 (T = 0 past a = 6), and Q a
+degree-7 polynomial fitted by csrc/fit_gelu.py to the whole of log2 T.  This test
 reads the coefficients as compiled into tg_kernels.cuh, replays the kernel's
 fp32 operations on every finite fp16 input in [-16, 16] (each fused
 multiply-add rounded once), and requires the fp16 result to be within one

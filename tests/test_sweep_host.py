@@ -91,3 +91,25 @@ def test_partial_sweep_keeps_the_other_rows(tmp_path):
     assert merged[1:] == committed[1:]
     sweep.write_table(results, path=str(out))
     assert len(sweep.read_table(str(out))) == 1
+
+
+def test_cost_rule_is_close_to_the_sweep_on_shapes_outside_the_table():
+    """Shapes missing from the table get the cost rule's choice.  On a set of
+    such shapes swept on a B200 (offtable_sweep.json: every configuration and
+    work division, timed), the rule's (configuration, split) must be within
+    20% of the fastest, and within 8% on average."""
+    import json
+    path = os.path.join(ROOT, "tensor_core_gemm_fp16_b200", "offtable_sweep.json")
+    with open(path) as f:
+        shapes = json.load(f)["shapes"]
+    assert len(shapes) >= 8
+    ratios = []
+    for s in shapes:
+        assert (s["M"], s["N"], s["K"]) not in {(r[0], r[1], r[2]) for r in sweep.read_table()}
+        best = min(r["us"] for r in s["rows"])
+        c = binding.tg_gemm_select_config(s["M"], s["N"], s["K"], s["epilogue"], 148)
+        mine = [r["us"] for r in s["rows"] if r["config"] == c["id"] and r["split"] == c["split"]]
+        assert mine, f"{s['shape']}: the rule's choice was not swept"
+        ratios.append(mine[0] / best)
+        assert mine[0] <= 1.2 * best, f"{s['shape']}: rule {mine[0]} us vs best {best} us"
+    assert sum(ratios) / len(ratios) <= 1.08, ratios

@@ -14,7 +14,7 @@ import torch
 import oracle
 from tensor_core_gemm_fp16_b200 import binding
 from tensor_core_gemm_fp16_b200 import workloads as wl
-from gpu_helpers import assert_close
+from gpu_helpers import assert_close, assert_close_blocked
 
 pytestmark = pytest.mark.gpu
 
@@ -150,22 +150,16 @@ def test_timeout_injection_reports_and_recovers():
 
 # ---------------------------------------------------------------- full-size workloads
 
-def _sample_rows(n_rows, n, seed):
-    rng = np.random.default_rng(seed)
-    fixed = [0, 1, 127, 128, 255, n_rows // 2, n_rows - 129, n_rows - 1]
-    return sorted(set(int(r) for r in fixed + list(rng.choice(n_rows, size=n, replace=False))))
-
-
 @pytest.mark.parametrize("name", list(wl.ATTN_WORKLOADS))
-def test_workload_sampled_rows(name):
-    """The full launch; every element of ~70 sampled query rows against the oracle."""
+def test_workload_full_output(name):
+    """The full launch of each attention workload (the benchmark's shapes),
+    every output element against the whole fp64 oracle result (a few seconds
+    of oracle time on the host cores)."""
     w = wl.ATTN_WORKLOADS[name]
     Q, K, V = wl.attn_workload_inputs(w)
     O = run_attn(Q, K, V, w.causal)
-    rows = _sample_rows(w.B * w.H * w.Sq, 60, seed=w.seed)
-    ref = oracle_attn(Q, K, V, w.causal, rows=rows)
-    assert_close(O.reshape(-1, w.D)[rows], ref, f"{name} sampled rows")
-    assert torch.isfinite(O.float()).all()
+    ref = oracle_attn(Q, K, V, w.causal).reshape(-1, w.D)
+    assert_close_blocked(O.reshape(-1, w.D), ref, f"{name} full output", block_rows=65536)
 
 
 # ---------------------------------------------------------------- key-half split

@@ -208,6 +208,19 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b)
     return d;
 }
 
+// 16 consecutive 32-bit TMEM columns of this thread's lane from r (the
+// 16-column form of tmem_st_32x32b_x32).
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi)
 {
     __half2 h = __floats2half2_rn(lo, hi);
@@ -499,8 +512,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             // which infinity).  The row maximum of the scaled scores is the scale
             // times the raw maximum (or minimum, for a negative scale), and each
             // exponent is one fused multiply-add: 2^(s * scale * log2 e - m).
-            // Two passes over the row in TMEM, 64 columns at a time (registers
-            // for a whole row would spill): the maximum, then the exponentials.
             const int64_t key0 = static_cast<int64_t>(kv_lo + j) * kTileK;
             const bool need_mask =
                 key0 + kTileK > p.Sk || (p.causal && key0 + kTileK - 1 > q0);
@@ -510,38 +521,51 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (p.causal && qi + 1 - key0 < lim) lim = qi + 1 - key0;
             }
             const float masked = pos ? -INFINITY : INFINITY;
-            auto load_half = [&](int h, float (&x)[64]) {
-                uint32_t sa[32], sb[32];
-                tmem_ld_32x32b_x32(t_lane + static_cast<uint32_t>(h * 64), sa);
-                tmem_ld_32x32b_x32(t_lane + static_cast<uint32_t>(h * 64 + 32), sb);
-                tmem_wait_ld_dep(sa);
-                tmem_wait_ld_dep(sb);
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    x[c] = __uint_as_float(sa[c]);
-                    x[32 + c] = __uint_as_float(sb[c]);
-                }
+            // The whole 128-score row comes out of TMEM in one round trip (four
+            // loads behind one wait) and stays in registers for both the
+            // maximum and the exponentials.
+            uint32_t s0[32], s1[32], s2[32], s3[32];
+            tmem_ld_32x32b_x32(t_lane + 0u, s0);
+            tmem_ld_32x32b_x32(t_lane + 32u, s1);
+            tmem_ld_32x32b_x32(t_lane + 64u, s2);
+            tmem_ld_32x32b_x32(t_lane + 96u, s3);
+            tmem_wait_ld_dep(s0);
+            tmem_wait_ld_dep(s1);
+            tmem_wait_ld_dep(s2);
+            tmem_wait_ld_dep(s3);
+            if constexpr (S::kSepP) {
+                // All of S_t,j is in registers: S_t,j+1 may land.
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_free[t]);
+            }
+            auto mask32 = [&](uint32_t (&x)[32], int c0) {
                 if (need_mask) {
 #pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        if (h * 64 + c >= lim) x[c] = masked;
+                    for (int c = 0; c < 32; ++c)
+                        if (c0 + c >= lim) x[c] = __float_as_uint(masked);
                 }
             };
+            mask32(s0, 0);
+            mask32(s1, 32);
+            mask32(s2, 64);
+            mask32(s3, 96);
             float mx[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) mx[u] = masked;
-#pragma unroll 1
-            for (int h = 0; h < 2; ++h) {
-                float x[64];
-                load_half(h, x);
+            auto ext32 = [&](const uint32_t (&x)[32]) {
                 if (pos) {
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+                    for (int c = 0; c < 32; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(x[c]));
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) mx[c & 7] = fminf(mx[c & 7], x[c]);
+                    for (int c = 0; c < 32; ++c) mx[c & 7] = fminf(mx[c & 7], __uint_as_float(x[c]));
                 }
-            }
+            };
+            ext32(s0);
+            ext32(s1);
+            ext32(s2);
+            ext32(s3);
             const float rext = pos ? fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                            fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])))
                                    : fminf(fminf(fminf(mx[0], mx[1]), fminf(mx[2], mx[3])),
@@ -587,28 +611,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_st_32x32b_x32(t_o, o);
                 }
             }
-            // P row into TMEM columns [0, 64), half h (keys 64h .. 64h + 63) into
-            // columns [32h, 32h + 32): half 0's P overwrites scores that half 0
-            // has already read, half 1's the rest of half 0.  Arguments and
-            // partial sums use the packed f32x2 FMA and add.
+            // P row into TMEM columns [0, 64): keys 2i, 2i + 1 packed into column
+            // i; with head width 128 this overwrites scores already in registers.
+            // Arguments and partial sums use the packed f32x2 FMA and add.
             const uint64_t sl2x2 = f2(sl2, sl2);
             const uint64_t nmu2 = f2(-mu, -mu);
             uint64_t ps2[4] = {0, 0, 0, 0};
-#pragma unroll 1
-            for (int h = 0; h < 2; ++h) {
-                float x[64];
-                load_half(h, x);
-                if (S::kSepP && h == 1) {
-                    // All of S_t,j is in registers or consumed: S_t,j+1 may land.
-                    tc_fence_before_sync();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&s_free[t]);
-                }
-                uint32_t hp[32];
+            // 32 scores -> 16 packed P columns at a time (keeps the live
+            // registers within the launch's budget).
+            auto exp32 = [&](const uint32_t (&x)[32], int q) {
+                uint32_t hp[16];
 #pragma unroll
-                for (int c = 0; c < 64; c += 2) {
+                for (int c = 0; c < 32; c += 2) {
                     const int pr = c >> 1;
-                    const uint64_t a2 = ffma2(f2(x[c], x[c + 1]), sl2x2, nmu2);
+                    const uint64_t a2 =
+                        ffma2(f2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])), sl2x2, nmu2);
                     float a0, a1;
                     f2split(a2, a0, a1);
                     const float e0 = ex2(a0);
@@ -616,8 +633,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ps2[pr & 3] = fadd2(ps2[pr & 3], f2(e0, e1));
                     hp[pr] = pack_half2(e0, e1);
                 }
-                tmem_st_32x32b_x32(t_lane + S::kPCol + static_cast<uint32_t>(h * 32), hp);
-            }
+                tmem_st_32x32b_x16(t_lane + S::kPCol + static_cast<uint32_t>(q * 16), hp);
+            };
+            exp32(s0, 0);
+            exp32(s1, 1);
+            exp32(s2, 2);
+            exp32(s3, 3);
             float q0, q1, q2, q3;
             f2split(fadd2(ps2[0], ps2[1]), q0, q1);
             f2split(fadd2(ps2[2], ps2[3]), q2, q3);

@@ -12,29 +12,30 @@
 // ten warps.
 //   warps 4t .. 4t+3  softmax of tile t: thread r owns query row r of the tile
 //              (TMEM lane r).  Reads S_t from TMEM, masks, exponentiates, and
-//              writes P_t (fp16, two values per 32-bit column) back into the
-//              first 64 columns of S_t, where the tensor core reads it as the
-//              A operand of P_t V; rescales O_t in TMEM when needed; stores
+//              writes P_t (fp16), where the tensor core reads it as the A
+//              operand of P_t V; rescales O_t in TMEM when needed; stores
 //              O_t / l at the end.
 //   warp 8     TMA producer (one lane): Q for both tiles, then the K and V
 //              tiles into their rings, polling both rings' empty barriers
 //              without blocking so neither ring waits on the other.
 //   warp 9     TMEM allocator and MMA issuer (one lane).
-// TMEM: tile t owns columns [256 t, 256 t + 256).  Head width 128: S_t (and
-// P_t, written over it) in the first 128, O_t in the next 128.  Head width
-// 64: S_t in the first 128, P_t in the next 64, O_t in the last 64; P no
-// longer overwrites S, so S_t,j+1 can be issued as soon as the softmax group
-// has read S_t,j, while it still exponentiates.  The two tiles' softmax phases
-// alternate on the SM: while one group's exponentials occupy the SFU, the
-// other's hand-offs and the tensor core's products proceed.
+// TMEM: tile t owns columns [256 t, 256 t + 256).  Head width 64: S_t in the
+// first 128, P_t (two fp16 per 32-bit column) in the next 64, O_t in the last
+// 64.  Head width 128: S_t in the first 128 and O_t in the next 128, which
+// fills TMEM, so P_t goes to shared memory instead: a 128 x 128 fp16 tile per
+// query tile in the 128-byte-swizzled layout of the tensor core's A operand
+// (room for it comes from a single V stage).  Either way P never overwrites
+// S, so S_t,j+1 can be issued as soon as the softmax group has read S_t,j,
+// while it still exponentiates; the group's next step then finds its scores
+// ready.  The two tiles' softmax phases run side by side on the SM, sharing
+// the SFU, while the tensor core's products proceed; a quarter of the
+// exponentials (head width 128) are computed on the FMA pipe instead of the
+// SFU, so that both units work.
 //
-// Order of the MMA issuer per key tile j (each wait bounded), head width 128:
-//   P_0,j V_j  ->  S_0,j+1 (after P_0,j V_j completed: it overwrites P_0,j)
-//   P_1,j V_j  ->  S_1,j+1 (likewise)
-// so a softmax group that sees S_t,j+1 complete knows P_t,j V_j is done and
-// may rescale O_t and overwrite P_t.  Head width 64: S_0,j+1 and S_1,j+1 as
-// soon as the groups have read S_t,j (s_free), then the P_t,j V_j; a group
-// waits for P_t,j-1 V_j-1 itself before it rescales O_t or writes P_t.
+// Order of the MMA issuer per key tile j (each wait bounded): S_0,j+1 and
+// S_1,j+1 as soon as the groups have read S_t,j (s_free), then P_0,j V_j and
+// P_1,j V_j as the groups publish P (p_full).  A group waits for
+// P_t,j-1 V_j-1 itself before it rescales O_t or writes P_t.
 //
 // Lazy rescaling: a row keeps its maximum m until a tile raises it by more
 // than 8 (in log2 units), so exponentials stay below 2^8 and O is rescaled
@@ -115,20 +116,26 @@ template <int D>
 struct AttnShape {
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
     static constexpr int kAtoms = D / kAtom;
-    static constexpr int kKStages = D == 64 ? 4 : 3;    // K ring depth
-    static constexpr int kVStages = D == 64 ? 4 : 2;    // V ring depth
-    // P in its own TMEM columns (head width 64), or written over S (128)
-    static constexpr bool kSepP = D == 64;
-    static constexpr uint32_t kPCol = kSepP ? 128u : 0u;
-    static constexpr uint32_t kOCol = kSepP ? 192u : 128u;
+    static constexpr int kKStages = D == 64 ? 4 : 2;    // K ring depth
+    static constexpr int kVStages = D == 64 ? 4 : 1;    // V ring depth
+    // P in its own TMEM columns (head width 64) or in shared memory (128)
+    static constexpr bool kPSmem = D == 128;
+    static constexpr uint32_t kPCol = 128u;             // head width 64
+    static constexpr uint32_t kOCol = kPSmem ? 128u : 192u;
+    // One pair of scores in kEmuShare takes the FMA-pipe exponential (0: none)
+    static constexpr int kEmuShare = D == 128 ? 4 : 0;
     static constexpr int kTileBytes = kAtoms * kAtomBytes;   // one 128-row Q, K or V tile
     static constexpr int kQOff = 0;                          // Q of both query tiles
     static constexpr int kKOff = kQOff + kTilesPerCta * kTileBytes;
     static constexpr int kVOff = kKOff + kKStages * kTileBytes;
+    // P of each query tile, 128 rows x 128 keys as two 64-key atoms (head width 128)
+    static constexpr int kPTileBytes = kTileQ * kTileK * 2;
+    static constexpr int kPOff = kVOff + kVStages * kTileBytes;
+    static constexpr int kPBytes = kPSmem ? kTilesPerCta * kPTileBytes : 0;
     // barriers: q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV],
     // s_full[2], p_full[2], pv_done[2], s_free[2], drain
     static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 8 + 1;
-    static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
+    static constexpr int kBarOff = kPOff + kPBytes;
     static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
     static constexpr int kAbortOff = kTmemSlotOff + 4;
     static constexpr int kDynamicBytes = kAbortOff + 4 + 1024;
@@ -208,6 +215,50 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b)
     return d;
 }
 
+// 2^x for two values on the FMA pipe, so that part of the softmax's
+// exponentials leave the SFU (fit_exp2.py fits R and checks this sequence):
+// x = n + r with n = round(x), r in [-1/2, 1/2]; R(r) = 1 + c1 r + c2 r^2 +
+// c3 r^3 ~ 2^r by Horner in packed f32x2 arithmetic; n is added to R's
+// exponent field, taken from the low bits of x + 1.5 * 2^23.  x is first
+// raised to -125 (a masked score, -inf, gives about 2^-125, which rounds to
+// 0 in fp16 P).  Integer x gives 2^x exactly; elsewhere the relative error
+// stays below 1.1e-4, under the fp16 rounding P gets next.  A NaN score does
+// not propagate here; the row maximum carries it instead.
+constexpr float kExp2C1 = 6.932827830e-01f;
+constexpr float kExp2C2 = 2.422083467e-01f;
+constexpr float kExp2C3 = 5.500787124e-02f;
+constexpr float kExp2Round = 12582912.0f;   // 1.5 * 2^23
+
+__device__ __forceinline__ float max_nan(float a, float b)
+{
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+__device__ __forceinline__ float min_nan(float a, float b)
+{
+    float r;
+    asm("min.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint64_t exp2_fma2(float x0, float x1)
+{
+    const uint64_t x2 = f2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+    const uint64_t t2 = fadd2(x2, f2(kExp2Round, kExp2Round));
+    const uint64_t n2 = fadd2(t2, f2(-kExp2Round, -kExp2Round));
+    const uint64_t r2 = ffma2(n2, f2(-1.f, -1.f), x2);
+    uint64_t p2 = ffma2(f2(kExp2C3, kExp2C3), r2, f2(kExp2C2, kExp2C2));
+    p2 = ffma2(p2, r2, f2(kExp2C1, kExp2C1));
+    p2 = ffma2(p2, r2, f2(1.f, 1.f));
+    float t0, t1, q0, q1;
+    f2split(t2, t0, t1);
+    f2split(p2, q0, q1);
+    return f2(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
+              __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
+}
+
 // 16 consecutive 32-bit TMEM columns of this thread's lane from r (the
 // 16-column form of tmem_st_32x32b_x32).
 __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16])
@@ -219,6 +270,14 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_
         "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
         "r"(r[15])
         : "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi)
@@ -261,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *s_full = v_empty + SV;     // [2]: S_t of the current key tile is in TMEM
     uint64_t *p_full = s_full + 2;       // [2]: P_t written to TMEM (4 arrivals)
     uint64_t *pv_done = p_full + 2;      // [2]: P_t V complete
-    uint64_t *s_free = pv_done + 2;      // [2]: S_t read (4 arrivals; head width 64)
+    uint64_t *s_free = pv_done + 2;      // [2]: S_t read out of TMEM (4 arrivals)
     uint64_t *drain_bar = s_free + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::kTmemSlotOff);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + S::kAbortOff);
@@ -413,16 +472,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_commit<1>(&s_full[t]);
                 issued = true;
             };
-            // O_t += P_t,j V_j, P_t from TMEM (8 columns per 16 keys).
+            // O_t += P_t,j V_j: P from shared memory (head width 128, the
+            // same 64-key atoms as Q) or from TMEM (8 columns per 16 keys).
             auto issue_pv = [&](int t, int j) {
                 const uint32_t va = sbase + S::kVOff + (j % SV) * S::kTileBytes;
                 tc_fence_after_sync();
 #pragma unroll
-                for (int kk = 0; kk < kTileK / 16; ++kk)
-                    mma_f16_ts(tmem_base + t * kTileCols + S::kOCol,
-                               tmem_base + t * kTileCols + S::kPCol + static_cast<uint32_t>(kk * 8),
-                               smem_desc_sw128(va + kk * 2048, kAtomBytes, 1024), kIdescO,
-                               (j > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < kTileK / 16; ++kk) {
+                    const uint64_t vdesc = smem_desc_sw128(va + kk * 2048, kAtomBytes, 1024);
+                    const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+                    if constexpr (S::kPSmem) {
+                        const uint32_t off = (kk >> 2) * kAtomBytes + (kk & 3) * 32;
+                        mma_f16_ss<1>(tmem_base + t * kTileCols + S::kOCol,
+                                      smem_desc_sw128(sbase + S::kPOff + t * S::kPTileBytes + off,
+                                                      16, 1024),
+                                      vdesc, kIdescO, acc);
+                    } else {
+                        mma_f16_ts(tmem_base + t * kTileCols + S::kOCol,
+                                   tmem_base + t * kTileCols + S::kPCol +
+                                       static_cast<uint32_t>(kk * 8),
+                                   vdesc, kIdescO, acc);
+                    }
+                }
                 mma_commit<1>(&pv_done[t]);
                 issued = true;
             };
@@ -432,46 +503,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_commit<1>(&k_empty[0]);
             }
             for (int j = 0; ok && j < n_all; ++j) {
-                const bool next = j + 1 < n_all;
+                // S_t,j+1 as soon as group t has read S_t,j.
                 bool k_next = false;   // K_j+1 waited for
-                if constexpr (S::kSepP) {
-                    // S_t,j+1 as soon as group t has read S_t,j.
-                    for (int t = 0; t < 2 && ok; ++t) {
-                        if (j + 1 < nt[t]) {
-                            if (!k_next && !wait(&k_full[(j + 1) % SK], ((j + 1) / SK) & 1)) break;
-                            k_next = true;
-                            if (!wait(&s_free[t], j & 1)) break;
-                            issue_s(t, j + 1);
-                        }
-                    }
-                    if (!ok || !wait(&v_full[j % SV], (j / SV) & 1)) break;
-                    for (int t = 0; t < 2 && ok; ++t)
-                        if (j < nt[t]) {
-                            if (!wait(&p_full[t], j & 1)) break;
-                            issue_pv(t, j);
-                        }
-                    if (!ok) break;
-                    mma_commit<1>(&v_empty[j % SV]);
-                    if (next) mma_commit<1>(&k_empty[(j + 1) % SK]);
-                    continue;
-                }
-                if (!wait(&v_full[j % SV], (j / SV) & 1)) break;
                 for (int t = 0; t < 2 && ok; ++t) {
+                    if (j + 1 < nt[t]) {
+                        if (!k_next && !wait(&k_full[(j + 1) % SK], ((j + 1) / SK) & 1)) break;
+                        k_next = true;
+                        if (!wait(&s_free[t], j & 1)) break;
+                        issue_s(t, j + 1);
+                    }
+                }
+                if (!ok || !wait(&v_full[j % SV], (j / SV) & 1)) break;
+                for (int t = 0; t < 2 && ok; ++t)
                     if (j < nt[t]) {
                         if (!wait(&p_full[t], j & 1)) break;
                         issue_pv(t, j);
                     }
-                    if (j + 1 < nt[t]) {
-                        if (!k_next && !wait(&k_full[(j + 1) % SK], ((j + 1) / SK) & 1)) break;
-                        k_next = true;
-                        // S_t,j+1 overwrites P_t,j: only after P_t,j V_j completed.
-                        if (!wait(&pv_done[t], j & 1)) break;
-                        issue_s(t, j + 1);
-                    }
-                }
                 if (!ok) break;
                 mma_commit<1>(&v_empty[j % SV]);
-                if (next) mma_commit<1>(&k_empty[(j + 1) % SK]);
+                if (j + 1 < n_all) mma_commit<1>(&k_empty[(j + 1) % SK]);
             }
             if (issued) {
                 mma_commit<1>(drain_bar);
@@ -533,12 +583,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld_dep(s1);
             tmem_wait_ld_dep(s2);
             tmem_wait_ld_dep(s3);
-            if constexpr (S::kSepP) {
-                // All of S_t,j is in registers: S_t,j+1 may land.
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s_free[t]);
-            }
+            // All of S_t,j is in registers: S_t,j+1 may land.
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free[t]);
             auto mask32 = [&](uint32_t (&x)[32], int c0) {
                 if (need_mask) {
 #pragma unroll
@@ -553,97 +601,133 @@ __global__ void __launch_bounds__(kThreads, 1)
             float mx[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) mx[u] = masked;
+            // The extreme keeps NaN (a NaN score makes the row NaN, as the
+            // exact softmax would).
             auto ext32 = [&](const uint32_t (&x)[32]) {
                 if (pos) {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(x[c]));
+                    for (int c = 0; c < 32; ++c) mx[c & 7] = max_nan(mx[c & 7], __uint_as_float(x[c]));
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) mx[c & 7] = fminf(mx[c & 7], __uint_as_float(x[c]));
+                    for (int c = 0; c < 32; ++c) mx[c & 7] = min_nan(mx[c & 7], __uint_as_float(x[c]));
                 }
             };
             ext32(s0);
             ext32(s1);
             ext32(s2);
             ext32(s3);
-            const float rext = pos ? fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])))
-                                   : fminf(fminf(fminf(mx[0], mx[1]), fminf(mx[2], mx[3])),
-                                           fminf(fminf(mx[4], mx[5]), fminf(mx[6], mx[7])));
+            const float rext =
+                pos ? max_nan(max_nan(max_nan(mx[0], mx[1]), max_nan(mx[2], mx[3])),
+                              max_nan(max_nan(mx[4], mx[5]), max_nan(mx[6], mx[7])))
+                    : min_nan(min_nan(min_nan(mx[0], mx[1]), min_nan(mx[2], mx[3])),
+                              min_nan(min_nan(mx[4], mx[5]), min_nan(mx[6], mx[7])));
             const float tmax = rext * sl2;
-            // Lazy rescale: move m only when the tile raises it by more than 8.
+            // Lazy rescale: move m only when the tile raises it by more than 8
+            // (or brings a NaN, which then reaches every exponential).
             float alpha = 1.f;
-            const bool raise = tmax > m + 8.f;
+            const bool raise = !(tmax <= m + 8.f);
             if (raise) {
                 alpha = (m == -INFINITY) ? 0.f : ex2(m - tmax);
                 m = tmax;
             }
             const float mu = (m == -INFINITY) ? 0.f : m;
-            // Head width 128: P_t,j-1 V_j-1 is complete (S_t,j was issued after
-            // it).  Head width 64: wait for it here.  Then O_t may be rescaled
-            // and P_t overwritten.
-            if constexpr (S::kSepP) {
-                if (j > 0) {
-                    int okv = 1;
-                    if (lane == 0)
-                        okv = mbar_wait_bounded(&pv_done[t], (j - 1) & 1, abort_flag, limit,
-                                                p.error_word, kErrAttnSoftmax)
-                                  ? 1
-                                  : 0;
-                    okv = __shfl_sync(0xffffffffu, okv, 0);
-                    if (!okv) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after_sync();
-                }
-            }
-            if (j > 0 && __any_sync(0xffffffffu, raise)) {
+            // Before O_t is rescaled or P_t written, P_t,j-1 V_j-1 must be
+            // complete.
+            auto wait_prev = [&]() -> bool {
+                int okv = 1;
+                if (lane == 0 && j > 0)
+                    okv = mbar_wait_bounded(&pv_done[t], (j - 1) & 1, abort_flag, limit,
+                                            p.error_word, kErrAttnSoftmax)
+                              ? 1
+                              : 0;
+                okv = __shfl_sync(0xffffffffu, okv, 0);
+                tc_fence_after_sync();
+                return okv != 0;
+            };
+            auto rescale_o = [&]() {
+                if (j > 0 && __any_sync(0xffffffffu, raise)) {
 #pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t o[32];
-                    const uint32_t t_o = t_lane + S::kOCol + static_cast<uint32_t>(c * 32);
-                    tmem_ld_32x32b_x32(t_o, o);
-                    tmem_wait_ld_dep(o);
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        const uint32_t t_o = t_lane + S::kOCol + static_cast<uint32_t>(c * 32);
+                        tmem_ld_32x32b_x32(t_o, o);
+                        tmem_wait_ld_dep(o);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    tmem_st_32x32b_x32(t_o, o);
+                        for (int e = 0; e < 32; ++e)
+                            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st_32x32b_x32(t_o, o);
+                    }
                 }
-            }
-            // P row into TMEM columns [0, 64): keys 2i, 2i + 1 packed into column
-            // i; with head width 128 this overwrites scores already in registers.
-            // Arguments and partial sums use the packed f32x2 FMA and add.
+            };
+            // P row: head width 64 into TMEM columns [128, 192), keys 2i, 2i + 1
+            // packed into column i; head width 128 into the shared P tile, row
+            // r of each 64-key atom at 128 r with its 16-byte chunks swizzled
+            // by r mod 8.  Arguments and partial sums use the packed f32x2 FMA
+            // and add.
             const uint64_t sl2x2 = f2(sl2, sl2);
             const uint64_t nmu2 = f2(-mu, -mu);
             uint64_t ps2[4] = {0, 0, 0, 0};
-            // 32 scores -> 16 packed P columns at a time (keeps the live
-            // registers within the launch's budget).
-            auto exp32 = [&](const uint32_t (&x)[32], int q) {
-                uint32_t hp[16];
+            // 32 scores -> 16 packed P values.
+            auto exp32 = [&](const uint32_t (&x)[32], uint32_t *hp) {
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
                     const int pr = c >> 1;
                     const uint64_t a2 =
                         ffma2(f2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])), sl2x2, nmu2);
-                    float a0, a1;
+                    float a0, a1, e0, e1;
                     f2split(a2, a0, a1);
-                    const float e0 = ex2(a0);
-                    const float e1 = ex2(a1);
+                    if (S::kEmuShare > 0 && pr % S::kEmuShare == S::kEmuShare - 1) {
+                        f2split(exp2_fma2(a0, a1), e0, e1);
+                    } else {
+                        e0 = ex2(a0);
+                        e1 = ex2(a1);
+                    }
                     ps2[pr & 3] = fadd2(ps2[pr & 3], f2(e0, e1));
                     hp[pr] = pack_half2(e0, e1);
                 }
-                tmem_st_32x32b_x16(t_lane + S::kPCol + static_cast<uint32_t>(q * 16), hp);
             };
-            exp32(s0, 0);
-            exp32(s1, 1);
-            exp32(s2, 2);
-            exp32(s3, 3);
+            if constexpr (S::kPSmem) {
+                // The whole P row in registers first, then (P_t,j-1 V_j-1 done)
+                // into the tile's P tile.
+                uint32_t hp[64];
+                exp32(s0, hp);
+                exp32(s1, hp + 16);
+                exp32(s2, hp + 32);
+                exp32(s3, hp + 48);
+                if (!wait_prev()) {
+                    ok = false;
+                    break;
+                }
+                rescale_o();
+                const uint32_t prow = sbase + S::kPOff + t * S::kPTileBytes + row * 128;
+#pragma unroll
+                for (int c = 0; c < 16; ++c)   // 16-byte chunk c: keys 8c .. 8c + 7
+                    st_shared_v4(prow + (c >> 3) * kAtomBytes + (((c & 7) ^ (row & 7)) << 4),
+                                 hp[4 * c], hp[4 * c + 1], hp[4 * c + 2], hp[4 * c + 3]);
+            } else {
+                if (!wait_prev()) {
+                    ok = false;
+                    break;
+                }
+                rescale_o();
+                // 32 scores -> 16 packed P columns at a time (keeps the live
+                // registers within the launch's budget).
+                auto exp_store = [&](const uint32_t (&x)[32], int q) {
+                    uint32_t hp[16];
+                    exp32(x, hp);
+                    tmem_st_32x32b_x16(t_lane + S::kPCol + static_cast<uint32_t>(q * 16), hp);
+                };
+                exp_store(s0, 0);
+                exp_store(s1, 1);
+                exp_store(s2, 2);
+                exp_store(s3, 3);
+            }
             float q0, q1, q2, q3;
             f2split(fadd2(ps2[0], ps2[1]), q0, q1);
             f2split(fadd2(ps2[2], ps2[3]), q2, q3);
             l = fmaf(l, alpha, (q0 + q1) + (q2 + q3));
             tmem_wait_st();
+            if constexpr (S::kPSmem) fence_proxy_async_smem();   // P visible to the tensor core
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[t]);

@@ -99,6 +99,32 @@ def test_first_causal_row_is_v0_exactly():
     assert torch.equal(O[:, :, 0], V[:, :, 0])
 
 
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("key", [6, 7, 70])
+def test_nan_key_makes_every_row_that_sees_it_nan(D, key):
+    """A NaN in one key makes every score against it NaN; the exact softmax is
+    then NaN for each row that sees the key, and stays finite for causal rows
+    before it.  With head width 128, keys 6, 7 and 70 fall among those whose
+    exponentials run on the FMA pipe, so the row maximum must carry the NaN."""
+    B, H, S = 1, 2, 200
+    Q, K, V = wl.attention_inputs(B, H, S, S, D, seed=164 + key)
+    K[:, :, key, 3] = float("nan")
+    O = run_attn_unchecked(Q, K, V, False)
+    assert torch.isnan(O.float()).any(dim=-1).all()
+    O = run_attn_unchecked(Q, K, V, True)
+    rows = torch.isnan(O.float()).any(dim=-1)
+    assert rows[:, :, key:].all() and not rows[:, :, :key].any()
+    assert torch.isfinite(O[:, :, :key].float()).all()
+
+
+def run_attn_unchecked(Q, K, V, causal):
+    dev = torch.device("cuda:0")
+    o = binding.attention(Q.to(dev), K.to(dev), V.to(dev), causal, 0.0)
+    torch.cuda.synchronize()
+    assert binding.tg_gemm_check_error(torch.cuda.current_stream().cuda_stream) == binding.TG_OK
+    return o.cpu()
+
+
 def test_empty_and_zero_keys():
     dev = torch.device("cuda:0")
     q = torch.randn(1, 2, 5, 64, device=dev).half()

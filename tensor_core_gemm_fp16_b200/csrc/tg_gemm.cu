@@ -178,6 +178,21 @@ struct Choice {
     int split;   // TG_SPLIT_TILES or TG_SPLIT_STREAM_K
 };
 
+// Stream-K units (CTAs, or CTA pairs): at most one per iteration, so that no
+// unit's range is empty.  When every tile can go to two or more units, each
+// tile's k-blocks are split evenly over S of them (S as large as fits and
+// divides the k-blocks): every tile then has one head and S - 1 contributors
+// that start and finish together, instead of ranges that straddle tiles.
+int64_t streamk_units(int64_t tiles, int64_t kb, int64_t units)
+{
+    if (tiles > 0 && tiles <= units / 2) {
+        int64_t S = units / tiles;
+        while (S > 1 && kb % S != 0) --S;
+        if (S >= 2) return tiles * S;
+    }
+    return std::min<int64_t>(tiles * kb, units);
+}
+
 void split_costs(int id, int64_t M, int64_t N, int64_t K, int sms, double *dp, double *sk)
 {
     const tg_config_t &ci = kConfigs[id].info;
@@ -189,10 +204,11 @@ void split_costs(int id, int64_t M, int64_t N, int64_t K, int sms, double *dp, d
     const double load_clk = (128.0 + static_cast<double>(ci.block_n) / cg) * ci.block_k * 2.0 / 64.0;
     const double iter_us = (mma_clk > load_clk ? mma_clk : load_clk) / (kClockGhz * 1e3);
     *dp = static_cast<double>(ceil_div(tiles, units) * kb) * iter_us;
+    const int64_t sk_units = streamk_units(tiles, kb, units);
     const double contributors =
-        units > tiles ? static_cast<double>(units) / static_cast<double>(tiles) : 1.0;
+        sk_units > tiles ? static_cast<double>(sk_units) / static_cast<double>(tiles) : 1.0;
     const double partial_bytes = 128.0 * ci.block_n * 4.0;
-    *sk = static_cast<double>(ceil_div(tiles * kb, units)) * iter_us + kStreamKFixedUs +
+    *sk = static_cast<double>(ceil_div(tiles * kb, sk_units)) * iter_us + kStreamKFixedUs +
           contributors * partial_bytes / (kFoldGBs * 1e3);
 }
 
@@ -630,9 +646,8 @@ tg_status_t launch_staged(const KernelConfig &cfg, const void *Aeff, int64_t lda
     p.wait_limit_ns = (opts && opts->wait_limit_ns) ? opts->wait_limit_ns : kDefaultWaitLimitNs;
     p.error_word = error_word;
     // Persistent grid: one CTA (or CTA pair) per SM (pair of SMs).  Whole
-    // tiles: never more units than tiles.
+    // tiles: never more units than tiles; stream-K: streamk_units.
     const int units = cfg.info.cta_pair ? num_sms / 2 : num_sms;
-    const int64_t iters = static_cast<int64_t>(p.num_tiles) * p.num_k_blocks;
     const bool stream_k = split == TG_SPLIT_STREAM_K;
     p.stream_k = stream_k ? 1 : 0;
     p.sk_partials = nullptr;
@@ -643,10 +658,10 @@ tg_status_t launch_staged(const KernelConfig &cfg, const void *Aeff, int64_t lda
             streamk_workspace(num_sms, stream, &p.sk_partials, &p.sk_flags, &p.sk_epoch);
         if (st != TG_OK) return st;
     }
-    // Stream-K: at most one unit per iteration, so that no unit's range is empty.
-    const int grid = static_cast<int>(stream_k ? std::min<int64_t>(iters, units)
-                                               : std::min<int64_t>(p.num_tiles, units)) *
-                     (cfg.info.cta_pair ? 2 : 1);
+    const int grid =
+        static_cast<int>(stream_k ? streamk_units(p.num_tiles, p.num_k_blocks, units)
+                                  : std::min<int64_t>(p.num_tiles, units)) *
+        (cfg.info.cta_pair ? 2 : 1);
 
     const cudaError_t e =
         cfg.fn[epilogue][store == tg::kStoreScalar ? 0 : 1](ta, tb, tc, p, grid, stream);

@@ -54,13 +54,14 @@ cudaError_t ensure_smem_attr(Kernel kern, int smem, std::atomic<uint64_t> &attr_
     return cudaSuccess;
 }
 
-template <int BN, int BK, int ST_REQ, int EPI, bool PAIR, int EW, int STORE, int LOAD>
+template <int BN, int BK, int ST_REQ, int EPI, bool PAIR, int EW, int STORE, int LOAD,
+          bool SHARE = false>
 cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc,
                         const tg::GemmParams &p, int grid, cudaStream_t stream)
 {
     constexpr int ST = tg::FittedStages<BN, BK, ST_REQ, PAIR, EW, STORE, LOAD>::value;
     using S = tg::KernelShape<BN, BK, ST, PAIR, EW, STORE, LOAD>;
-    auto kern = tg::gemm_persistent_kernel<BN, BK, ST, EPI, PAIR, EW, STORE, LOAD>;
+    auto kern = tg::gemm_persistent_kernel<BN, BK, ST, EPI, PAIR, EW, STORE, LOAD, SHARE>;
     static std::atomic<uint64_t> attr_set{0};
     cudaError_t e = ensure_smem_attr(kern, S::kDynamicBytes, attr_set);
     if (e != cudaSuccess) return e;
@@ -105,10 +106,22 @@ constexpr LaunchFn softmax_fn()
 
 constexpr int kNumEpilogues = 5;
 
+template <int BN, int BK, int ST, int EPI, bool PAIR, int EW, int STORE, int LOAD>
+constexpr LaunchFn share_fn()
+{
+    if constexpr (LOAD == tg::kLoadTma)
+        return launch_gemm<BN, BK, ST, EPI, PAIR, EW, STORE, LOAD, true>;
+    else
+        return nullptr;
+}
+
 struct KernelConfig {
     tg_config_t info;
     int store_pref;                  // store mode when C rows are 16-byte aligned
     LaunchFn fn[kNumEpilogues][2];   // [epilogue][0: element stores, 1: store_pref]
+    // Variants for an even stream-K split with a shared fold (store_pref, no
+    // row softmax; nullptr for the plain loader).
+    LaunchFn fn_share[kNumEpilogues - 1];
 };
 
 #define TG_FNS(BN, BK, ST, PAIR, EW, SP, LD)                                                \
@@ -125,9 +138,13 @@ struct KernelConfig {
              softmax_fn<BN, BK, ST, PAIR, EW, SP, LD>()},                                   \
     }
 
+#define TG_FNS_SHARE(BN, BK, ST, PAIR, EW, SP, LD)                                          \
+    {share_fn<BN, BK, ST, 0, PAIR, EW, SP, LD>(), share_fn<BN, BK, ST, 1, PAIR, EW, SP, LD>(),  \
+     share_fn<BN, BK, ST, 2, PAIR, EW, SP, LD>(), share_fn<BN, BK, ST, 3, PAIR, EW, SP, LD>()}
+
 #define TG_CONFIG(ID, BN, BK, ST, PAIR, EW, SP, GROUP, LD)                                  \
     {{ID, 128 * ((PAIR) ? 2 : 1), BN, BK, ST, (PAIR) ? 1 : 0, GROUP, EW, 0, LD}, SP,        \
-     TG_FNS(BN, BK, ST, PAIR, EW, SP, LD)}
+     TG_FNS(BN, BK, ST, PAIR, EW, SP, LD), TG_FNS_SHARE(BN, BK, ST, PAIR, EW, SP, LD)}
 
 // {id, BN, BK, stages, CTA pair, epilogue warps, store mode for aligned C, group_m, loader}
 // Configurations 9 and 10 load operands with plain loads (any row pitch, no
@@ -183,12 +200,16 @@ struct Choice {
 // tile's k-blocks are split evenly over S of them (S as large as fits and
 // divides the k-blocks): every tile then has one head and S - 1 contributors
 // that start and finish together, instead of ranges that straddle tiles.
-int64_t streamk_units(int64_t tiles, int64_t kb, int64_t units)
+int64_t streamk_units(int64_t tiles, int64_t kb, int64_t units, int *share = nullptr)
 {
+    if (share) *share = 0;
     if (tiles > 0 && tiles <= units / 2) {
         int64_t S = units / tiles;
         while (S > 1 && kb % S != 0) --S;
-        if (S >= 2) return tiles * S;
+        if (S >= 2) {
+            if (share) *share = static_cast<int>(S);
+            return tiles * S;
+        }
     }
     return std::min<int64_t>(tiles * kb, units);
 }
@@ -658,13 +679,26 @@ tg_status_t launch_staged(const KernelConfig &cfg, const void *Aeff, int64_t lda
             streamk_workspace(num_sms, stream, &p.sk_partials, &p.sk_flags, &p.sk_epoch);
         if (st != TG_OK) return st;
     }
+    // An even stream-K split shares each tile's fold among its units (not for
+    // the row softmax, whose epilogue needs whole rows).
+    int share = 0;
     const int grid =
-        static_cast<int>(stream_k ? streamk_units(p.num_tiles, p.num_k_blocks, units)
+        static_cast<int>(stream_k ? streamk_units(p.num_tiles, p.num_k_blocks, units, &share)
                                   : std::min<int64_t>(p.num_tiles, units)) *
         (cfg.info.cta_pair ? 2 : 1);
+    p.sk_share = (stream_k && epilogue != TG_EPILOGUE_BIAS_SOFTMAX) ? share : 0;
 
-    const cudaError_t e =
-        cfg.fn[epilogue][store == tg::kStoreScalar ? 0 : 1](ta, tb, tc, p, grid, stream);
+    LaunchFn fn = cfg.fn[epilogue][store == tg::kStoreScalar ? 0 : 1];
+    if (p.sk_share > 0) {
+        // The shared-fold variant exists for the preferred store mode only;
+        // otherwise the tile's first unit folds alone.
+        LaunchFn shared = store == tg::kStoreScalar ? nullptr : cfg.fn_share[epilogue];
+        if (shared)
+            fn = shared;
+        else
+            p.sk_share = 0;
+    }
+    const cudaError_t e = fn(ta, tb, tc, p, grid, stream);
     if (e != cudaSuccess) {
         cudaGetLastError();
         return TG_ERR_LAUNCH;

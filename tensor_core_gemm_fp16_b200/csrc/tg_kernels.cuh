@@ -82,6 +82,12 @@ struct GemmParams {
     unsigned *sk_flags;     // per CTA and epilogue warp: epoch at which that warp's
                             // rows / columns of the CTA's partial are complete
     unsigned sk_epoch;      // this launch's epoch (never 0)
+    // Stream-K with every tile split evenly over sk_share consecutive units
+    // (0: not so): the units of a tile share its fold.  Each writes its
+    // partial of the 32-column chunks it does not own, then adds the others'
+    // partials to the chunks it owns (chunk c: unit c mod sk_share of the
+    // tile) and runs their epilogue.  Not for the row softmax.
+    int sk_share;
 };
 
 // The work of one unit, as segments (tile, k-blocks [k0, k1)).
@@ -493,7 +499,11 @@ __device__ __forceinline__ __half half_of(uint32_t w, int hi)
 //   warp EPI_WARPS        TMA producer (one lane)
 //   warp EPI_WARPS + 1    TMEM allocator; MMA issuer (one lane; the leader CTA
 //                         of a pair issues for both)
-template <int BN, int BK, int STAGES, int EPI, bool PAIR, int EPI_WARPS, int STORE, int LOAD>
+// SHARE: the kernel variant launched for an even stream-K split, whose
+// tile's units share the fold (GemmParams::sk_share); the other variants
+// carry none of that code.
+template <int BN, int BK, int STAGES, int EPI, bool PAIR, int EPI_WARPS, int STORE, int LOAD,
+          bool SHARE = false>
 __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, STORE, LOAD>::kThreads,
                                   1)
     gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -835,14 +845,49 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                                                  static_cast<size_t>(slot) * kBlockM * BN) +
                        ((warp * S::kChunksPerWarp + (c - chunk0)) * 8 + q) * 32 + lane;
             };
-            int first_contrib = 0, last_contrib = -1;   // units whose partials a head adds
-            if (role == kSegHead) {
+            // Shared fold (an even split, sk_share units per tile): this unit is
+            // member `me` of the tile's units and owns its chunks c with
+            // c mod sk_share == me.
+            const bool shared =
+                SHARE && EPI != kEpiBiasSoftmax && p.sk_share > 0 && role != kSegFull;
+            const int share = shared ? p.sk_share : 1;
+            const int me = shared ? unit % share : 0;
+            auto owned = [&](int c) { return !shared || c % share == me; };
+            int first_contrib = 0, last_contrib = -1;   // units whose partials this unit adds,
+            int skip_v = -1;                            // except this one
+            if (shared) {
+                // First the chunks this unit does not own, for their owners.
+#pragma unroll 1
+                for (int c = chunk0; c < chunk0 + S::kChunksPerWarp; ++c) {
+                    if (owned(c)) continue;
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * kStoreCols), r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        __stcg(partial_group(unit * CG + cta_rank, c, q),
+                               make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]));
+                }
+                __threadfence();
+                __syncwarp();
+                if (lane == 0 && p.inject != 2)
+                    st_release_gpu(p.sk_flags + (unit * CG + cta_rank) * EPI_WARPS + warp,
+                                   p.sk_epoch);
+                first_contrib = unit - me;
+                last_contrib = unit - me + share - 1;
+                skip_v = unit;
+            } else if (role == kSegHead) {
                 const long long tile_end = static_cast<long long>(tile + 1) * p.num_k_blocks;
                 first_contrib = unit + 1;
                 last_contrib = WorkIter::last_contributor(p, unit, num_units, tile_end);
-                // Warp w of a head reads exactly the rows and columns that warp w
-                // of each contributing CTA wrote, so it waits for those flags only.
-                for (int v = first_contrib; v <= last_contrib; ++v) {
+            }
+            // The contributing units in the order their partials are added.
+            const int v_begin = first_contrib == skip_v ? first_contrib + 1 : first_contrib;
+            auto next_v = [&](int v) { return v + 1 == skip_v ? v + 2 : v + 1; };
+            {
+                // Warp w reads exactly the rows and columns that warp w of each
+                // contributing CTA wrote, so it waits for those flags only.
+                for (int v = v_begin; v <= last_contrib; v = next_v(v)) {
                     const unsigned *flag = p.sk_flags + (v * CG + cta_rank) * EPI_WARPS + warp;
                     if (ld_acquire_gpu(flag) == p.sk_epoch) continue;
                     const uint64_t t0 = global_timer_ns();
@@ -870,12 +915,17 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
             // ascending -- the order the sums are taken in -- and item i is
             // copied into slot i % kFoldSlots of this warp's part of the ring,
             // kFoldSlots items ahead of its use.
-            bool folding = first_contrib <= last_contrib && chunk_end > chunk0 && *abort_flag == 0;
+            // The first chunk this warp finishes (shared fold: the first it owns).
+            int first_owned = chunk0;
+            while (first_owned < chunk_end && !owned(first_owned)) ++first_owned;
+            const int chunk_step = shared ? share : 1;
+            bool folding =
+                v_begin <= last_contrib && first_owned < chunk_end && *abort_flag == 0;
             bool fold_ok = true;
             uint64_t *fold_bar = bars + S::kFoldBar + warp * S::kFoldSlots;
             const uint32_t fold_smem =
                 smem_base + static_cast<uint32_t>(warp * S::kFoldSlots * kFoldSlotBytes);
-            int issue_c = chunk0, issue_v = first_contrib;
+            int issue_c = first_owned, issue_v = v_begin;
             uint32_t issued = 0, waited = 0;
             auto fold_issue = [&]() {
                 if (!folding || !fold_ok || issue_c >= chunk_end) return;
@@ -893,9 +943,10 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                                   &fold_bar[slot]);
                 }
                 ++issued;
-                if (++issue_v > last_contrib) {
-                    issue_v = first_contrib;
-                    ++issue_c;
+                issue_v = next_v(issue_v);
+                if (issue_v > last_contrib) {
+                    issue_v = v_begin;
+                    issue_c += chunk_step;
                 }
             };
             if (folding) {
@@ -911,7 +962,7 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                 tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * kStoreCols), r);
                 tmem_wait_ld();
                 if (!folding) return;
-                for (int v = first_contrib; v <= last_contrib; ++v) {
+                for (int v = v_begin; v <= last_contrib; v = next_v(v)) {
                     const uint32_t slot = waited % S::kFoldSlots;
                     if (fold_ok) {
                         const int ok = mbar_wait_bounded(&fold_bar[slot],
@@ -950,7 +1001,7 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                             atomicOr(p.error_word, kErrDrain);
                 __syncwarp();
             };
-            if (role == kSegPartial) {
+            if (role == kSegPartial && !shared) {
                 // Write this warp's rows / columns of the unit's partial
                 // accumulator; once every lane's stores are fenced, flag them.
 #pragma unroll 1
@@ -1154,10 +1205,25 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
             // flight while the previous chunk is converted and stored.  (Heads
             // of a stream-K split load through the fold, one chunk at a time.)
             uint32_t ra[32], rb[32];
-            if (!folding && chunk_end > chunk0)
+            if (shared) {
+                // The chunks this unit owns, each with every unit's partial.
+#pragma unroll 1
+                for (int c = first_owned; c < chunk_end; c += share) {
+                    fetch_bias32<EPI>(p.bias, static_cast<int64_t>(nt) * BN + c * kStoreCols, p.N,
+                                      bias_vec, bias_next);
+                    if (folding) {
+                        load_acc_chunk(c, ra);
+                    } else {
+                        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * kStoreCols), ra);
+                        tmem_wait_ld_dep(ra);
+                    }
+                    emit(c, ra);
+                }
+            }
+            if (!shared && !folding && chunk_end > chunk0)
                 tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(chunk0 * kStoreCols), ra);
 #pragma unroll 1
-            for (int c = chunk0; c < chunk_end; c += 2) {
+            for (int c = chunk0; !shared && c < chunk_end; c += 2) {
                 if (folding)
                     load_acc_chunk(c, ra);
                 else

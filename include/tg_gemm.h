@@ -55,7 +55,8 @@
  *     or base address is not a multiple of 16 bytes the operands are first
  *     repacked into a padded temporary, a stream-ordered allocation on
  *     `stream` from a memory pool private to the library (freed on `stream`
- *     after the GEMM); TG_ERR_OOM if that allocation fails.
+ *     after the GEMM); TG_ERR_OOM if that allocation fails.  One repacking
+ *     kernel makes the copies before the GEMM kernel.
  *   - C must not overlap A, B or bias (TG_ERR_INVALID_ARG).
  *   - The device must be compute capability 10.0 (B200 class, sm_100a);
  *     otherwise TG_ERR_UNSUPPORTED_DEVICE.  There is no CPU fallback.
@@ -128,7 +129,9 @@ typedef enum {
  * would add a whole wave to a whole-tile launch, the tensor-core kernel
  * covers the first q * BN columns and a second kernel computes the last r
  * columns on the CUDA cores (fp32 sums of the same fp16 products, the same
- * epilogue), launched before it on `stream`.  Not for the row softmax.
+ * epilogue), launched after it on `stream` and running alongside it; the
+ * repacking gathers those r columns of B for it (into the same temporary).
+ * Not for the row softmax.
  */
 tg_status_t tg_gemm(const void *A, const void *B, const void *bias, void *C,
                     int64_t M, int64_t N, int64_t K, int epilogue, void *stream);
@@ -259,10 +262,11 @@ tg_status_t tg_gemm_host(const void *A_host, const void *B_host, const void *bia
  * tg_gemm_launch_count -- number of kernels tg_gemm would launch for these
  * arguments (host only, no device call; the configuration choice assumes
  * 148 SMs): 0 for an empty problem, 1 for the GEMM kernel (or the K == 0
- * kernel), plus one repacking kernel (it repacks both operands) when the
- * base address or row pitch of A or B is not a multiple of 16 bytes and the
- * chosen configuration loads with TMA (a table row choosing a plain-loader
- * configuration repacks nothing), plus one kernel for the last N mod 256 (at
+ * kernel), plus one repacking kernel (it repacks both operands and gathers
+ * the thin remainder's columns of B) when the base address or row pitch of A
+ * or B is not a multiple of 16 bytes and the chosen configuration loads with
+ * TMA (a table row choosing a plain-loader configuration repacks nothing) or
+ * when there is a thin remainder, plus one kernel for the last N mod 256 (at
  * most 16) columns when that thin remainder would otherwise cost the
  * tensor-core kernel a whole extra wave of tiles (see tg_gemm).  Returns -1
  * if the arguments would be rejected.
@@ -296,10 +300,13 @@ tg_status_t tg_gemm_check_error(void *stream);
  * calls no cudaMalloc, cudaFree, memory-pool or other allocating routine.
  *
  *   - The scratch a call needs is 2*M*K8 bytes (rounded up to 256) when A
- *     must be repacked plus 2*K*N8 bytes when B must be repacked (K8, N8 =
- *     K, N rounded up to a multiple of 8); aligned operands need none.  A
- *     call needing more than TG_NOALLOC_SCRATCH_BYTES returns
- *     TG_ERR_SCRATCH_LIMIT and launches nothing.
+ *     must be repacked, plus 2*K*N8 bytes (rounded up to 256) when B must be
+ *     repacked, plus 2*r*KA bytes (rounded up to 256) and 256 more for a
+ *     thin remainder of r columns (K8, N8 = K, N rounded up to a multiple of
+ *     8; KA = K8 when A is repacked, else K); aligned operands without a
+ *     remainder need none.  A call needing more than
+ *     TG_NOALLOC_SCRATCH_BYTES returns TG_ERR_SCRATCH_LIMIT and launches
+ *     nothing.
  *   - The first call on each device performs a one-time set-up on that
  *     device (it looks up the device address of the scratch array, which may
  *     load the library's GPU module); make that first call before any stream

@@ -478,24 +478,22 @@ tg_status_t launch_k0(const void *bias, void *C, int64_t M, int64_t N, int epilo
 // Thin N remainder: when N = q * BN + r with 0 < r <= kTailMaxCols and the
 // last, nearly empty column of tiles would cost the persistent GEMM a whole
 // extra wave, the GEMM covers the first q * BN columns and tail_cols_kernel
-// the last r on the CUDA cores (one pass over A, read from L2 right after the
-// repack or the GEMM's own loads).  Whole-tile TMA configurations only (the
-// tail kernel reads A with 16-byte loads), not the row softmax (it needs whole
-// rows), and only while B's r columns fit the tail kernel's shared memory.
+// the last r on the CUDA cores, alongside the GEMM.  Whole-tile TMA
+// configurations only (the tail kernel reads A with 16-byte loads), not the
+// row softmax (it needs whole rows).
 constexpr int kTailMaxCols = 16;
-constexpr int64_t kTailSmemBytes = 64 * 1024;
 
 int tail_round(int r) { return r <= 1 ? 1 : r <= 2 ? 2 : r <= 4 ? 4 : r <= 8 ? 8 : 16; }
 
 int tail_cols(const tg_config_t &ci, int64_t M, int64_t N, int64_t K, int epilogue, int split,
               int num_sms)
 {
+    (void)K;
     if (split == TG_SPLIT_STREAM_K || epilogue == TG_EPILOGUE_BIAS_SOFTMAX ||
         ci.loader != tg::kLoadTma)
         return 0;
     const int64_t r = N % ci.block_n;
     if (r == 0 || r > kTailMaxCols || N < ci.block_n) return 0;
-    if (K * tail_round(static_cast<int>(r)) * 2 > kTailSmemBytes) return 0;
     const int64_t units = ci.cta_pair ? num_sms / 2 : num_sms;
     const int64_t m_tiles = ceil_div(M, ci.block_m);
     const int64_t waves_all = ceil_div(m_tiles * ceil_div(N, ci.block_n), units);
@@ -503,33 +501,61 @@ int tail_cols(const tg_config_t &ci, int64_t M, int64_t N, int64_t K, int epilog
     return waves_main < waves_all ? static_cast<int>(r) : 0;
 }
 
-template <int EPI>
-cudaError_t launch_tail_epi(const __half *A, int64_t lda, const __half *B, int64_t ldb,
-                            const __half *bias, __half *C, int64_t ldc, int64_t M, int64_t K,
-                            int64_t n0, int r, int grid, cudaStream_t stream)
+// The tail kernel's launch: programmatic stream serialisation, so that it may
+// start while the GEMM before it runs (the GEMM allows it once its CTAs are
+// resident; the tail waits for the GEMM's completion at its end).
+struct TailArgs {
+    const __half *A, *slab;
+    int64_t ld;
+    const __half *bias;
+    __half *C;
+    int64_t ldc, M, n0;
+    int r;
+    unsigned long long *next_row;
+};
+
+template <int EPI, int RT>
+cudaError_t launch_tail_kernel(const TailArgs &t, int grid, cudaStream_t stream)
 {
-    const int rt = tail_round(r);
-    const size_t smem = static_cast<size_t>(K) * rt * 2;
-    switch (rt) {
-    case 1: tg::tail_cols_kernel<EPI, 1><<<grid, 256, smem, stream>>>(A, lda, B, ldb, bias, C, ldc, M, K, n0, r); break;
-    case 2: tg::tail_cols_kernel<EPI, 2><<<grid, 256, smem, stream>>>(A, lda, B, ldb, bias, C, ldc, M, K, n0, r); break;
-    case 4: tg::tail_cols_kernel<EPI, 4><<<grid, 256, smem, stream>>>(A, lda, B, ldb, bias, C, ldc, M, K, n0, r); break;
-    case 8: tg::tail_cols_kernel<EPI, 8><<<grid, 256, smem, stream>>>(A, lda, B, ldb, bias, C, ldc, M, K, n0, r); break;
-    default: tg::tail_cols_kernel<EPI, 16><<<grid, 256, smem, stream>>>(A, lda, B, ldb, bias, C, ldc, M, K, n0, r); break;
-    }
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(tg::kTailThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, tg::tail_cols_kernel<EPI, RT>, t.A, t.slab, t.ld, t.bias, t.C,
+                              t.ldc, t.M, t.n0, t.r, t.next_row);
 }
 
-// Opt every tail kernel into up to kTailSmemBytes of dynamic shared memory
-// (once per device).
 template <int EPI>
-cudaError_t tail_smem_attrs()
+cudaError_t launch_tail_epi(const TailArgs &t, int grid, cudaStream_t stream)
+{
+    switch (tail_round(t.r)) {
+    case 1: return launch_tail_kernel<EPI, 1>(t, grid, stream);
+    case 2: return launch_tail_kernel<EPI, 2>(t, grid, stream);
+    case 4: return launch_tail_kernel<EPI, 4>(t, grid, stream);
+    case 8: return launch_tail_kernel<EPI, 8>(t, grid, stream);
+    default: return launch_tail_kernel<EPI, 16>(t, grid, stream);
+    }
+}
+
+// The tail kernel's blocks share SMs with the GEMM's CTAs, which take nearly
+// all of the shared memory: an SM runs blocks of one shared-memory
+// configuration at a time, so the tail kernels ask for the largest carveout
+// too (once per device), else they would run only on SMs without a GEMM CTA.
+template <int EPI>
+cudaError_t tail_carveout_epi()
 {
     cudaError_t e = cudaSuccess;
     auto set = [&](auto kern) {
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(kTailSmemBytes));
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     static_cast<int>(cudaSharedmemCarveoutMaxShared));
     };
     set(tg::tail_cols_kernel<EPI, 1>);
     set(tg::tail_cols_kernel<EPI, 2>);
@@ -539,9 +565,7 @@ cudaError_t tail_smem_attrs()
     return e;
 }
 
-tg_status_t launch_tail(const void *A, int64_t lda, const void *B, int64_t ldb, const void *bias,
-                        void *C, int64_t ldc, int64_t M, int64_t K, int64_t n0, int r,
-                        int epilogue, int num_sms, cudaStream_t stream)
+tg_status_t tail_carveout()
 {
     static std::atomic<uint64_t> attr_set{0};
     int dev = 0;
@@ -550,33 +574,31 @@ tg_status_t launch_tail(const void *A, int64_t lda, const void *B, int64_t ldb, 
         return TG_ERR_CUDA;
     }
     const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
-    if (!bit || !(attr_set.load() & bit)) {
-        const cudaError_t e = tail_smem_attrs<0>() == cudaSuccess && tail_smem_attrs<1>() == cudaSuccess &&
-                                      tail_smem_attrs<2>() == cudaSuccess && tail_smem_attrs<3>() == cudaSuccess
-                                  ? cudaSuccess
-                                  : cudaErrorInvalidValue;
-        if (e != cudaSuccess) {
-            cudaGetLastError();
-            return TG_ERR_CUDA;
-        }
-        attr_set.fetch_or(bit);
+    if (bit && (attr_set.load() & bit)) return TG_OK;
+    if (tail_carveout_epi<0>() != cudaSuccess || tail_carveout_epi<1>() != cudaSuccess ||
+        tail_carveout_epi<2>() != cudaSuccess || tail_carveout_epi<3>() != cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_CUDA;
     }
-    // one row per warp at a time, and enough warps that every row's loads go
-    // out at once on moderate M
-    const int grid = static_cast<int>(std::min<int64_t>(ceil_div(M, 8), 32ll * num_sms));
-    const __half *a = static_cast<const __half *>(A);
-    const __half *b = static_cast<const __half *>(B);
-    const __half *bb = static_cast<const __half *>(bias);
-    __half *c = static_cast<__half *>(C);
+    attr_set.fetch_or(bit);
+    return TG_OK;
+}
+
+tg_status_t launch_tail(const TailArgs &t, int epilogue, int num_sms, cudaStream_t stream)
+{
+    const tg_status_t st = tail_carveout();
+    if (st != TG_OK) return st;
+    // one warp per row, up to eight two-warp blocks per SM in the grid
+    const int grid = static_cast<int>(std::min<int64_t>(ceil_div(t.M, 2), 8ll * num_sms));
     cudaError_t e;
     if (epilogue == TG_EPILOGUE_NONE)
-        e = launch_tail_epi<0>(a, lda, b, ldb, bb, c, ldc, M, K, n0, r, grid, stream);
+        e = launch_tail_epi<0>(t, grid, stream);
     else if (epilogue == TG_EPILOGUE_BIAS)
-        e = launch_tail_epi<1>(a, lda, b, ldb, bb, c, ldc, M, K, n0, r, grid, stream);
+        e = launch_tail_epi<1>(t, grid, stream);
     else if (epilogue == TG_EPILOGUE_BIAS_GELU)
-        e = launch_tail_epi<2>(a, lda, b, ldb, bb, c, ldc, M, K, n0, r, grid, stream);
+        e = launch_tail_epi<2>(t, grid, stream);
     else
-        e = launch_tail_epi<3>(a, lda, b, ldb, bb, c, ldc, M, K, n0, r, grid, stream);
+        e = launch_tail_epi<3>(t, grid, stream);
     if (e != cudaSuccess) {
         cudaGetLastError();
         return TG_ERR_LAUNCH;
@@ -598,18 +620,80 @@ tg::PackJob pack_job(const void *src, int64_t rows, int64_t cols, void *dst, int
     return j;
 }
 
-// One launch repacks both operands (either job may be empty): up to eight
-// 256-thread blocks per SM, each thread kPackGroups 16-byte groups per step.
-tg_status_t launch_pack2(const tg::PackJob &a, const tg::PackJob &b, cudaStream_t stream,
-                         int num_sms)
+// Where a GEMM's operands come from: the operands as the GEMM reads them and
+// the tail's columns and slab.
+struct Staging {
+    const void *A = nullptr, *B = nullptr;
+    int64_t lda = 0, ldb = 0;
+    int tail = 0;                      // thin remainder columns (0: none)
+    __half *slab = nullptr;            // tail: B's last columns, r rows of lda
+    unsigned long long *next_row = nullptr;   // tail: its row counter
+};
+
+// Bytes of scratch a call needs: A and B repacked (when not 16-byte
+// addressable) and the tail's slab and row counter, each part 256-byte
+// aligned.
+struct ScratchPlan {
+    size_t a_off = 0, b_off = 0, slab_off = 0, counter_off = 0, bytes = 0;
+};
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+ScratchPlan scratch_plan(bool a_direct, bool b_direct, int64_t M, int64_t N, int64_t K, int tail)
 {
-    const uint64_t total = a.groups + b.groups;
+    ScratchPlan s;
+    const int64_t lda = a_direct ? K : (K + 7) / 8 * 8;
+    const int64_t ldb = b_direct ? N : (N + 7) / 8 * 8;
+    s.a_off = 0;
+    s.b_off = s.a_off + round256(a_direct ? 0 : static_cast<size_t>(2 * M * lda));
+    s.slab_off = s.b_off + round256(b_direct ? 0 : static_cast<size_t>(2 * K * ldb));
+    s.counter_off = s.slab_off + round256(static_cast<size_t>(2 * tail * lda));
+    s.bytes = s.counter_off + (tail > 0 ? 256 : 0);
+    return s;
+}
+
+// The repacking pre-pass: one launch makes every copy a call needs (the
+// repacked operands and the tail's slab) before the GEMM: up to eight
+// 256-thread blocks per SM, each thread kPackGroups 16-byte groups per step.
+tg_status_t launch_pack(const tg::PackJob &a, const tg::PackJob &b, const tg::SlabJob &sl,
+                        int num_sms, cudaStream_t stream)
+{
+    const uint64_t total = a.groups + b.groups + sl.groups;
     if (total == 0) return TG_OK;
     const uint64_t per_block = 256ull * tg::kPackGroups;
     const int grid = static_cast<int>(std::min<uint64_t>((total + per_block - 1) / per_block,
                                                          8ull * static_cast<uint64_t>(num_sms)));
-    tg::pack_pad2_kernel<<<grid, 256, 0, stream>>>(a, b);
+    tg::pack_pad2_kernel<<<grid, 256, 0, stream>>>(a, b, sl);
     return cudaGetLastError() == cudaSuccess ? TG_OK : TG_ERR_LAUNCH;
+}
+
+// Fills in where the GEMM reads its operands and launches the repacking
+// pre-pass a call needs (repacked operands and the tail's slab, in `scratch`
+// as `plan` lays them out), if any.
+tg_status_t stage_operands(const void *A, const void *B, int64_t M, int64_t N, int64_t K,
+                           bool a_direct, bool b_direct, const ScratchPlan &plan,
+                           unsigned char *scratch, int num_sms, cudaStream_t stream, Staging *sg)
+{
+    sg->lda = a_direct ? K : (K + 7) / 8 * 8;
+    sg->ldb = b_direct ? N : (N + 7) / 8 * 8;
+    sg->A = a_direct ? A : scratch + plan.a_off;
+    sg->B = b_direct ? B : scratch + plan.b_off;
+    sg->slab = sg->tail > 0 ? reinterpret_cast<__half *>(scratch + plan.slab_off) : nullptr;
+    sg->next_row = sg->tail > 0 ? reinterpret_cast<unsigned long long *>(scratch + plan.counter_off)
+                                : nullptr;
+    if (plan.bytes == 0) return TG_OK;
+    const tg::PackJob ja = pack_job(a_direct ? nullptr : A, M, K, scratch + plan.a_off, sg->lda);
+    const tg::PackJob jb = pack_job(b_direct ? nullptr : B, K, N, scratch + plan.b_off, sg->ldb);
+    tg::SlabJob js;
+    js.src = static_cast<const __half *>(B);
+    js.dst = sg->slab;
+    js.ldb = N;
+    js.n0 = N - sg->tail;
+    js.K = K;
+    js.ld_slab = sg->lda;
+    js.groups = static_cast<uint64_t>(sg->tail) * static_cast<uint64_t>(sg->lda / 8);
+    js.next_row = sg->next_row;
+    return launch_pack(ja, jb, js, num_sms, stream);
 }
 
 // Tensor maps, kernel parameters, work division and launch of the GEMM on
@@ -618,22 +702,19 @@ tg_status_t launch_pack2(const tg::PackJob &a, const tg::PackJob &b, cudaStream_
 // pitch).  Shared by tg_gemm and tg_gemm_noalloc, which differ only in where
 // repacked operands live.  `split` is TG_SPLIT_TILES or TG_SPLIT_STREAM_K;
 // stream-K takes the (device, stream) workspace.
-tg_status_t launch_staged(const KernelConfig &cfg, const void *Aeff, int64_t lda, const void *Beff,
-                          int64_t ldb, const void *bias, void *C, int64_t M, int64_t N, int64_t K,
-                          int epilogue, int split, const tg_options_t *opts, int num_sms,
-                          unsigned *error_word, cudaStream_t stream)
+tg_status_t launch_staged(const KernelConfig &cfg, const Staging &sg, const void *bias, void *C,
+                          int64_t M, int64_t N, int64_t K, int epilogue, int split,
+                          const tg_options_t *opts, int num_sms, unsigned *error_word,
+                          cudaStream_t stream)
 {
+    const void *Aeff = sg.A, *Beff = sg.B;
+    const int64_t lda = sg.lda, ldb = sg.ldb;
     const bool plain = cfg.info.loader == tg::kLoadPlain;
     const bool c_rows16 = aligned(C, 16) && (N % 8 == 0);
     const int store = c_rows16 ? cfg.store_pref : tg::kStoreScalar;
     // The GEMM covers columns [0, n_main); a thin remainder goes to the tail kernel.
-    const int tail = tail_cols(cfg.info, M, N, K, epilogue, split, num_sms);
+    const int tail = sg.tail;
     const int64_t n_main = N - tail;
-    if (tail > 0) {
-        const tg_status_t st = launch_tail(Aeff, lda, Beff, ldb, bias, C, N, M, K, n_main, tail,
-                                           epilogue, num_sms, stream);
-        if (st != TG_OK) return st;
-    }
     CUtensorMap ta, tb, tc;
     std::memset(&ta, 0, sizeof(ta));
     std::memset(&tb, 0, sizeof(tb));
@@ -666,6 +747,7 @@ tg_status_t launch_staged(const KernelConfig &cfg, const void *Aeff, int64_t lda
     p.bias_vec = (bias && aligned(bias, 16)) ? 1 : 0;
     p.wait_limit_ns = (opts && opts->wait_limit_ns) ? opts->wait_limit_ns : kDefaultWaitLimitNs;
     p.error_word = error_word;
+    p.early_trigger = tail > 0 ? 1 : 0;
     // Persistent grid: one CTA (or CTA pair) per SM (pair of SMs).  Whole
     // tiles: never more units than tiles; stream-K: streamk_units.
     const int units = cfg.info.cta_pair ? num_sms / 2 : num_sms;
@@ -703,6 +785,20 @@ tg_status_t launch_staged(const KernelConfig &cfg, const void *Aeff, int64_t lda
         cudaGetLastError();
         return TG_ERR_LAUNCH;
     }
+    if (tail > 0) {
+        TailArgs t;
+        t.A = static_cast<const __half *>(Aeff);
+        t.slab = sg.slab;
+        t.ld = lda;
+        t.bias = static_cast<const __half *>(bias);
+        t.C = static_cast<__half *>(C);
+        t.ldc = N;
+        t.M = M;
+        t.n0 = n_main;
+        t.r = tail;
+        t.next_row = sg.next_row;
+        return launch_tail(t, epilogue, num_sms, stream);
+    }
     return TG_OK;
 }
 
@@ -734,6 +830,7 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
         choice = {opts->config_id, rule_split(opts->config_id, M, N, K, epilogue, dev->num_sms)};
     else
         choice = choose_config(M, N, K, epilogue, dev->num_sms);
+    if (opts && opts->split != TG_SPLIT_AUTO) choice.split = opts->split;
     // Stream-K flags hold a per-call epoch, which a replayed graph would
     // repeat: whole tiles while the stream is capturing.
     if (tg_internal_capturing(stream)) {
@@ -747,37 +844,26 @@ tg_status_t gemm_impl(const void *A, const void *B, const void *bias, void *C, i
     const bool plain = cfg.info.loader == tg::kLoadPlain;
     const bool a_direct = plain || a_aligned;
     const bool b_direct = plain || b_aligned;
-    const int64_t lda = a_direct ? K : (K + 7) / 8 * 8;
-    const int64_t ldb = b_direct ? N : (N + 7) / 8 * 8;
+    Staging sg;
+    sg.tail = tail_cols(cfg.info, M, N, K, epilogue, choice.split, dev->num_sms);
+    const ScratchPlan plan = scratch_plan(a_direct, b_direct, M, N, K, sg.tail);
     void *tmp = nullptr;
-    const void *Aeff = A, *Beff = B;
-    if (!a_direct || !b_direct) {
-        const size_t a_bytes = a_direct ? 0 : static_cast<size_t>(2 * M * lda);
-        const size_t a_pad = (a_bytes + 255) / 256 * 256;
-        const size_t b_bytes = b_direct ? 0 : static_cast<size_t>(2 * K * ldb);
-        if (cudaMallocFromPoolAsync(&tmp, a_pad + b_bytes, dev->pool, stream) != cudaSuccess) {
+    if (plan.bytes > 0) {
+        if (cudaMallocFromPoolAsync(&tmp, plan.bytes, dev->pool, stream) != cudaSuccess) {
             cudaGetLastError();
             return TG_ERR_OOM;
         }
-        void *bdst = static_cast<char *>(tmp) + a_pad;
-        if (!a_direct) Aeff = tmp;
-        if (!b_direct) Beff = bdst;
-        st = launch_pack2(pack_job(a_direct ? nullptr : A, M, K, tmp, lda),
-                          pack_job(b_direct ? nullptr : B, K, N, bdst, ldb), stream, dev->num_sms);
-        if (st != TG_OK) {
-            cudaFreeAsync(tmp, stream);
-            return st;
-        }
+        st = stage_operands(A, B, M, N, K, a_direct, b_direct, plan,
+                            static_cast<unsigned char *>(tmp), dev->num_sms, stream, &sg);
+    } else {
+        st = stage_operands(A, B, M, N, K, true, true, plan, nullptr, dev->num_sms, stream, &sg);
     }
-
-    st = launch_staged(cfg, Aeff, lda, Beff, ldb, bias, C, M, N, K, epilogue,
-                       (opts && opts->split != TG_SPLIT_AUTO) ? opts->split : choice.split, opts,
-                       dev->num_sms, dev->error_word, stream);
+    if (st == TG_OK)
+        st = launch_staged(cfg, sg, bias, C, M, N, K, epilogue, choice.split, opts, dev->num_sms,
+                           dev->error_word, stream);
     if (tmp) cudaFreeAsync(tmp, stream);
     return st;
 }
-
-size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 // The end-to-end entry point overlaps its copies with the GEMM: B (and the
 // bias) go up first, then A in row panels on an internal copy-in stream;
@@ -989,13 +1075,14 @@ int tg_gemm_launch_count(const void *A, const void *B, const void *bias, const v
     if (validate(A, B, bias, C, M, N, K, epilogue) != TG_OK) return -1;
     if (M == 0 || N == 0) return 0;
     if (K == 0) return 1;
-    const bool a_direct = aligned(A, 16) && (K % 8 == 0);
-    const bool b_direct = aligned(B, 16) && (N % 8 == 0);
     const Choice c = choose_config(M, N, K, epilogue, 148);
     const tg_config_t &ci = kConfigs[c.config].info;
     if (ci.loader == tg::kLoadPlain) return 1;
-    return 1 + ((a_direct && b_direct) ? 0 : 1) +
-           (tail_cols(ci, M, N, K, epilogue, c.split, 148) > 0 ? 1 : 0);
+    const bool a_direct = aligned(A, 16) && (K % 8 == 0);
+    const bool b_direct = aligned(B, 16) && (N % 8 == 0);
+    const int tail = tail_cols(ci, M, N, K, epilogue, c.split, 148);
+    // the GEMM, one repacking pass (operands or the tail's slab), the tail
+    return 1 + ((a_direct && b_direct && tail == 0) ? 0 : 1) + (tail > 0 ? 1 : 0);
 }
 
 tg_status_t tg_gemm_check_error(void *stream)
@@ -1112,12 +1199,12 @@ tg_status_t gemm_noalloc_impl(const void *A, const void *B, const void *bias, vo
     // Scratch needed by the repacking step, checked before any device call.
     const bool a_direct = aligned(A, 16) && (K % 8 == 0);
     const bool b_direct = aligned(B, 16) && (N % 8 == 0);
-    const int64_t lda = a_direct ? K : (K + 7) / 8 * 8;
-    const int64_t ldb = b_direct ? N : (N + 7) / 8 * 8;
-    const size_t a_bytes = (a_direct || K == 0) ? 0 : static_cast<size_t>(2 * M * lda);
-    const size_t a_pad = (a_bytes + 255) / 256 * 256;
-    const size_t b_bytes = (b_direct || K == 0) ? 0 : static_cast<size_t>(2 * K * ldb);
-    if (a_pad + b_bytes > static_cast<size_t>(TG_NOALLOC_SCRATCH_BYTES)) return TG_ERR_SCRATCH_LIMIT;
+    const Choice choice = K == 0 ? Choice{0, TG_SPLIT_TILES} : choose_config(M, N, K, epilogue, 148, false);
+    const int tail = K == 0 ? 0 : tail_cols(kConfigs[choice.config].info, M, N, K, epilogue,
+                                            TG_SPLIT_TILES, 148);
+    if (K > 0 && scratch_plan(a_direct, b_direct, M, N, K, tail).bytes >
+                     static_cast<size_t>(TG_NOALLOC_SCRATCH_BYTES))
+        return TG_ERR_SCRATCH_LIMIT;
 
     NoallocDevice *dev = nullptr;
     st = noalloc_device(&dev);
@@ -1128,16 +1215,16 @@ tg_status_t gemm_noalloc_impl(const void *A, const void *B, const void *bias, vo
     const int cfg_id =
         choose_config(M, N, K, epilogue, dev->num_sms, false).config;
     const KernelConfig &cfg = kConfigs[cfg_id];
-    const void *Aeff = a_direct ? A : dev->scratch;
-    const void *Beff = b_direct ? B : dev->scratch + a_pad;
-    st = launch_pack2(pack_job(a_direct ? nullptr : A, M, K, dev->scratch, lda),
-                      pack_job(b_direct ? nullptr : B, K, N, dev->scratch + a_pad, ldb), stream,
-                      dev->num_sms);
-    if (st != TG_OK) return st;
-
     // stream-K needs a workspace; this entry point allocates nothing
-    return launch_staged(cfg, Aeff, lda, Beff, ldb, bias, C, M, N, K, epilogue, TG_SPLIT_TILES,
-                         nullptr, dev->num_sms, dev->error_word, stream);
+    Staging sg;
+    sg.tail = tail_cols(cfg.info, M, N, K, epilogue, TG_SPLIT_TILES, dev->num_sms);
+    const ScratchPlan plan = scratch_plan(a_direct, b_direct, M, N, K, sg.tail);
+    if (plan.bytes > static_cast<size_t>(TG_NOALLOC_SCRATCH_BYTES)) return TG_ERR_SCRATCH_LIMIT;
+    st = stage_operands(A, B, M, N, K, a_direct, b_direct, plan, dev->scratch, dev->num_sms,
+                        stream, &sg);
+    if (st != TG_OK) return st;
+    return launch_staged(cfg, sg, bias, C, M, N, K, epilogue, TG_SPLIT_TILES, nullptr,
+                         dev->num_sms, dev->error_word, stream);
 }
 
 }  // namespace

@@ -188,8 +188,9 @@ def test_valid_call_without_a_device_reports_unsupported_device():
 
 def test_launch_count_is_host_only():
     """One GEMM kernel, plus one repacking kernel for both operands when
-    either row pitch or base is not a multiple of 16 bytes, plus the thin
-    N-remainder kernel when it saves the GEMM a wave."""
+    either row pitch or base is not a multiple of 16 bytes (it also gathers the
+    thin remainder's columns of B), plus the thin N-remainder kernel when it
+    saves the GEMM a wave."""
     f = binding.tg_gemm_launch_count
     assert f(0x1000, 0x100000, None, 0x1000000, 256, 256, 256, NONE) == 1
     assert f(0x1000, 0x100000, None, 0x1000000, 256, 256, 250, NONE) == 2   # K % 8

@@ -39,12 +39,12 @@ def _run(entry, a, b, bias, M, N, K, epilogue):
 
 
 def _scratch_needed(M, N, K):
-    """Bytes of repacking scratch a call with 16-byte aligned bases needs, as
-    the header states it: 2*M*K8 rounded up to 256 when K % 8 != 0, plus
-    2*K*N8 when N % 8 != 0."""
+    """Bytes of repacking scratch a call with 16-byte aligned bases and no
+    thin N remainder needs, as the header states it: 2*M*K8 rounded up to 256
+    when K % 8 != 0, plus 2*K*N8 rounded up to 256 when N % 8 != 0."""
     k8, n8 = -(-K // 8) * 8, -(-N // 8) * 8
     a = 0 if K % 8 == 0 else -(-(2 * M * k8) // 256) * 256
-    b = 0 if N % 8 == 0 else 2 * K * n8
+    b = 0 if N % 8 == 0 else -(-(2 * K * n8) // 256) * 256
     return a + b
 
 

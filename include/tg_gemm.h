@@ -54,9 +54,12 @@
  *     Any 2-byte-aligned address and any K, N are accepted: when a row pitch
  *     or base address is not a multiple of 16 bytes the operands are first
  *     repacked into a padded temporary, a stream-ordered allocation on
- *     `stream` from a memory pool private to the library (freed on `stream`
- *     after the GEMM); TG_ERR_OOM if that allocation fails.  One repacking
- *     kernel makes the copies before the GEMM kernel.
+ *     `stream` from a memory pool private to the library; TG_ERR_OOM if that
+ *     allocation fails.  Up to 64 MiB of it is kept for the next call on the
+ *     same stream (and grown, stream-ordered, when a call needs more); a
+ *     larger temporary, or one made while `stream` is capturing a graph, is
+ *     freed on `stream` after the GEMM.  One repacking kernel makes the
+ *     copies before the GEMM kernel.
  *   - C must not overlap A, B or bias (TG_ERR_INVALID_ARG).
  *   - The device must be compute capability 10.0 (B200 class, sm_100a);
  *     otherwise TG_ERR_UNSUPPORTED_DEVICE.  There is no CPU fallback.

@@ -1,7 +1,7 @@
 """Operands that TMA cannot address (a row pitch or base that is not a
 multiple of 16 bytes) are repacked by one kernel before the GEMM, which also
 gathers B's last columns for the thin N-remainder kernel; that kernel runs
-alongside the GEMM, launched after it.  tg_gemm (pool scratch) and
+alongside the GEMM, launched after it.  tg_gemm (scratch kept per stream) and
 tg_gemm_noalloc (the fixed scratch array) take the same steps and must give
 the same C, bit for bit; on integer inputs C is exact.  The same calls
 captured in a CUDA graph replay correctly on new inputs.
@@ -119,3 +119,38 @@ def test_graph_capture_replays_on_new_inputs(M, N, K):
         _check(torch.cuda.current_stream().cuda_stream)
         assert np.array_equal(c.cpu().double().numpy(), run_oracle(A2, B2, bias2, BIAS)), seed
     del g
+
+
+def test_kept_scratch_grows_and_is_reused_in_stream_order():
+    # calls in a row on one stream, without synchronising: the scratch kept
+    # for the stream grows for the second call and is reused by the third
+    dev = torch.device("cuda:0")
+    stream = torch.cuda.current_stream().cuda_stream
+    shapes = [(300, 777, 130), (3000, 1537, 2050), (500, 333, 514), (3000, 1537, 2050)]
+    runs = []
+    for i, (M, N, K) in enumerate(shapes):
+        A, B, bias = wl.integer_inputs(M, N, K, seed=650 + i, bias=True)
+        c = torch.empty(M, N, dtype=torch.float16, device=dev)
+        _call(binding.tg_gemm, A.to(dev), B.to(dev), bias.to(dev), c, M, N, K, BIAS, stream)
+        runs.append((A, B, bias, c))
+    _check(stream)
+    for A, B, bias, c in runs:
+        assert np.array_equal(c.cpu().double().numpy(), run_oracle(A, B, bias, BIAS))
+
+
+def test_two_streams_keep_separate_scratch():
+    M, N, K = 1000, 777, 1030
+    dev = torch.device("cuda:0")
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    ins = [wl.integer_inputs(M, N, K, seed=660 + i, bias=True) for i in range(2)]
+    dins = [(A.to(dev), B.to(dev), bias.to(dev)) for A, B, bias in ins]
+    torch.cuda.synchronize()
+    outs = [torch.empty(M, N, dtype=torch.float16, device=dev) for _ in range(2)]
+    for _ in range(3):
+        for s, (a, b, bb), c in zip((s1, s2), dins, outs):
+            _call(binding.tg_gemm, a, b, bb, c, M, N, K, BIAS, s.cuda_stream)
+    torch.cuda.synchronize()
+    for s in (s1, s2):
+        assert binding.tg_gemm_check_error(s.cuda_stream) == binding.TG_OK
+    for (A, B, bias), c in zip(ins, outs):
+        assert np.array_equal(c.cpu().double().numpy(), run_oracle(A, B, bias, BIAS))

@@ -23,7 +23,7 @@
 
 #include "tg_gemm.h"
 #include "tg_internal.h"
-#include "tg_kernels.cuh"
+#include "tg_aux.cuh"
 
 // Per-device error word: bounded-wait expiries are OR-ed in here.
 __device__ unsigned g_tg_error_word;

@@ -258,17 +258,18 @@ def test_unaligned_c_rows_bit_exact(config_id, off_c):
     assert bool((guard == -7.0).all()), "wrote outside C"
 
 
-TAIL_CASES = [((3000, 1537, 2050), 1, NONE), ((2048, 2307, 64), 0, BIAS), ((3000, 1552, 130), 1, BIAS),
-              ((1100, 2051, 96), 0, NONE)]
+TAIL_CASES = [((3000, 1537, 2050), 1, NONE), ((2048, 2306, 64), 0, BIAS), ((3000, 1552, 130), 1, BIAS),
+              ((2048, 2307, 64), 0, NONE), ((1100, 2051, 96), 0, NONE)]
 
 
 @pytest.mark.parametrize("shape,config_id,epi", TAIL_CASES,
                          ids=["x".join(map(str, c[0])) for c in TAIL_CASES])
 def test_thin_n_remainder_bit_exact(shape, config_id, epi):
-    """N = q * 256 + r with r <= 16, where the last column of 256-wide tiles
-    would add a wave: the GEMM covers q * 256 columns and the CUDA-core tail
-    kernel the last r (r = 1, 3, 16; and a shape that keeps the extra wave
-    and no tail).  Integer-valued inputs make the exact result an fp16 value."""
+    """N = q * 256 + r where the last column of 256-wide tiles would add a
+    wave: for r <= 2 the GEMM covers q * 256 columns and the CUDA-core tail
+    kernel the last r (r = 1, 2); wider remainders (r = 3, 16) and a shape
+    whose extra column of tiles fits the wave keep whole tiles.  Integer-valued
+    inputs make the exact result an fp16 value."""
     M, N, K = shape
     A, B, bias = wl.integer_inputs(M, N, K, seed=480 + N, lo=-1, hi=1, bias=True)
     exp = oracle.gemm_int_exact(wl.to_bits(A), wl.to_bits(B),

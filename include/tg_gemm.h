@@ -127,7 +127,7 @@ typedef enum {
  * a per-call epoch, which every replay of the graph would repeat.  Such calls
  * run whole tiles (an explicit TG_SPLIT_STREAM_K returns TG_ERR_INVALID_ARG).
  *
- * Thin N remainder: when N = q * BN + r with 0 < r <= 2 (BN the tile width
+ * Thin N remainder: when N = q * BN + r with 0 < r <= 4 (BN the tile width
  * of the chosen configuration) and the last, nearly empty column of tiles
  * would add a whole wave to a whole-tile launch, the tensor-core kernel
  * covers the first q * BN columns and a second kernel computes the last r
@@ -270,7 +270,7 @@ tg_status_t tg_gemm_host(const void *A_host, const void *B_host, const void *bia
  * or B is not a multiple of 16 bytes and the chosen configuration loads with
  * TMA (a table row choosing a plain-loader configuration repacks nothing) or
  * when there is a thin remainder, plus one kernel for the last N mod 256 (at
- * most 2) columns when that thin remainder would otherwise cost the
+ * most 4) columns when that thin remainder would otherwise cost the
  * tensor-core kernel a whole extra wave of tiles (see tg_gemm).  Returns -1
  * if the arguments would be rejected.
  */

@@ -482,12 +482,13 @@ tg_status_t launch_k0(const void *bias, void *C, int64_t M, int64_t N, int epilo
 // configurations only (the tail kernel reads A with 16-byte loads), not the
 // row softmax (it needs whole rows).  Measured on 3000 x (1536 + r) x 2048
 // (bias + GELU, cold L2): the tail path takes 42.0, 42.1, 48.3, 56.7 and
-// 80.9 us for r = 1, 2, 4, 8, 16, while the extra wave of whole tiles takes
-// 36.5-38.7 us on aligned N (plus a repack of B and element stores of C on
-// unaligned N), so only r <= 2 goes to the tail.
-constexpr int kTailMaxCols = 2;
+// 80.9 us for r = 1, 2, 4, 8, 16; the extra wave of whole tiles 50.3 us for
+// r = 4 (B repacked, C stored element by element) and 36.9-37.7 us for the
+// aligned r = 8, 16.  So r <= 4 goes to the tail (N is then not a multiple
+// of 8).
+constexpr int kTailMaxCols = 4;
 
-int tail_round(int r) { return r <= 1 ? 1 : 2; }
+int tail_round(int r) { return r <= 1 ? 1 : r <= 2 ? 2 : 4; }
 
 int tail_cols(const tg_config_t &ci, int64_t M, int64_t N, int64_t K, int epilogue, int split,
               int num_sms)
@@ -539,8 +540,11 @@ cudaError_t launch_tail_kernel(const TailArgs &t, int grid, cudaStream_t stream)
 template <int EPI>
 cudaError_t launch_tail_epi(const TailArgs &t, int grid, cudaStream_t stream)
 {
-    return tail_round(t.r) == 1 ? launch_tail_kernel<EPI, 1>(t, grid, stream)
-                                : launch_tail_kernel<EPI, 2>(t, grid, stream);
+    switch (tail_round(t.r)) {
+    case 1: return launch_tail_kernel<EPI, 1>(t, grid, stream);
+    case 2: return launch_tail_kernel<EPI, 2>(t, grid, stream);
+    default: return launch_tail_kernel<EPI, 4>(t, grid, stream);
+    }
 }
 
 // The tail kernel's blocks share SMs with the GEMM's CTAs, which take nearly
@@ -558,6 +562,7 @@ cudaError_t tail_carveout_epi()
     };
     set(tg::tail_cols_kernel<EPI, 1>);
     set(tg::tail_cols_kernel<EPI, 2>);
+    set(tg::tail_cols_kernel<EPI, 4>);
     return e;
 }
 

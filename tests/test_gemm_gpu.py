@@ -266,8 +266,8 @@ TAIL_CASES = [((3000, 1537, 2050), 1, NONE), ((2048, 2306, 64), 0, BIAS), ((3000
                          ids=["x".join(map(str, c[0])) for c in TAIL_CASES])
 def test_thin_n_remainder_bit_exact(shape, config_id, epi):
     """N = q * 256 + r where the last column of 256-wide tiles would add a
-    wave: for r <= 2 the GEMM covers q * 256 columns and the CUDA-core tail
-    kernel the last r (r = 1, 2); wider remainders (r = 3, 16) and a shape
+    wave: for r <= 4 the GEMM covers q * 256 columns and the CUDA-core tail
+    kernel the last r (r = 1, 2, 3); a wider remainder (r = 16) and a shape
     whose extra column of tiles fits the wave keep whole tiles.  Integer-valued
     inputs make the exact result an fp16 value."""
     M, N, K = shape

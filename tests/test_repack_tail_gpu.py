@@ -46,6 +46,7 @@ def _check(stream):
     (640, 256, 390, NONE, 3),      # A alone repacked
     (700, 333, 512, BIAS, 4),      # B alone repacked
     (2048, 2306, 64, NONE, 5),     # two thin columns (the tail kernel's RT = 2 form)
+    (2048, 2307, 64, BIAS, 7),     # three thin columns (RT = 4)
     (3000, 1544, 2048, NONE, 6),   # aligned, 8 columns past 1536: whole tiles, nothing repacked
 ])
 def test_tg_gemm_and_noalloc_agree_bit_exact(M, N, K, epi, seed):

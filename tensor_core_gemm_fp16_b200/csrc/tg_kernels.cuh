@@ -457,8 +457,9 @@ __device__ __forceinline__ void unpack_bias8(const uint4 &u, float (&b)[8])
 }
 
 // Eight fp32 accumulators + bias -> epilogue -> eight fp16 packed in a uint4.
-// For the row softmax, sm_max / sm_scale are the row's maximum and
-// 1 / sum(exp(v - max)).
+// For the row softmax, r holds exp(v - m_c) already (written back by the
+// statistics pass, m_c the running maximum when that chunk was read) and
+// sm_scale is the chunk's exp(m_c - max) / sum(exp(v - max)); sm_max is unused.
 template <int EPI>
 __device__ __forceinline__ uint4 epilogue8(const uint32_t *r, const float (&b)[8],
                                            float sm_max = 0.f, float sm_scale = 0.f)
@@ -474,9 +475,8 @@ __device__ __forceinline__ uint4 epilogue8(const uint32_t *r, const float (&b)[8
             f2_unpack(v, lo, hi);
             gelu_erf2(lo, hi);
         } else if constexpr (EPI == kEpiBiasSoftmax) {
-            lo = exp2_approx((__uint_as_float(r[2 * e]) + b[2 * e] - sm_max) * kLog2e) * sm_scale;
-            hi = exp2_approx((__uint_as_float(r[2 * e + 1]) + b[2 * e + 1] - sm_max) * kLog2e) *
-                 sm_scale;
+            lo = __uint_as_float(r[2 * e]) * sm_scale;
+            hi = __uint_as_float(r[2 * e + 1]) * sm_scale;
         } else {
             lo = apply_epilogue<EPI>(__uint_as_float(r[2 * e]), b[2 * e]);
             hi = apply_epilogue<EPI>(__uint_as_float(r[2 * e + 1]), b[2 * e + 1]);
@@ -1039,8 +1039,13 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
             // of exp(v - max) over the valid columns, kept as a running pair: a
             // chunk raising the maximum from m to m' rescales the sum by
             // exp(m - m').  Two chunks are read per TMEM wait, and each chunk's
-            // maximum and sum are taken over eight independent partials.
+            // maximum and sum are taken over eight independent partials.  The
+            // chunk's exponentials go back into TMEM in place of its accumulator,
+            // with the maximum they were taken against (chunk_shift, in log2
+            // units), so that the output pass multiplies instead of exponentiating
+            // again.
             float sm_max = 0.f, sm_scale = 0.f;
+            float chunk_shift[S::kChunksPerWarp];
             if constexpr (EPI == kEpiBiasSoftmax) {
                 static_assert(EPI_WARPS == 4, "the softmax epilogue needs whole rows per thread");
                 // The statistics pass and the output pass both read the
@@ -1056,7 +1061,8 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                     folding = false;
                 }
                 float run_max = -INFINITY, run_sum = 0.f;
-                auto stats_chunk = [&](const uint32_t (&r)[32], const uint4 (&bq)[4], int64_t col0) {
+                auto stats_chunk = [&](const uint32_t (&r)[32], const uint4 (&bq)[4], int64_t col0,
+                                       int ci, uint32_t taddr) {
                     float v[32];
                     const bool full = col0 + kStoreCols <= p.N;
 #pragma unroll
@@ -1081,9 +1087,15 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                     float sp[8];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) sp[j] = 0.f;
+                    uint32_t ex[32];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        sp[e & 7] += exp2_approx(fmaf(v[e], kLog2e, -shift));
+                    for (int e = 0; e < 32; ++e) {
+                        const float x = exp2_approx(fmaf(v[e], kLog2e, -shift));
+                        ex[e] = __float_as_uint(x);
+                        sp[e & 7] += x;
+                    }
+                    tmem_st_32x32b_x32(taddr, ex);
+                    chunk_shift[ci] = shift;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) sp[j] += sp[j + 4];
                     const float csum = (sp[0] + sp[1]) + (sp[2] + sp[3]);
@@ -1103,9 +1115,13 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                     if (two) fetch_bias32<EPI>(p.bias, col0 + kStoreCols, p.N, bias_vec, bb);
                     tmem_wait_ld_dep(ra);
                     if (two) tmem_wait_ld_dep(rb);
-                    stats_chunk(ra, ba, col0);
-                    if (two) stats_chunk(rb, bb, col0 + kStoreCols);
+                    stats_chunk(ra, ba, col0, c - chunk0,
+                                t_row + static_cast<uint32_t>(c * kStoreCols));
+                    if (two)
+                        stats_chunk(rb, bb, col0 + kStoreCols, c + 1 - chunk0,
+                                    t_row + static_cast<uint32_t>((c + 1) * kStoreCols));
                 }
+                tmem_wait_st();
                 sm_max = run_max;
                 sm_scale = rcp_approx(run_sum);
             }
@@ -1118,6 +1134,11 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
             // fetched here.
             auto emit = [&](int c, const uint32_t (&r)[32]) {
                 const int64_t col0 = static_cast<int64_t>(nt) * BN + c * kStoreCols;
+                // row softmax: this chunk's factor exp(m_c - max) / sum
+                float chunk_scale = 0.f;
+                if constexpr (EPI == kEpiBiasSoftmax)
+                    chunk_scale =
+                        exp2_approx(fmaf(sm_max, -kLog2e, chunk_shift[c - chunk0])) * sm_scale;
                 uint4 bias_cur[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) bias_cur[q] = bias_next[q];
@@ -1130,7 +1151,7 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                         for (int q = 0; q < 4; ++q) {
                             float b[8];
                             unpack_bias8(bias_cur[q], b);
-                            const uint4 u = epilogue8<EPI>(r + q * 8, b, sm_max, sm_scale);
+                            const uint4 u = epilogue8<EPI>(r + q * 8, b, sm_max, chunk_scale);
                             if (full) {
                                 *reinterpret_cast<uint4 *>(crow + col0 + q * 8) = u;
                             } else {
@@ -1164,7 +1185,7 @@ __global__ void __launch_bounds__(KernelShape<BN, BK, STAGES, PAIR, EPI_WARPS, S
                 for (int q = 0; q < 4; ++q) {
                     float b[8];
                     unpack_bias8(bias_cur[q], b);
-                    const uint4 u = epilogue8<EPI>(r + q * 8, b, sm_max, sm_scale);
+                    const uint4 u = epilogue8<EPI>(r + q * 8, b, sm_max, chunk_scale);
                     const uint32_t phys = static_cast<uint32_t>(q) ^ ((lane >> 1) & 3u);
                     const uint32_t addr = buf + lane * 64u + phys * 16u;
                     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
